@@ -58,12 +58,13 @@ static uint16_t f32_to_bf16_rne(float f) {
   return (uint16_t)(u >> 16);
 }
 
-/* A table is 8 fp32 magnitudes.  Accepted: all finite, all >= 0, max > 0
- * (the pack rule divides the block amax by the largest level). */
+/* A table is 8 fp32 magnitudes.  Accepted: all finite, none with the sign
+ * bit set (a magnitude is >= 0; -0.0 is not a magnitude), max > 0 (the pack
+ * rule divides the block amax by the largest level). */
 static int table_ok(const float* t) {
   float mx = 0.0f;
   for (int i = 0; i < 8; ++i) {
-    if (!isfinite(t[i]) || t[i] < 0.0f) return 0;
+    if (!isfinite(t[i]) || signbit(t[i])) return 0;
     if (t[i] > mx) mx = t[i];
   }
   return mx > 0.0f;

@@ -114,6 +114,10 @@ def test_dequant_rejects_bad_arguments():
     neg[0, 0] = -0.5
     with pytest.raises(oracle.OracleError):
         oracle.dequant(w, s, neg, np.zeros(1, np.uint8), 1, 1, 32)
+    negz = grid.copy()
+    negz[0, 0] = -0.0
+    with pytest.raises(oracle.OracleError):
+        oracle.dequant(w, s, negz, np.zeros(1, np.uint8), 1, 1, 32)
 
 
 def test_wrong_table_decode_is_large_error():
