@@ -1,0 +1,428 @@
+"""Benchmark of the routed-expert MoE layer over 4-bit codebook weights.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload decode_t1|decode_t8|decode_t64|prefill_t2048|prefill_t8192]
+
+One step = one pass of the whole layer (route -> gate/up + SwiGLU -> down ->
+combine) over one batch of synthetic GLM-5.2-shaped input (hidden 6144,
+intermediate 2048, 256 experts, top-8; 4-bit Lloyd codebook + E8M0/32
+weights).  The default workload is decode at T=1.  Inputs rotate over 8
+seeded batches resident in HBM; L2 is flushed (a 256 MiB write) before every
+timed step, outside the step's own CUDA events.  Prints one JSON line (rank 0).
+
+--impl reference times the fp64 CPU oracle on the host cores on the same
+workload, each step a bounded sample (one expert's contribution for one
+token, over a slice of the intermediate channels, on every thread).
+
+N > 1: independent replicas, one per GPU (the layer is single-GPU); the
+device time is the max over ranks; value = tokens of all ranks / that time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from bit_codebook_quantized_router_b200 import inputs  # noqa: E402
+
+METRIC = "MoE layer tokens/s"
+UNIT = "tokens/s"
+FLUSH_BYTES = 256 << 20
+ROTATE = 8
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+def workload_desc(w: inputs.Workload) -> dict:
+    sh = w.shape
+    d = {"workload": f"{w.name}: GLM-5.2-shaped routed-expert MoE layer, T={w.T}, H={sh.H}, I={sh.I}, "
+                     f"E={sh.E}, top-{sh.k}, 4-bit Lloyd-codebook codes + E8M0 scale per 32",
+         "T": w.T, "H": sh.H, "I": sh.I, "E": sh.E, "top_k": sh.k,
+         "routing": "zipf-skewed" if w.zipf else "uniform random",
+         "tables": "lloyd + e2m1 (5 experts)" if w.mixed_tables else "lloyd",
+         "inputs": f"{ROTATE} rotating seeded batches, resident in HBM",
+         "l2": "flushed (256 MiB write) before every timed step, outside its events"}
+    return d
+
+
+def expert_bytes(sh: inputs.Shape) -> tuple[int, int]:
+    """(gate+up bytes, down bytes) of one expert: codes + E8M0 scales."""
+    gu = 2 * sh.I * (sh.H // 2 + sh.H // 32)
+    dn = sh.H * (sh.I // 2 + sh.I // 32)
+    return gu, dn
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", FALLBACK_HBM_GBS), d.get("bf16_tflops", FALLBACK_BF16_TFLOPS), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def source_digest(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel_key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f).get(kernel_key)
+    if not d:
+        return None
+    if d.get("source_digest") != source_digest(d.get("sources", [])):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.index, self.period = index, period_s
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            return self
+        names = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                 "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                    r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                    for n, bit in names.items():
+                        if r & bit:
+                            self.reasons.add(n)
+                except Exception:
+                    pass
+                time.sleep(self.period)
+
+        self._t = threading.Thread(target=run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+        return False
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": len(self.samples)}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (the reference arm and the cpu_baseline of our arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample_layer(w, x_bits, lg, tokens, device):
+    """Oracle layer with the experts the sampled tokens route to, packed by the
+    oracle itself from the same bf16 weights (setup, not timed)."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    ids, wts = oracle.route(lg[tokens], w.shape.k)
+    experts = sorted(set(ids.reshape(-1).tolist()))
+    tables, tid = inputs.layer_tables(w)
+    sh = w.shape
+    L = oracle.Layer(sh.E, sh.H, sh.I, tables, tid)
+
+    def job(e_blobs):
+        e, blobs = e_blobs
+        out = []
+        for proj in inputs.PROJECTIONS:
+            N, K = inputs.proj_shape(sh, proj)
+            c, s = oracle.pack(blobs[proj][None], tables, tid[e:e + 1], 1, N, K)
+            out += [c[0], s[0]]
+        return e, out
+
+    jobs = [(e, {p: inputs.bf16_bits(inputs.expert_weight(w, e, p, device=device)) for p in inputs.PROJECTIONS})
+            for e in experts]
+    with ThreadPoolExecutor(max_workers=os.cpu_count()) as ex:
+        for e, parts in ex.map(job, jobs):
+            L.set_expert(e, *parts)
+    return L, ids, wts
+
+
+def time_oracle_units(L, x_bits, units, threads):
+    """Run oracle units (token, slot, i0, i1) on `threads` threads; wall time."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda u: oracle.expert_partial(L, u[1], x_bits[u[0]], u[2], u[3]), units))
+    return time.perf_counter() - t0
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    sh = w.shape
+    x_bits = inputs.bf16_bits(inputs.activations(w))
+    lg = inputs.router_logits(w).numpy()
+    threads = max(1, os.cpu_count() or 1)
+    tokens = list(range(min(w.T, 4)))
+    L, ids, wts = oracle_sample_layer(w, x_bits, lg, tokens, "cpu")
+    # calibrate one unit (one token, one expert, I/8 channels) to size a step
+    t_cal = time_oracle_units(L, x_bits, [(0, int(ids[0, 0]), 0, sh.I // 8)], 1) * 8
+    budget = 150.0
+    q = 1
+    while q < sh.I // 32 and (args.steps + args.warmup) * t_cal / q > budget:
+        q *= 2
+    chunk = sh.I // q
+
+    def step_units(s):
+        # `threads` units per step, walking (token, slot, chunk) in order
+        out = []
+        for u in range(threads):
+            n = s * threads + u
+            t = tokens[(n // (sh.k * q)) % len(tokens)]
+            j = (n // q) % sh.k
+            c = n % q
+            out.append((t, int(ids[tokens.index(t), j]), c * chunk, (c + 1) * chunk))
+        return out
+
+    for s in range(args.warmup):
+        time_oracle_units(L, x_bits, step_units(s), threads)
+    times = [time_oracle_units(L, x_bits, step_units(args.warmup + s), threads) for s in range(args.steps)]
+    tokens_per_step = threads / (sh.k * q)
+    total = sum(times)
+    value = tokens_per_step * args.steps / total
+    sample = (f"each step: {threads} units of one token x one routed expert x {chunk} of {sh.I} intermediate "
+              f"channels ({tokens_per_step:.4g} token-equivalents), fp64 oracle, {len(tokens)} sampled tokens")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_desc(w),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(w, x_bits, lg):
+    """The oracle on this host: 2 tokens x all routed experts, full channels."""
+    import oracle
+    oracle.build()
+    sh = w.shape
+    tokens = [0, 1] if w.T > 1 else [0]
+    L, ids, _ = oracle_sample_layer(w, x_bits, lg, tokens, "cuda")
+    units = [(t, int(ids[i, j]), 0, sh.I) for i, t in enumerate(tokens) for j in range(sh.k)]
+    threads = min(len(units), os.cpu_count() or 1)
+    dt = time_oracle_units(L, x_bits, units, threads)
+    return {"value": len(tokens) / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{len(tokens)} token(s) x {sh.k} routed experts, full layer arithmetic in fp64, "
+                      f"one (token, expert) per thread"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def build_device_layer(w):
+    import bit_codebook_quantized_router_b200 as q4
+    sh = w.shape
+    tables, tid = inputs.layer_tables(w)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    parts = {}
+    for proj in inputs.PROJECTIONS:
+        N, K = inputs.proj_shape(sh, proj)
+        big = torch.empty((sh.E, N, K), dtype=torch.bfloat16, device="cuda")
+        for e in range(sh.E):
+            big[e] = inputs.expert_weight(w, e, proj, device="cuda")
+        parts[proj] = q4.pack(big, tables, tid, status=status)
+        del big
+    torch.cuda.empty_cache()
+    assert q4.lib().moe_q4_read_status(q4._lib._ptr(status), q4._lib._stream()) == 0
+    return q4.Layer(*parts["gate"], *parts["up"], *parts["down"], tables, tid)
+
+
+def run_ours(args, w):
+    import torch.distributed as dist
+
+    import bit_codebook_quantized_router_b200 as q4
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    sh = w.shape
+    T, k = w.T, sh.k
+    layer = build_device_layer(w)
+    xs = [inputs.activations(w, device="cuda", variant=v) for v in range(ROTATE)]
+    lgs = [inputs.router_logits(w, device="cuda", variant=v) for v in range(ROTATE)]
+    # distinct experts touched per batch (for the algorithmic bytes)
+    touched = []
+    for lg in lgs:
+        ids = torch.topk(lg, k, dim=1).indices
+        touched.append(int(torch.unique(ids).numel()))
+    ws = q4.alloc_workspace(q4.forward_workspace(layer, T, k))
+    out = torch.empty((T, sh.H), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for i in range(args.warmup):
+        q4.forward(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)
+    torch.cuda.synchronize()
+    assert q4.forward_status(ws) == 0
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)
+            starts[i].record(stream)
+            q4.forward(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    total_ms = float(tmax.item())
+    value = T * args.steps * world / (total_ms / 1e3)
+
+    # stage times (separate pass, events between the kernels)
+    n_prof = min(args.steps, 100)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_prof)]
+    for i in range(n_prof):
+        flush.fill_(i & 0xFF)
+        q4.forward_stages(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out, ws, evs[i])
+    torch.cuda.synchronize()
+    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(n_prof)])
+    stage_mean = stage_ms.mean(0)
+    assert q4.forward_status(ws) == 0
+
+    # e2e through the host-buffer entry point (pinned host memory)
+    n_e2e = min(args.steps, 200)
+    xh = [x.cpu().pin_memory() for x in xs]
+    lh = [l.cpu().pin_memory() for l in lgs]
+    oh = torch.empty((T, sh.H), dtype=torch.bfloat16).pin_memory()
+    wsh = q4.alloc_workspace(q4.forward_host_workspace(layer, T, k))
+    for i in range(3):
+        q4.forward_host(layer, xh[i % ROTATE], lh[i % ROTATE], k, oh, wsh)
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e)]
+    torch.cuda.synchronize()
+    for i in range(n_e2e):
+        flush.fill_(i & 0xFF)
+        e_s[i].record(stream)
+        st = q4.forward_host(layer, xh[i % ROTATE], lh[i % ROTATE], k, oh, wsh)
+        e_e[i].record(stream)
+        assert st == 0
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))
+    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
+    e2e_value = T * n_e2e * world / (float(e2e_t.item()) / 1e3)
+
+    # roofline of the dominant kernel (gate/up + SwiGLU: the largest byte stream)
+    hbm_peak, tf_peak, peak_src = load_peaks()
+    gu, dn = expert_bytes(sh)
+    mean_touched = float(np.mean(touched))
+    R = T * k
+    gu_bytes = mean_touched * gu + T * sh.H * 2 + R * sh.I * 2 * 2
+    gu_ms = float(stage_mean[1])
+    achieved = gu_bytes / (gu_ms / 1e3) / 1e9
+    layer_bytes = mean_touched * (gu + dn) + T * sh.H * 2 * 2
+    kernels_per_step = (1 if T <= 256 else 2) + 3
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_desc(w), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+        "roofline": {"kernel": "decode gate/up + SwiGLU (packed 4-bit stream, mma.sync)", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                     "peak_source": peak_src, "traffic": profile_traffic("decode_gateup"),
+                     "algorithmic_bytes_per_launch": gu_bytes, "launch_ms": gu_ms},
+        "stages_ms": {"route": float(stage_mean[0]), "gate_up": float(stage_mean[1]),
+                      "down": float(stage_mean[2]), "combine": float(stage_mean[3])},
+        "layer_hbm": {"touched_experts": mean_touched, "bytes_per_step": layer_bytes,
+                      "gbs": layer_bytes / (total_ms / args.steps / 1e3) / 1e9,
+                      "frac_of_peak": layer_bytes / (total_ms / args.steps / 1e3) / 1e9 / hbm_peak,
+                      "frac_of_8tbs": layer_bytes / (total_ms / args.steps / 1e3) / 8e12},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * sh.H * 2 + T * sh.E * 4,
+                "d2h_bytes_per_step": T * sh.H * 2},
+        "gpu_launches": kernels_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inputs.bf16_bits(xs[0]), lgs[0].cpu().numpy())
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode_t1", choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    w = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

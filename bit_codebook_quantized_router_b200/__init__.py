@@ -1,0 +1,14 @@
+"""B200-native routed-expert MoE feed-forward over 4-bit codebook weights.
+
+The compute lives in ``libmoe_q4.so`` (hand-written sm_100a CUDA kernels
+behind a C ABI, declared in ``include/moe_q4.h``); this package is a thin
+binding.  Importing it does not load the library; the first call does, and
+raises if the library was not built (there is no CPU fallback).
+"""
+from ._lib import (Layer, MoeQ4Error, alloc_workspace, dequant, forward, forward_host,
+                   forward_host_workspace, forward_stages, forward_status, forward_workspace, lib, pack, route,
+                   status_string)
+
+__all__ = ["Layer", "MoeQ4Error", "alloc_workspace", "dequant", "forward", "forward_host",
+           "forward_host_workspace", "forward_stages", "forward_status", "forward_workspace", "lib", "pack",
+           "route", "status_string"]

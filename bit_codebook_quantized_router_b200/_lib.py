@@ -1,0 +1,229 @@
+"""ctypes binding of libmoe_q4 (argument marshalling only: every step of the
+layer runs in the library's CUDA kernels).  Torch provides device memory and
+streams; tensors are passed as raw pointers."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe_q4.so")
+
+OK, EINVAL, ECUDA, EWORKSPACE, ETIMEOUT, EDEVICE, ENOTSUP = range(7)
+MAX_TABLES, MAX_EXPERTS, MAX_TOPK = 16, 512, 16
+
+
+class MoeQ4Error(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: moe_q4 status {status} ({status_string(status)})")
+
+
+class _LayerStruct(ctypes.Structure):
+    _fields_ = [
+        ("E", ctypes.c_int), ("H", ctypes.c_int), ("I", ctypes.c_int),
+        ("gate_w", ctypes.c_void_p), ("gate_s", ctypes.c_void_p),
+        ("up_w", ctypes.c_void_p), ("up_s", ctypes.c_void_p),
+        ("down_w", ctypes.c_void_p), ("down_s", ctypes.c_void_p),
+        ("tables", ctypes.c_void_p), ("n_tables", ctypes.c_int), ("table_id", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded library.  Raises if it was not built: there is no fallback."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m bit_codebook_quantized_router_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, ci, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        L.moe_q4_abi_version.restype = ci
+        L.moe_q4_status_string.argtypes = [ci]
+        L.moe_q4_status_string.restype = ctypes.c_char_p
+        L.moe_q4_pack.argtypes = [vp, ci, ci, ci, vp, ci, vp, vp, vp, vp, vp]
+        L.moe_q4_dequant.argtypes = [vp, vp, vp, ci, vp, ci, ci, ci, vp, vp]
+        L.moe_q4_forward_workspace.argtypes = [ctypes.POINTER(_LayerStruct), ci, ci]
+        L.moe_q4_forward_workspace.restype = sz
+        L.moe_q4_forward_host_workspace.argtypes = [ctypes.POINTER(_LayerStruct), ci, ci]
+        L.moe_q4_forward_host_workspace.restype = sz
+        L.moe_q4_forward.argtypes = [ctypes.POINTER(_LayerStruct), vp, vp, ci, ci, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_q4_forward_host.argtypes = [ctypes.POINTER(_LayerStruct), vp, vp, ci, ci, vp, vp, sz, vp]
+        L.moe_q4_forward_status.argtypes = [vp, vp]
+        L.moe_q4_read_status.argtypes = [vp, vp]
+        L.moe_q4_route_workspace.argtypes = [ci, ci, ci]
+        L.moe_q4_route_workspace.restype = sz
+        L.moe_q4_route.argtypes = [vp, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_q4_forward_stages.argtypes = [ctypes.POINTER(_LayerStruct), vp, vp, ci, ci, vp, vp, sz, vp,
+                                            ctypes.POINTER(ctypes.c_void_p), ci]
+        for f in (L.moe_q4_pack, L.moe_q4_dequant, L.moe_q4_forward, L.moe_q4_forward_host,
+                  L.moe_q4_forward_status, L.moe_q4_read_status, L.moe_q4_route,
+                  L.moe_q4_forward_stages):
+            f.restype = ci
+        if L.moe_q4_abi_version() != 1:
+            raise ImportError("libmoe_q4 ABI version mismatch")
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().moe_q4_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc, what):
+    if rc != OK:
+        raise MoeQ4Error(rc, what)
+
+
+def _host_tables(tables, table_id, E):
+    t = np.ascontiguousarray(np.asarray(tables, np.float32).reshape(-1, 8))
+    tid = np.ascontiguousarray(np.asarray(table_id, np.uint8).reshape(-1))
+    if tid.shape[0] != E:
+        raise ValueError("table_id must hold one entry per expert")
+    return t, tid
+
+
+class Layer:
+    """A packed layer resident on the device.
+
+    gate_w/up_w: uint8 [E, I, H/2], gate_s/up_s: uint8 [E, I, H/32],
+    down_w: uint8 [E, H, I/2], down_s: uint8 [E, H, I/32] (CUDA tensors);
+    tables: fp32 [n, 8] magnitudes; table_id: uint8 [E] (host arrays)."""
+
+    def __init__(self, gate_w, gate_s, up_w, up_s, down_w, down_s, tables, table_id):
+        self.E, self.I, hh = gate_w.shape
+        self.H = hh * 2
+        self.gate_w, self.gate_s, self.up_w, self.up_s = gate_w, gate_s, up_w, up_s
+        self.down_w, self.down_s = down_w, down_s
+        self.tables, self.table_id = _host_tables(tables, table_id, self.E)
+        for t in (gate_w, gate_s, up_w, up_s, down_w, down_s):
+            if not (t.is_cuda and t.dtype == torch.uint8 and t.is_contiguous()):
+                raise ValueError("packed tensors must be contiguous uint8 CUDA tensors")
+
+    def struct(self) -> _LayerStruct:
+        return _LayerStruct(self.E, self.H, self.I,
+                            self.gate_w.data_ptr(), self.gate_s.data_ptr(),
+                            self.up_w.data_ptr(), self.up_s.data_ptr(),
+                            self.down_w.data_ptr(), self.down_s.data_ptr(),
+                            self.tables.ctypes.data, self.tables.shape[0], self.table_id.ctypes.data)
+
+
+def pack(w: torch.Tensor, tables, table_id, status: torch.Tensor | None = None, stream=None):
+    """bf16 [E, N, K] CUDA tensor -> (codes uint8 [E, N, K/2], scales uint8 [E, N, K/32])."""
+    if w.dim() != 3 or w.dtype != torch.bfloat16 or not w.is_cuda:
+        raise ValueError("w must be a bf16 CUDA tensor [E, N, K]")
+    w = w.contiguous()
+    E, N, K = w.shape
+    t, tid = _host_tables(tables, table_id, E)
+    codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=w.device)
+    scales = torch.empty((E, N, K // 32), dtype=torch.uint8, device=w.device)
+    own = status is None
+    if own:
+        status = torch.zeros(1, dtype=torch.int32, device=w.device)
+    _check(lib().moe_q4_pack(_ptr(w), E, N, K, t.ctypes.data, t.shape[0], tid.ctypes.data,
+                             _ptr(codes), _ptr(scales), _ptr(status), _stream(stream)), "moe_q4_pack")
+    if own:
+        st = lib().moe_q4_read_status(_ptr(status), _stream(stream))
+        _check(st, "moe_q4_pack (device)")
+    return codes, scales
+
+
+def dequant(codes: torch.Tensor, scales: torch.Tensor, tables, table_id, stream=None) -> torch.Tensor:
+    """uint8 codes [E, N, K/2] + scales [E, N, K/32] -> bf16 [E, N, K]."""
+    E, N, Kh = codes.shape
+    K = Kh * 2
+    t, tid = _host_tables(tables, table_id, E)
+    out = torch.empty((E, N, K), dtype=torch.bfloat16, device=codes.device)
+    _check(lib().moe_q4_dequant(_ptr(codes.contiguous()), _ptr(scales.contiguous()), t.ctypes.data,
+                                t.shape[0], tid.ctypes.data, E, N, K, _ptr(out), _stream(stream)),
+           "moe_q4_dequant")
+    return out
+
+
+def forward_workspace(layer: Layer, T: int, k: int) -> int:
+    return int(lib().moe_q4_forward_workspace(ctypes.byref(layer.struct()), T, k))
+
+
+def forward_host_workspace(layer: Layer, T: int, k: int) -> int:
+    return int(lib().moe_q4_forward_host_workspace(ctypes.byref(layer.struct()), T, k))
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def forward(layer: Layer, x: torch.Tensor, logits: torch.Tensor, k: int, out=None, ws=None,
+            topk_ids=None, topk_w=None, counts=None, out_f32=None, stream=None) -> torch.Tensor:
+    """One MoE layer: x bf16 [T, H], logits fp32 [T, E] -> out bf16 [T, H]
+    (and, when given, the fp32 combine result in out_f32 [T, H])."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, layer.H), dtype=torch.bfloat16, device=x.device)
+    if ws is None:
+        ws = alloc_workspace(forward_workspace(layer, T, k), x.device)
+    st = layer.struct()
+    _check(lib().moe_q4_forward(ctypes.byref(st), _ptr(x), _ptr(logits), T, k, _ptr(out),
+                                _ptr(out_f32), _ptr(topk_ids), _ptr(topk_w), _ptr(counts), _ptr(ws), ws.numel(),
+                                _stream(stream)), "moe_q4_forward")
+    return out
+
+
+def forward_status(ws: torch.Tensor, stream=None) -> int:
+    return int(lib().moe_q4_forward_status(_ptr(ws), _stream(stream)))
+
+
+def forward_host(layer: Layer, x_host: torch.Tensor, logits_host: torch.Tensor, k: int,
+                 out_host: torch.Tensor, ws: torch.Tensor, stream=None) -> int:
+    """Host tensors in and out (pinned memory for asynchronous copies)."""
+    T = x_host.shape[0]
+    st = layer.struct()
+    return int(lib().moe_q4_forward_host(ctypes.byref(st), _ptr(x_host), _ptr(logits_host), T, k,
+                                         _ptr(out_host), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def route(logits: torch.Tensor, k: int, stream=None):
+    """Routing + grouping alone: (ids, w, counts, offsets, row_token, inv)."""
+    T, E = logits.shape
+    dev = logits.device
+    ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    w = torch.empty((T, k), dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    row_token = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty((T, k), dtype=torch.int32, device=dev)
+    need = int(lib().moe_q4_route_workspace(E, T, k))
+    if need == 0:
+        raise MoeQ4Error(EINVAL, "moe_q4_route_workspace")
+    ws = alloc_workspace(need, dev)
+    _check(lib().moe_q4_route(_ptr(logits.contiguous()), T, E, k, _ptr(ids), _ptr(w), _ptr(counts),
+                              _ptr(offsets), _ptr(row_token), _ptr(inv), _ptr(ws), ws.numel(),
+                              _stream(stream)), "moe_q4_route")
+    st = forward_status(ws, stream)
+    return ids, w, counts, offsets, row_token, inv, st
+
+
+def forward_stages(layer: Layer, x, logits, k: int, out, ws, events, stream=None) -> None:
+    """moe_q4_forward with torch.cuda.Event records at the 5 stage boundaries."""
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    st = layer.struct()
+    _check(lib().moe_q4_forward_stages(ctypes.byref(st), _ptr(x), _ptr(logits), x.shape[0], k, _ptr(out),
+                                       _ptr(ws), ws.numel(), _stream(stream), arr, len(events)),
+           "moe_q4_forward_stages")

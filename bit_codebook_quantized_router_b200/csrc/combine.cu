@@ -1,0 +1,55 @@
+// Weighted combine of the routed experts' outputs back into token order:
+//   out[t] = sum_{j=0..k-1} w[t][j] * y[inv[t][j]]
+// ("GLM-5.2 EXL3 TR3 v4" README, "Shared residual rotations, private
+// intermediate rotations": expert outputs are routing-weighted and summed
+// back into the residual space).  Each output element is summed by one
+// thread in slot order in fp32, then rounded to bf16: deterministic, no
+// atomics.
+#include "q4_api_internal.h"
+#include "q4_common.cuh"
+
+namespace q4 {
+
+__global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ FwdArgs a) {
+  pdl_wait();
+  pdl_trigger();
+  const int n4 = (blockIdx.x * 256 + threadIdx.x) * 4;
+  if (n4 >= a.H) return;
+  for (int t = blockIdx.y; t < a.T; t += gridDim.y) {
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < a.k; ++j) {
+    const int r = a.inv[t * a.k + j];
+    const float wj = a.w[t * a.k + j];
+    const float4 v = *reinterpret_cast<const float4*>(a.y + (size_t)r * a.H + n4);
+    acc.x = fmaf(wj, v.x, acc.x);
+    acc.y = fmaf(wj, v.y, acc.y);
+    acc.z = fmaf(wj, v.z, acc.z);
+    acc.w = fmaf(wj, v.w, acc.w);
+  }
+  if (a.out_f32) *reinterpret_cast<float4*>(a.out_f32 + (size_t)t * a.H + n4) = acc;
+  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+  uint2 pk;
+  pk.x = *reinterpret_cast<uint32_t*>(&lo);
+  pk.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(a.out + (size_t)t * a.H + n4) = pk;
+  }
+}
+
+}  // namespace q4
+
+using namespace q4;
+
+int q4_launch_combine(const FwdArgs& a, cudaStream_t s) {
+  if (a.T == 0) return MOE_Q4_OK;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((a.H / 4 + 255) / 256, a.T < 65535 ? a.T : 65535);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, a) == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
+}

@@ -1,0 +1,51 @@
+// Host/device interface between the moe_q4 C-ABI layer and its kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe_q4.h"
+
+namespace q4 {
+struct TableParams;
+
+// Everything a forward kernel needs, passed by value.  Workspace arrays are
+// carved by q4_carve_workspace(); see the layout there.
+struct FwdArgs {
+  int T, k, E, H, I;
+  int dec_max;     // experts with 1..dec_max rows take the streaming path
+  int tile_n;      // token tile of the tensor-core path
+  const __nv_bfloat16* x;  // [T][H]
+  const float* logits;     // [T][E]
+  __nv_bfloat16* out;      // [T][H]
+  int32_t* hdr;            // header words (HeaderWord)
+  int32_t* ids;            // [T*k]
+  float* w;                // [T*k]
+  int32_t* counts;         // [E]
+  int32_t* offsets;        // [E+1]
+  int32_t* row_token;      // [T*k]
+  int32_t* inv;            // [T*k]
+  int32_t* dec_list;       // [E]
+  int32_t* pre_list;       // [E]
+  int32_t* tiles;          // [max_tiles][2] (expert, first row)
+  __nv_bfloat16* h;        // [T*k][I] bf16 rounding of silu(g)*u
+  __nv_bfloat16* h_lo;     // [T*k][I] bf16 rounding of the remainder silu(g)*u - h
+  float* y;                // [T*k][H]
+  float* out_f32;          // optional [T][H] fp32 combine result
+  __nv_bfloat16* xg;       // [T*k][H] expert-grouped activations (tensor-core path)
+  int32_t* user_ids;
+  float* user_w;
+  int32_t* user_counts;
+  const uint8_t *gate_w, *gate_s, *up_w, *up_s, *down_w, *down_s;
+};
+}  // namespace q4
+
+// Validate host tables / table ids and fill the kernel parameter block.
+int q4_fill_tables(q4::TableParams* tp, const float* tables, int n_tables, const uint8_t* table_id,
+                   int E);
+
+// Kernel launchers (return MOE_Q4_OK or MOE_Q4_ECUDA).
+int q4_launch_route(const q4::FwdArgs& a, cudaStream_t s);
+int q4_launch_decode(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, cudaStream_t s);
+int q4_launch_combine(const q4::FwdArgs& a, cudaStream_t s);

@@ -1,0 +1,315 @@
+// Router top-k + softmax-over-k, and the grouping of (token, slot) rows by
+// expert (counts, exclusive-scan offsets, stable token order, inverse map,
+// per-path expert lists).
+//
+// Geometry: "Round 7 -- Rewrite the GLM-5.2 routed-expert encoder", "Ground
+// truth and corrections" (256 routed experts, top-8).  Rows per expert form
+// the "route blocks" of "GLM-5.2 EXL3 TR3 v4" README, "Tuning: prefill route
+// block size".  The pages give no router formula; the reading implemented:
+// top-k by logit (equal logits -> lower expert id), softmax over the k kept.
+#include <math.h>
+
+#include "q4_api_internal.h"
+#include "q4_common.cuh"
+
+namespace q4 {
+
+constexpr int kRouteThreads = 1024;
+constexpr int kRouteWarps = kRouteThreads / 32;
+constexpr int kFusedMaxT = 256;  // above this, top-k runs on many CTAs first
+constexpr int kMaxLogitsPerLane = kMaxExperts / 32;
+
+// One warp routes one token: lane l holds logits of experts l, l+32, ...
+// Each of the k rounds takes the best remaining (value, then lower id) by a
+// warp argmax; lane j ends up holding slot j.  Non-finite logits are
+// recorded as a device error and treated as -inf.
+__device__ __forceinline__ void topk_warp(const float* __restrict__ row, int E, int k, int lane,
+                                          int32_t* status, int& my_id, float& my_w) {
+  float v[kMaxLogitsPerLane];
+  uint32_t avail = 0;
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < kMaxLogitsPerLane; ++i) {
+    const int id = lane + 32 * i;
+    v[i] = -INFINITY;
+    if (id < E) {
+      float x = row[id];
+      if (!isfinite(x)) {
+        bad = true;
+        x = -INFINITY;
+      }
+      v[i] = x;
+      avail |= 1u << i;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(status, MOE_Q4_EDEVICE);
+  float mine = -INFINITY;
+  my_id = -1;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = -1;
+#pragma unroll
+    for (int i = 0; i < kMaxLogitsPerLane; ++i)
+      if (((avail >> i) & 1u) && (bi < 0 || v[i] > bv)) {
+        bv = v[i];
+        bi = i;
+      }
+    int bid = bi < 0 ? 0x7fffffff : lane + 32 * bi;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
+      if (ov > bv || (ov == bv && oid < bid)) {
+        bv = ov;
+        bid = oid;
+      }
+    }
+    if ((bid & 31) == lane) avail &= ~(1u << (bid >> 5));
+    if (lane == j) {
+      my_id = bid;
+      mine = bv;
+    }
+  }
+  const float m = __shfl_sync(0xffffffffu, mine, 0);
+  float ex = (lane < k) ? expf(mine - m) : 0.0f;
+  float sum = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  my_w = ex / sum;
+}
+
+__device__ __forceinline__ void store_route(const FwdArgs& a, int t, int lane, int id, float w) {
+  if (lane < a.k) {
+    const int r = t * a.k + lane;
+    a.ids[r] = id;
+    a.w[r] = w;
+    if (a.user_ids) a.user_ids[r] = id;
+    if (a.user_w) a.user_w[r] = w;
+  }
+}
+
+// Block-wide exclusive scan of one value per thread (kRouteThreads threads).
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int o = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += o;
+  }
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int wv = warp_tot[lane];
+    int winc = wv;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int o = __shfl_up_sync(0xffffffffu, winc, off);
+      if (lane >= off) winc += o;
+    }
+    warp_tot[lane] = winc - wv;  // exclusive prefix of warp totals
+    if (lane == 31) warp_tot[32] = winc;
+  }
+  __syncthreads();
+  const int res = warp_tot[warp] + inc - v;
+  total = warp_tot[32];
+  __syncthreads();
+  return res;
+}
+
+// Grouping by one CTA of kRouteThreads threads, ids already in a.ids.
+// Shared memory: counts[E] | offs[E+1] | running[E] | mask[32][E] | pre[32][E].
+__device__ void group_rows(const FwdArgs& a, int* sm) {
+  const int E = a.E, T = a.T, k = a.k;
+  int* counts = sm;
+  int* offs = counts + E;
+  int* running = offs + E + 1;
+  int* mask = running + E;
+  int* pre = mask + kRouteWarps * E;
+  __shared__ int warp_tot[33];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int e = tid; e < E; e += kRouteThreads) {
+    counts[e] = 0;
+    running[e] = 0;
+  }
+  __syncthreads();
+  // ids come from topk_warp and are always < E; a value out of range would be
+  // a library bug: record it and leave the row out rather than index past smem.
+  for (int r = tid; r < T * k; r += kRouteThreads) {
+    const int e = a.ids[r];
+    if ((unsigned)e < (unsigned)E)
+      atomicAdd(&counts[e], 1);
+    else
+      record_error(a.hdr + kStatus, MOE_Q4_EDEVICE);
+  }
+  __syncthreads();
+  // offsets and per-path expert lists (E <= kRouteThreads)
+  const int c = tid < E ? counts[tid] : 0;
+  int total;
+  const int off = block_exclusive_scan(c, warp_tot, total);
+  const bool fd = c > 0 && c <= a.dec_max, fp = c > a.dec_max;
+  int nd, np;
+  const int pd = block_exclusive_scan(fd ? 1 : 0, warp_tot, nd);
+  const int pp = block_exclusive_scan(fp ? 1 : 0, warp_tot, np);
+  if (tid < E) {
+    offs[tid] = off;
+    a.offsets[tid] = off;
+    a.counts[tid] = c;
+    if (a.user_counts) a.user_counts[tid] = c;
+    if (fd) a.dec_list[pd] = tid;
+    if (fp) a.pre_list[pp] = tid;
+  }
+  if (tid == 0) {
+    offs[E] = total;
+    a.offsets[E] = total;
+    a.hdr[kNumDecode] = nd;
+    a.hdr[kNumPrefill] = np;
+  }
+  __syncthreads();
+  // stable placement, kRouteThreads tokens per round
+  for (int base = 0; base < T; base += kRouteThreads) {
+    for (int i = tid; i < kRouteWarps * E; i += kRouteThreads) mask[i] = 0;
+    __syncthreads();
+    const int t = base + tid;
+    if (t < T)
+      for (int j = 0; j < k; ++j) {
+        const int e = a.ids[t * k + j];
+        if ((unsigned)e < (unsigned)E) atomicOr(&mask[warp * E + e], 1 << lane);
+      }
+    __syncthreads();
+    for (int e = tid; e < E; e += kRouteThreads) {
+      int acc = running[e];
+      for (int w2 = 0; w2 < kRouteWarps; ++w2) {
+        pre[w2 * E + e] = acc;
+        acc += __popc(mask[w2 * E + e]);
+      }
+      running[e] = acc;
+    }
+    __syncthreads();
+    if (t < T) {
+      const uint32_t below = (1u << lane) - 1u;
+      for (int j = 0; j < k; ++j) {
+        const int e = a.ids[t * k + j];
+        if ((unsigned)e >= (unsigned)E) continue;
+        const int pos = offs[e] + pre[warp * E + e] + __popc(mask[warp * E + e] & below);
+        a.row_token[pos] = t;
+        a.inv[t * k + j] = pos;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// Small T: one CTA routes every token and groups.
+__global__ void __launch_bounds__(kRouteThreads) route_fused_kernel(const __grid_constant__ FwdArgs a) {
+  extern __shared__ int sm[];
+  pdl_wait();
+  if (threadIdx.x == 0) a.hdr[kStatus] = MOE_Q4_OK;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int t = warp; t < a.T; t += kRouteWarps) {
+    int id;
+    float w;
+    topk_warp(a.logits + (size_t)t * a.E, a.E, a.k, lane, a.hdr + kStatus, id, w);
+    store_route(a, t, lane, id, w);
+  }
+  __syncthreads();
+  group_rows(a, sm);
+  pdl_trigger();
+}
+
+// Large T: top-k on many CTAs (one warp per token; the host clears the
+// status word before this launch) ...
+__global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__ FwdArgs a) {
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t < a.T) {
+    int id;
+    float w;
+    topk_warp(a.logits + (size_t)t * a.E, a.E, a.k, lane, a.hdr + kStatus, id, w);
+    store_route(a, t, lane, id, w);
+  }
+  pdl_trigger();
+}
+
+// ... then one CTA groups.
+__global__ void __launch_bounds__(kRouteThreads) route_group_kernel(const __grid_constant__ FwdArgs a) {
+  extern __shared__ int sm[];
+  pdl_wait();
+  group_rows(a, sm);
+  pdl_trigger();
+}
+
+// Gather the activation rows in expert-grouped order for the tensor-core
+// path: xg[row] = x[row_token[row]] (rows of experts on that path only).
+__global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant__ FwdArgs a) {
+  pdl_wait();
+  const int np = a.hdr[kNumPrefill];
+  const int vec_per_row = a.H / 8;  // 16-byte vectors
+  for (int p = blockIdx.y; p < np; p += gridDim.y) {
+    const int e = a.pre_list[p];
+    const int r0 = a.offsets[e], r1 = a.offsets[e + 1];
+    for (int64_t v = blockIdx.x * 256 + threadIdx.x; v < (int64_t)(r1 - r0) * vec_per_row;
+         v += (int64_t)gridDim.x * 256) {
+      const int r = r0 + (int)(v / vec_per_row);
+      const int q = (int)(v % vec_per_row);
+      const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)a.row_token[r] * a.H) + q;
+      reinterpret_cast<uint4*>(a.xg + (size_t)r * a.H)[q] = *src;
+    }
+  }
+  pdl_trigger();
+}
+
+}  // namespace q4
+
+using namespace q4;
+
+static size_t group_smem_bytes(int E) { return sizeof(int) * ((size_t)3 * E + 1 + (size_t)2 * kRouteWarps * E); }
+
+int q4_launch_route(const FwdArgs& a, cudaStream_t s) {
+  const size_t smem = group_smem_bytes(a.E);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (a.T <= kFusedMaxT) {
+    if (cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return MOE_Q4_ECUDA;
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kRouteThreads);
+    cfg.dynamicSmemBytes = smem;
+    if (cudaLaunchKernelEx(&cfg, route_fused_kernel, a) != cudaSuccess) return MOE_Q4_ECUDA;
+  } else {
+    if (cudaFuncSetAttribute(route_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return MOE_Q4_ECUDA;
+    if (cudaMemsetAsync(a.hdr + kStatus, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_Q4_ECUDA;
+    cfg.gridDim = dim3((a.T + 7) / 8);
+    cfg.blockDim = dim3(256);
+    cfg.dynamicSmemBytes = 0;
+    if (cudaLaunchKernelEx(&cfg, route_topk_kernel, a) != cudaSuccess) return MOE_Q4_ECUDA;
+    cfg.gridDim = dim3(1);
+    cfg.blockDim = dim3(kRouteThreads);
+    cfg.dynamicSmemBytes = smem;
+    if (cudaLaunchKernelEx(&cfg, route_group_kernel, a) != cudaSuccess) return MOE_Q4_ECUDA;
+  }
+  return MOE_Q4_OK;
+}
+
+int q4_launch_gather(const FwdArgs& a, cudaStream_t s) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cfg.gridDim = dim3(64, 64);
+  cfg.blockDim = dim3(256);
+  return cudaLaunchKernelEx(&cfg, gather_rows_kernel, a) == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
+}

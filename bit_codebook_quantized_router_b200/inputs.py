@@ -154,10 +154,10 @@ def expert_weight(w: Workload, e: int, proj: str, device="cpu") -> torch.Tensor:
     return (t * WEIGHT_STD).to(torch.bfloat16)
 
 
-def activations(w: Workload, device="cpu", T: int | None = None) -> torch.Tensor:
-    """bf16 [T, H] activations, N(0, 1)."""
+def activations(w: Workload, device="cpu", T: int | None = None, variant: int = 0) -> torch.Tensor:
+    """bf16 [T, H] activations, N(0, 1); `variant` > 0 draws another batch."""
     T = w.T if T is None else T
-    g = _gen(w.seed_x * 7919 + 1, device)
+    g = _gen(w.seed_x * 7919 + 1 + variant * 1_000_033, device)
     return torch.randn((T, w.shape.H), generator=g, device=device).to(torch.bfloat16)
 
 
@@ -168,10 +168,11 @@ def zipf_bias(w: Workload, s: float = 1.1) -> np.ndarray:
     return (-s * np.log(rank.astype(np.float64))).astype(np.float32)
 
 
-def router_logits(w: Workload, device="cpu", T: int | None = None) -> torch.Tensor:
-    """fp32 [T, E] router logits: N(0, 1), plus the Zipf bias when skewed."""
+def router_logits(w: Workload, device="cpu", T: int | None = None, variant: int = 0) -> torch.Tensor:
+    """fp32 [T, E] router logits: N(0, 1), plus the Zipf bias when skewed;
+    `variant` > 0 draws another batch (same bias)."""
     T = w.T if T is None else T
-    g = _gen(w.seed_logits * 7919 + 2, device)
+    g = _gen(w.seed_logits * 7919 + 2 + variant * 1_000_033, device)
     lg = torch.randn((T, w.shape.E), generator=g, device=device, dtype=torch.float32)
     if w.zipf:
         lg = lg + torch.from_numpy(zipf_bias(w)).to(device)

@@ -1,0 +1,238 @@
+/*
+ * moe_q4 -- routed-expert MoE feed-forward over 4-bit codebook weights,
+ * for NVIDIA B200 (sm_100a).  C ABI.
+ *
+ * Weight format ("aidendle94/GLM-5.2-NF4-Lloyd-Experts-GPTQ", sections
+ * "Contents" and "Codes are indices into the per-layer grid -- not E2M1"):
+ *   - every weight is a 4-bit code: code & 0x7 indexes an 8-entry magnitude
+ *     table (the layer's Lloyd-Max grid, or the E2M1 table), code & 0x8 is
+ *     the sign;
+ *   - two codes per byte, the LOW nibble holds the EVEN K index;
+ *   - one E8M0 scale byte per 32 weights along K; the weight is
+ *       w = sign * table[code & 7] * 2^(scale_byte - 127);
+ *   - a projection W[N][K] is stored as `weight` uint8 [N][K/2] and
+ *     `weight_scale` uint8 [N][K/32], K contiguous; E experts are stacked
+ *     along a leading dimension.
+ * The layer (shapes as in "Round 7 -- Rewrite the GLM-5.2 routed-expert
+ * encoder", "Ground truth and corrections" and "Owner-locked decisions" 4, 6):
+ *   route:   top-k of E router logits per token, softmax over the k kept;
+ *   gate/up: g = W_gate x, u = W_up x          (W_gate, W_up: [I][H]);
+ *   SwiGLU:  h = silu(g) * u;
+ *   down:    y = W_down h                      (W_down: [H][I]);
+ *   combine: out = sum_j w_j * y_j over the k routed experts, in slot order.
+ *
+ * Conventions for every entry point:
+ *   - "device" pointers are CUDA device memory on the current device;
+ *     "host" pointers are ordinary host memory read during the call.
+ *   - The caller allocates and owns every buffer.  The library allocates
+ *     nothing inside these calls (moe_q4_forward_host excepted: none either,
+ *     it only stages through the caller's workspace).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without waiting, except where stated.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and return MOE_Q4_EINVAL (or MOE_Q4_EWORKSPACE); nothing is written.
+ *   - Errors that only the device can see (a NaN router logit, a non-finite
+ *     weight given to pack) are recorded in a device status word; read it
+ *     with moe_q4_forward_status / moe_q4_read_status.  Kernels never trap.
+ *   - bf16 tensors are passed as `void*` holding IEEE bfloat16 values.
+ */
+#ifndef MOE_Q4_H
+#define MOE_Q4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define MOE_Q4_API __attribute__((visibility("default")))
+#else
+#define MOE_Q4_API
+#endif
+
+#define MOE_Q4_ABI_VERSION 1
+
+/* Status codes. */
+#define MOE_Q4_OK 0
+#define MOE_Q4_EINVAL 1      /* null pointer, bad shape, K % 32, top_k > E, bad table, bad table id */
+#define MOE_Q4_ECUDA 2       /* a CUDA runtime/driver call or a launch failed */
+#define MOE_Q4_EWORKSPACE 3  /* workspace null or smaller than moe_q4_forward_workspace() */
+#define MOE_Q4_ETIMEOUT 4    /* a bounded device-side wait gave up */
+#define MOE_Q4_EDEVICE 5     /* the device flagged bad data (non-finite logit / weight) */
+#define MOE_Q4_ENOTSUP 6     /* a size beyond what this build supports */
+
+/* Limits of this build. */
+#define MOE_Q4_MAX_TABLES 16
+#define MOE_Q4_MAX_EXPERTS 512
+#define MOE_Q4_MAX_TOPK 16
+
+/* Version of this ABI (MOE_Q4_ABI_VERSION of the built library).  A caller
+ * compares it with the header it was built against before any other call. */
+MOE_Q4_API int moe_q4_abi_version(void);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+MOE_Q4_API const char* moe_q4_status_string(int status);
+
+/* ---------------------------------------------------------------------------
+ * moe_q4_pack -- quantise bf16 weights into codes + E8M0 scales.
+ *
+ * Rule ("Codes are indices into the per-layer grid -- not E2M1": codes are
+ * packed against gmax * 2^e >= amax, the grid is not amax-normalised), per
+ * 32-weight block along K of expert e with table t = tables[table_id[e]]:
+ *   e_blk = the smallest integer with max(t) * 2^e_blk >= max |x|, clamped to
+ *           [-127, 127] (an all-zero block takes -127); scale byte = e_blk+127;
+ *   code  = (x < 0 ? 8 : 0) | argmin_i |(|x| / 2^e_blk) - t[i]|, distances in
+ *           fp64, a tie taking the lower index.
+ * Arguments:
+ *   w            device, bf16 [E][N][K] (K contiguous);
+ *   E, N, K      E >= 0, N >= 0, K >= 0, K % 32 == 0;
+ *   tables       host, fp32 [n_tables][8] magnitudes, each finite and >= 0
+ *                with a positive maximum; 1 <= n_tables <= MOE_Q4_MAX_TABLES;
+ *   table_id     host, uint8 [E], each < n_tables;
+ *   weight       device, uint8 [E][N][K/2] (out);
+ *   weight_scale device, uint8 [E][N][K/32] (out);
+ *   status       device, one int32 (in/out): left unchanged when all inputs
+ *                are finite, set to MOE_Q4_EDEVICE if any input is NaN/Inf
+ *                (the affected block's bytes are then unspecified).
+ * Bit-exact with the reference definition above.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API int moe_q4_pack(const void* w, int E, int N, int K, const float* tables, int n_tables,
+                const uint8_t* table_id, uint8_t* weight, uint8_t* weight_scale,
+                int32_t* status, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_q4_dequant -- materialise packed weights as bf16 (the "materialize once"
+ * step of "GLM-5.2-EXL3-DENSE6-MTP78", "Serving stack" patch 2).
+ *
+ * out[e][n][k] = bf16(fp32(t[code & 7]) * 2^(s - 127)) with the fp32 multiply
+ * and the bf16 conversion both rounding to nearest even, the sign then
+ * applied by flipping bit 15 (a signed zero level gives -0.0), and scale byte
+ * 0xFF (E8M0 NaN) giving 0x7FC0 with the code's sign.  Bit-exact.
+ *   weight        device, uint8 [E][N][K/2];
+ *   weight_scale  device, uint8 [E][N][K/32];
+ *   tables, n_tables, table_id: as for moe_q4_pack (host);
+ *   out           device, bf16 [E][N][K] (out).
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API int moe_q4_dequant(const uint8_t* weight, const uint8_t* weight_scale, const float* tables,
+                   int n_tables, const uint8_t* table_id, int E, int N, int K, void* out,
+                   void* stream);
+
+/* A packed MoE layer.  Device pointers are borrowed for the duration of
+ * each call; tables and table_id are host memory read during each call. */
+typedef struct moe_q4_layer {
+  int E;                    /* routed experts, 1..MOE_Q4_MAX_EXPERTS */
+  int H;                    /* hidden size, % 128 == 0 */
+  int I;                    /* expert intermediate size, % 128 == 0 */
+  const uint8_t* gate_w;    /* device [E][I][H/2] */
+  const uint8_t* gate_s;    /* device [E][I][H/32] */
+  const uint8_t* up_w;      /* device [E][I][H/2] */
+  const uint8_t* up_s;      /* device [E][I][H/32] */
+  const uint8_t* down_w;    /* device [E][H][I/2] */
+  const uint8_t* down_s;    /* device [E][H][I/32] */
+  const float* tables;      /* host [n_tables][8] magnitudes */
+  int n_tables;             /* 1..MOE_Q4_MAX_TABLES */
+  const uint8_t* table_id;  /* host [E]: table of each expert */
+} moe_q4_layer;
+
+/* Bytes of device workspace moe_q4_forward needs for T tokens and top_k
+ * (0 if the arguments are invalid).  Deterministic in (layer shape, T, top_k). */
+MOE_Q4_API size_t moe_q4_forward_workspace(const moe_q4_layer* layer, int T, int top_k);
+
+/* ---------------------------------------------------------------------------
+ * moe_q4_forward -- one MoE layer for T tokens.
+ *
+ * Routing: per token the top_k largest logits (equal logits: lower expert id
+ * first), ids in descending-logit order; weights softmax over the kept
+ * logits in fp32.  Rows are grouped by expert (ascending id), tokens
+ * ascending within an expert.  Each expert's rows go through the small-M
+ * streaming path or the tensor-core path, chosen on the device from the
+ * per-expert row count.  The intermediate h = silu(g)*u is kept as a pair of
+ * bf16 values (its rounding and the rounding of the remainder), so the down
+ * GEMM sees it to ~16 significant bits; y is fp32; the combine sums
+ * the top_k slots in slot order in fp32 (deterministic, no atomics).
+ * Arguments:
+ *   layer      see moe_q4_layer;
+ *   x          device, bf16 [T][H];
+ *   logits     device, fp32 [T][E];
+ *   T          0 <= T; T * top_k <= 2^24;
+ *   top_k      1 <= top_k <= min(E, MOE_Q4_MAX_TOPK);
+ *   out        device, bf16 [T][H] (out): out_f32 rounded to nearest even;
+ *   out_f32    optional device fp32 [T][H] (out), NULL to skip: the combine's
+ *              fp32 sum, before the bf16 rounding of `out`;
+ *   topk_ids   optional device int32 [T][top_k] (out), NULL to skip;
+ *   topk_w     optional device fp32 [T][top_k] (out), NULL to skip;
+ *   counts     optional device int32 [E] rows per expert (out), NULL to skip;
+ *   ws         device workspace, 256-byte aligned, at least
+ *              moe_q4_forward_workspace(layer, T, top_k) bytes; the call owns
+ *              it until the enqueued work completes;
+ *   ws_bytes   size of ws.
+ * Device-detected errors (a non-finite logit) set the workspace status word;
+ * the output is then unspecified.  No host synchronisation, no allocation.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API int moe_q4_forward(const moe_q4_layer* layer, const void* x, const float* logits,
+                              int T, int top_k, void* out, float* out_f32, int32_t* topk_ids,
+                              float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                              void* stream);
+
+/* Synchronise `stream`, then return the status recorded in the workspace by
+ * the last moe_q4_forward on it (MOE_Q4_OK, MOE_Q4_EDEVICE, MOE_Q4_ETIMEOUT),
+ * or MOE_Q4_ECUDA if the stream itself reports an error. */
+MOE_Q4_API int moe_q4_forward_status(const void* ws, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_q4_forward_host -- the same layer with HOST activations and output.
+ * Copies x and logits host->device into the workspace, runs moe_q4_forward,
+ * copies out device->host and waits for the stream; returns the forward's
+ * device status.  x, logits and out are host pointers (pinned memory gives
+ * asynchronous copies); the weights stay on the device.  The workspace must
+ * hold moe_q4_forward_host_workspace(layer, T, top_k) bytes.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API size_t moe_q4_forward_host_workspace(const moe_q4_layer* layer, int T, int top_k);
+MOE_Q4_API int moe_q4_forward_host(const moe_q4_layer* layer, const void* x_host, const float* logits_host,
+                        int T, int top_k, void* out_host, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_q4_route -- the routing and grouping steps of moe_q4_forward alone,
+ * into caller buffers (all device, all required):
+ *   ids [T][top_k] int32, w [T][top_k] fp32: as moe_q4_forward's topk_ids/w;
+ *   counts [E] int32; offsets [E+1] int32 (exclusive scan of counts);
+ *   row_token [T*top_k] int32: token of each expert-grouped row (experts
+ *     ascending, tokens ascending within an expert);
+ *   inv [T][top_k] int32: grouped row of (token, slot).
+ * logits: device fp32 [T][E].  ws: device workspace of at least
+ * moe_q4_route_workspace(E, T, top_k) bytes, 256-byte aligned; its first
+ * int32 is the status word (read with moe_q4_forward_status(ws, stream)).
+ * Bit-exact: the grouping is unique given the ids, and the ids are unique
+ * under the ordering above.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API size_t moe_q4_route_workspace(int E, int T, int top_k);
+MOE_Q4_API int moe_q4_route(const float* logits, int T, int E, int top_k, int32_t* ids, float* w,
+                            int32_t* counts, int32_t* offsets, int32_t* row_token, int32_t* inv,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_q4_forward_stages -- moe_q4_forward with cudaEvent_t records at the
+ * stage boundaries, for timing each kernel on the launching stream:
+ *   events[0] before routing, [1] after routing/grouping, [2] after
+ *   gate/up + SwiGLU, [3] after the down projection, [4] after the combine.
+ * events: host array of n_events (>= 5) cudaEvent_t handles created by the
+ * caller.  The records separate the stages (no programmatic overlap across
+ * them), so throughput is measured with moe_q4_forward itself.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API int moe_q4_forward_stages(const moe_q4_layer* layer, const void* x,
+                                     const float* logits, int T, int top_k, void* out,
+                                     void* ws, size_t ws_bytes, void* stream,
+                                     void* const* events, int n_events);
+
+/* Synchronise `stream` and return the int32 at device address `status`
+ * (as written by moe_q4_pack), or MOE_Q4_ECUDA. */
+MOE_Q4_API int moe_q4_read_status(const int32_t* status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_Q4_H */

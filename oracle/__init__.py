@@ -63,7 +63,9 @@ def lib():
         L.oq_route.argtypes = [vp, ci, ci, ci, vp, vp]
         L.oq_group.argtypes = [vp, ci, ci, ci, vp, vp, vp, vp]
         L.oq_moe_tokens.argtypes = [ctypes.POINTER(_Layer), vp, vp, ci, ci, vp, vp, vp]
-        for f in (L.oq_dequant, L.oq_decode_matrix_f64, L.oq_pack, L.oq_route, L.oq_group, L.oq_moe_tokens):
+        L.oq_expert_partial.argtypes = [ctypes.POINTER(_Layer), ci, vp, ci, ci, vp]
+        for f in (L.oq_dequant, L.oq_decode_matrix_f64, L.oq_pack, L.oq_route, L.oq_group, L.oq_moe_tokens,
+                  L.oq_expert_partial):
             f.restype = ci
         _lib = L
     return _lib
@@ -204,3 +206,14 @@ def moe_tokens(layer: Layer, x_bf16_bits, logits, k, return_routing=False):
     if return_routing:
         return out, ids, w
     return out
+
+
+def expert_partial(layer: Layer, e: int, x_bits_row, i0: int, i1: int):
+    """fp64 [H]: expert e's output for one token (x bf16 bits [H]) restricted
+    to intermediate channels [i0, i1)."""
+    x = _c(x_bits_row, np.uint16).reshape(-1)
+    y = np.empty(layer.H, np.float64)
+    st, keep = layer._struct()
+    _check(lib().oq_expert_partial(ctypes.byref(st), e, _p(x), i0, i1, _p(y)))
+    del keep
+    return y

@@ -398,3 +398,39 @@ done:
   free(wts);
   return rc;
 }
+
+/* One expert's output for one token restricted to intermediate channels
+ * [i0, i1):  y[n] = sum_{i0 <= i < i1} Wd_e[n][i] * silu(g_i) * u_i, with
+ * g = Wg_e x and u = Wu_e x as in oq_moe_tokens.  The expert's full output is
+ * the sum of these over any partition of [0, I); the benchmark's CPU
+ * baseline times such pieces as bounded samples of the layer.
+ * x: [H] bf16 bits; y: [H] fp64 (out). */
+int oq_expert_partial(const oq_layer* L, int e, const uint16_t* x, int i0, int i1, double* y) {
+  if (!L || e < 0 || e >= L->E || i0 < 0 || i1 > L->I || i0 > i1 || !x || !y) return OQ_EINVAL;
+  if (!tables_ok(L->tables, L->n_tables, L->table_id, L->E)) return OQ_EINVAL;
+  if (!L->gate_w[e] || !L->gate_s[e] || !L->up_w[e] || !L->up_s[e] || !L->down_w[e] || !L->down_s[e])
+    return OQ_EINVAL;
+  const int H = L->H, I = L->I;
+  const float* tb = L->tables + 8 * L->table_id[e];
+  double* xv = (double*)malloc(sizeof(double) * H);
+  if (!xv) return OQ_EINVAL;
+  for (int h = 0; h < H; ++h) xv[h] = (double)bf16_bits_to_f32(x[h]);
+  for (int n = 0; n < H; ++n) y[n] = 0.0;
+  for (int i = i0; i < i1; ++i) {
+    double g = 0.0, u = 0.0;
+    const uint8_t* gw = L->gate_w[e] + (size_t)i * (H / 2);
+    const uint8_t* gs = L->gate_s[e] + (size_t)i * (H / 32);
+    const uint8_t* uw = L->up_w[e] + (size_t)i * (H / 2);
+    const uint8_t* us = L->up_s[e] + (size_t)i * (H / 32);
+    for (int k = 0; k < H; ++k) {
+      g += decode_f64(code_at(gw, k), gs[k / 32], tb) * xv[k];
+      u += decode_f64(code_at(uw, k), us[k / 32], tb) * xv[k];
+    }
+    const double hi = g / (1.0 + exp(-g)) * u;
+    for (int n = 0; n < H; ++n)
+      y[n] += decode_f64(code_at(L->down_w[e] + (size_t)n * (I / 2), i),
+                         L->down_s[e][(size_t)n * (I / 32) + i / 32], tb) * hi;
+  }
+  free(xv);
+  return OQ_OK;
+}

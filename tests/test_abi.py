@@ -1,0 +1,96 @@
+"""The C-ABI library (no GPU needed): it loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any launch."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import bit_codebook_quantized_router_b200 as q4
+from bit_codebook_quantized_router_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_q4.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_codebook_quantized_router_b200 import build
+    build.build()
+    return _lib.lib()
+
+
+def declared_symbols():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"MOE_Q4_API\s+[\w\s\*]+?\b(moe_q4_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for s in ("moe_q4_pack", "moe_q4_dequant", "moe_q4_forward", "moe_q4_forward_workspace",
+              "moe_q4_abi_version", "moe_q4_status_string", "moe_q4_route", "moe_q4_forward_host"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(L):
+    for s in declared_symbols():
+        assert hasattr(L, s), s
+    assert L.moe_q4_abi_version() == 1
+    for code in range(8):
+        assert L.moe_q4_status_string(code)
+
+
+def _layer(E=8, H=256, I=128, tables=None, table_id=None, null=False):
+    t = np.ascontiguousarray(tables if tables is not None else np.linspace(0.1, 2, 8, dtype=np.float32)[None])
+    tid = np.ascontiguousarray(table_id if table_id is not None else np.zeros(E, np.uint8))
+    fake = 0 if null else 1 << 20  # never dereferenced: validation fails first
+    st = _lib._LayerStruct(E, H, I, fake, fake, fake, fake, fake, fake, t.ctypes.data, t.shape[0], tid.ctypes.data)
+    return st, (t, tid)
+
+
+def test_workspace_query_and_shape_validation(L):
+    st, keep = _layer()
+    assert L.moe_q4_forward_workspace(ctypes.byref(st), 4, 2) > 0
+    assert L.moe_q4_forward_workspace(ctypes.byref(st), 4, 9) == 0  # k > E
+    assert L.moe_q4_forward_workspace(ctypes.byref(st), -1, 2) == 0
+    bad, keep2 = _layer(H=250)
+    assert L.moe_q4_forward_workspace(ctypes.byref(bad), 4, 2) == 0  # H % 128
+    nul, keep3 = _layer(null=True)
+    assert L.moe_q4_forward_workspace(ctypes.byref(nul), 4, 2) == 0
+
+
+def test_forward_rejects_bad_arguments_before_launch(L):
+    st, keep = _layer()
+    f = L.moe_q4_forward
+    # top_k out of range
+    assert f(ctypes.byref(st), 16, 16, 4, 0, 16, None, None, None, None, 256, 1 << 20, None) == _lib.EINVAL
+    # null activations
+    assert f(ctypes.byref(st), None, 16, 4, 2, 16, None, None, None, None, 256, 1 << 20, None) == _lib.EINVAL
+    # workspace too small / misaligned
+    assert f(ctypes.byref(st), 16, 16, 4, 2, 16, None, None, None, None, 256, 10, None) == _lib.EWORKSPACE
+    assert f(ctypes.byref(st), 16, 16, 4, 2, 16, None, None, None, None, 100, 1 << 30, None) == _lib.EWORKSPACE
+    # bad tables: NaN, negative, -0.0, all zero, table id out of range
+    for tb in ([np.nan] + [1.0] * 7, [-1.0] + [1.0] * 7, [-0.0] + [1.0] * 7, [0.0] * 8):
+        bt, k2 = _layer(tables=np.array([tb], np.float32))
+        assert f(ctypes.byref(bt), 16, 16, 4, 2, 16, None, None, None, None, 256, 1 << 30, None) == _lib.EINVAL
+    bt, k3 = _layer(table_id=np.full(8, 1, np.uint8))
+    assert f(ctypes.byref(bt), 16, 16, 4, 2, 16, None, None, None, None, 256, 1 << 30, None) == _lib.EINVAL
+
+
+def test_pack_dequant_reject_bad_shapes(L):
+    t = np.linspace(0.1, 2, 8, dtype=np.float32)
+    tid = np.zeros(2, np.uint8)
+    # K % 32 != 0
+    assert L.moe_q4_pack(16, 2, 4, 48, t.ctypes.data, 1, tid.ctypes.data, 16, 16, 16, None) == _lib.EINVAL
+    assert L.moe_q4_dequant(16, 16, t.ctypes.data, 1, tid.ctypes.data, 2, 4, 48, 16, None) == _lib.EINVAL
+    # too many tables
+    assert L.moe_q4_dequant(16, 16, t.ctypes.data, 17, tid.ctypes.data, 2, 4, 64, 16, None) == _lib.EINVAL
+    # empty is a no-op
+    assert L.moe_q4_dequant(None, None, t.ctypes.data, 1, tid.ctypes.data, 0, 4, 64, None, None) == _lib.OK
+
+
+def test_route_workspace_validation(L):
+    assert L.moe_q4_route_workspace(256, 8, 8) > 0
+    assert L.moe_q4_route_workspace(256, 8, 17) == 0
+    assert L.moe_q4_route_workspace(600, 8, 8) == 0

@@ -171,3 +171,18 @@ def test_missing_expert_is_an_error(tiny_layer):
     lg[0, 1] = 1.0
     with pytest.raises(oracle.OracleError):
         oracle.moe_tokens(L2, np.zeros((1, L.H), np.uint16), lg, 1)
+
+
+def test_expert_partials_sum_to_the_layer(tiny_layer):
+    # Partials over a partition of the intermediate channels, weighted by the
+    # routing weights, reproduce the layer output.
+    L, _ = tiny_layer
+    x = inputs.bf16_bits(inputs.activations(TINY))
+    lg = inputs.router_logits(TINY).numpy()
+    out, ids, w = oracle.moe_tokens(L, x, lg, 2, return_routing=True)
+    for t in range(TINY.T):
+        acc = np.zeros(L.H)
+        for j in range(2):
+            for i0, i1 in ((0, 40), (40, 41), (41, 128)):
+                acc += w[t, j] * oracle.expert_partial(L, int(ids[t, j]), x[t], i0, i1)
+        np.testing.assert_allclose(acc, out[t], rtol=1e-12, atol=1e-14 * np.abs(out[t]).max())
