@@ -46,7 +46,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 
 def workload_desc(w: inputs.Workload) -> dict:
     sh = w.shape
-    d = {"workload": f"{w.name}: GLM-5.2-shaped routed-expert MoE layer, T={w.T}, H={sh.H}, I={sh.I}, "
+    kind = "GLM-5.2-shaped" if sh == inputs.GLM else "small"
+    d = {"workload": f"{w.name}: {kind} routed-expert MoE layer, T={w.T}, H={sh.H}, I={sh.I}, "
                      f"E={sh.E}, top-{sh.k}, 4-bit Lloyd-codebook codes + E8M0 scale per 32",
          "T": w.T, "H": sh.H, "I": sh.I, "E": sh.E, "top_k": sh.k,
          "routing": "zipf-skewed" if w.zipf else "uniform random",
@@ -335,6 +336,10 @@ def run_ours(args, w):
     # stage times (separate pass, events between the kernels)
     n_prof = min(args.steps, 100)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_prof)]
+    for row in evs:  # torch creates the CUDA event on first record
+        for ev in row:
+            ev.record(stream)
+    torch.cuda.synchronize()
     for i in range(n_prof):
         flush.fill_(i & 0xFF)
         q4.forward_stages(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out, ws, evs[i])

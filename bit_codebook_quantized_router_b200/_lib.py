@@ -221,7 +221,8 @@ def route(logits: torch.Tensor, k: int, stream=None):
 
 
 def forward_stages(layer: Layer, x, logits, k: int, out, ws, events, stream=None) -> None:
-    """moe_q4_forward with torch.cuda.Event records at the 5 stage boundaries."""
+    """moe_q4_forward with torch.cuda.Event records at the 5 stage boundaries
+    (the events must have been recorded once: torch creates them lazily)."""
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     st = layer.struct()
     _check(lib().moe_q4_forward_stages(ctypes.byref(st), _ptr(x), _ptr(logits), x.shape[0], k, _ptr(out),

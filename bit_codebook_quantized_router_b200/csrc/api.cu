@@ -14,6 +14,11 @@ using namespace q4;
 namespace {
 
 constexpr size_t kAlign = 256;
+// Experts with at most this many rows take the streaming (mma.sync) path;
+// larger ones the tcgen05 path.
+constexpr int kDecodeMaxRows = 16;
+
+bool uses_prefill(int T) { return T > kDecodeMaxRows; }
 
 size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
@@ -38,10 +43,11 @@ bool shape_ok(const moe_q4_layer* L, int T, int top_k) {
 // Workspace layout, every array 256-byte aligned:
 //   header int32[64] | ids int32[T*k] | w f32[T*k] | counts int32[E] |
 //   offsets int32[E+1] | row_token int32[T*k] | inv int32[T*k] |
-//   dec_list int32[E] | pre_list int32[E] | h bf16[T*k][I] | h_lo bf16[T*k][I] |
-//   y f32[T*k][H]
+//   dec_list int32[E] | pre_list int32[E] | tiles int32[E+1] | h bf16[T*k][I] |
+//   h_lo bf16[T*k][I] | y f32[T*k][H] | xg bf16[T*k][H] (only when T > 16:
+//   activation rows in expert order for the tensor-core path)
 struct Layout {
-  size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, h, h_lo, y, end;
+  size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, tiles, h, h_lo, y, xg, end;
 };
 
 Layout layout(const moe_q4_layer* L, int T, int k) {
@@ -66,12 +72,16 @@ Layout layout(const moe_q4_layer* L, int T, int k) {
   p = align_up(p + sizeof(int32_t) * L->E);
   o.pre_list = p;
   p = align_up(p + sizeof(int32_t) * L->E);
+  o.tiles = p;
+  p = align_up(p + sizeof(int32_t) * (L->E + 1));
   o.h = p;
   p = align_up(p + sizeof(__nv_bfloat16) * R * L->I);
   o.h_lo = p;
   p = align_up(p + sizeof(__nv_bfloat16) * R * L->I);
   o.y = p;
   p = align_up(p + sizeof(float) * R * L->H);
+  o.xg = p;
+  if (uses_prefill(T)) p = align_up(p + sizeof(__nv_bfloat16) * R * L->H);
   o.end = p;
   return o;
 }
@@ -105,8 +115,8 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   a.E = L->E;
   a.H = L->H;
   a.I = L->I;
-  a.dec_max = INT_MAX;
-  a.tile_n = 0;
+  a.dec_max = kDecodeMaxRows;
+  a.tile_n = q4_prefill_tile_n();
   a.x = (const __nv_bfloat16*)x;
   a.logits = logits;
   a.out = (__nv_bfloat16*)out;
@@ -119,6 +129,8 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   a.inv = (int32_t*)(ws + o.inv);
   a.dec_list = (int32_t*)(ws + o.dec_list);
   a.pre_list = (int32_t*)(ws + o.pre_list);
+  a.tiles = (int32_t*)(ws + o.tiles);
+  a.xg = uses_prefill(T) ? (__nv_bfloat16*)(ws + o.xg) : nullptr;
   a.h = (__nv_bfloat16*)(ws + o.h);
   a.h_lo = (__nv_bfloat16*)(ws + o.h_lo);
   a.y = (float*)(ws + o.y);
@@ -136,11 +148,17 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
     if (events && cudaEventRecord((cudaEvent_t)events[i], s) != cudaSuccess) return MOE_Q4_ECUDA;
     return MOE_Q4_OK;
   };
+  // With T <= kDecodeMaxRows no expert can have more rows than the streaming
+  // path takes, so the tensor-core kernels are not launched at all.
+  const bool pre = uses_prefill(T);
   int rc = mark(0);
   if (rc == MOE_Q4_OK) rc = q4_launch_route(a, s);
   if (rc == MOE_Q4_OK) rc = mark(1);
+  if (rc == MOE_Q4_OK && pre) rc = q4_launch_gather(a, s);
+  if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, true, s);
   if (rc == MOE_Q4_OK) rc = q4_launch_decode(a, tp, true, s);
   if (rc == MOE_Q4_OK) rc = mark(2);
+  if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, false, s);
   if (rc == MOE_Q4_OK) rc = q4_launch_decode(a, tp, false, s);
   if (rc == MOE_Q4_OK) rc = mark(3);
   if (rc == MOE_Q4_OK) rc = q4_launch_combine(a, s);

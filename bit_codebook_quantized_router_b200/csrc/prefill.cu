@@ -1,0 +1,406 @@
+// Large-M ("prefill") expert GEMMs on the 5th-generation tensor cores.
+//
+//   gate/up: h[row] = silu(W_gate x) * (W_up x)     (fused SwiGLU epilogue)
+//   down:    y[row] = W_down h[row]
+// ("Round 7 -- Rewrite the GLM-5.2 routed-expert encoder", "Owner-locked
+// decisions" 4 and 6), for the experts whose row count exceeds the streaming
+// path's limit.
+//
+// Swap-AB grouped GEMM: the MMA's M = 128 weight rows, N = a tile of BN
+// tokens of one expert, K streamed in steps of 64.  A persistent CTA per SM
+// walks tiles ordered (expert, weight m-tile, token tile) so the token tiles
+// of one weight tile run back to back and re-read it from L2.
+//
+// Warp roles (448 threads):
+//   warp 0       TMA producer: packed codes of the m-tile (128 rows x 32 B per
+//                k-step, 32-byte swizzle) and the token tile (BN rows x 128 B,
+//                128-byte swizzle) into a 3-4 stage ring;
+//   warp 1       allocates TMEM and issues tcgen05.mma (one thread): for each
+//                k-step, 4 MMAs of K=16 per weight matrix into fp32 TMEM
+//                accumulators, double-buffered across tiles;
+//   warps 2..9   dequantise: codes -> bf16 through the PRMT byte-plane lookup
+//                of the expert's table, E8M0 scale by an exact bf16x2
+//                multiply, stored to smem in the canonical 128-byte-swizzle
+//                K-major layout the MMA reads ("aidendle94/GLM-5.2-NF4-Lloyd-
+//                Experts-GPTQ", "Codes are indices into the per-layer grid");
+//   warps 10..13 epilogue: tcgen05.ld of the accumulators (one TMEM lane = one
+//                weight row per thread), SwiGLU in fp32, bf16 stores of h (or
+//                fp32 stores of y).
+// Every mbarrier wait is bounded; on a timeout the CTA sets the status word
+// to MOE_Q4_ETIMEOUT, drains its own copies and MMAs (bounded), frees TMEM
+// and exits.
+#include <cuda.h>
+
+#include "q4_api_internal.h"
+#include "q4_common.cuh"
+#include "sm100.cuh"
+
+namespace q4 {
+
+using namespace sm100;
+
+constexpr int kBN = 128;          // token tile (MMA N)
+constexpr int kBM = 128;          // weight rows per tile (MMA M)
+constexpr int kBK = 64;           // K per pipeline stage (128 bytes of bf16)
+constexpr int kThreads = 448;
+constexpr int kDequantThreads = 256;
+constexpr int kEpiWarp0 = 10;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+template <bool GATEUP>
+struct TcCfg {
+  static constexpr int kMats = GATEUP ? 2 : 1;
+  static constexpr int kStages = GATEUP ? 3 : 4;
+  static constexpr int kATile = kBM * kBK * 2;        // 16 KB bf16 per matrix
+  static constexpr int kBTile = kBN * kBK * 2;        // 16 KB
+  static constexpr int kCTile = kBM * kBK / 2;        // 4 KB codes per matrix
+  static constexpr int kStageBytes = kMats * kATile + kBTile + kMats * kCTile;
+  static constexpr int kTmemCols = 2 * kMats * kBN;   // double-buffered accumulators
+  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 1024 /*barriers*/;
+};
+
+struct TcParams {
+  FwdArgs a;
+  int m_tiles;  // weight rows / 128
+  int k_steps;  // K / 64
+};
+
+// Tile id -> (prefill slot p, m-tile, token tile) with tiles ordered
+// (expert, m, n); ntile_off[p] = token tiles of the prefill experts before p.
+__device__ __forceinline__ void tile_coords(const FwdArgs& a, int m_tiles, int np, int tile, int& p, int& m,
+                                            int& nt) {
+  int lo = 0, hi = np - 1;
+  while (lo < hi) {  // last p with m_tiles * ntile_off[p] <= tile
+    const int mid = (lo + hi + 1) >> 1;
+    if (m_tiles * a.tiles[mid] <= tile)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  p = lo;
+  const int n_tiles_p = a.tiles[p + 1] - a.tiles[p];
+  const int local = tile - m_tiles * a.tiles[p];
+  m = local / n_tiles_p;
+  nt = local - m * n_tiles_p;
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    tc_gemm_kernel(const __grid_constant__ TcParams P, const __grid_constant__ TableParams tp,
+                   const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_wa,
+                   const __grid_constant__ CUtensorMap tm_wb) {
+  using C = TcCfg<GATEUP>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                                        // [S][mats][128][128 B]
+  uint8_t* sB = sA + C::kStages * C::kMats * C::kATile;      // [S][BN][128 B]
+  uint8_t* sC = sB + C::kStages * C::kBTile;                 // [S][mats][128][32 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + C::kStages * C::kMats * C::kCTile);
+  uint64_t* full_c = bars;                       // [S] codes landed
+  uint64_t* full_b = full_c + C::kStages;        // [S] token tile landed
+  uint64_t* a_ready = full_b + C::kStages;       // [S] bf16 A tiles written
+  uint64_t* empty = a_ready + C::kStages;        // [S] stage consumed by the MMAs
+  uint64_t* acc_full = empty + C::kStages;       // [2]
+  uint64_t* acc_empty = acc_full + 2;            // [2]
+  uint64_t* drain = acc_empty + 2;               // [1] final MMA completion
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const FwdArgs& a = P.a;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full_c[s], 1);
+      mbar_init(&full_b[s], 1);
+      mbar_init(&a_ready[s], kDequantThreads);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_b);
+    prefetch_tmap(&tm_wa);
+    if (GATEUP) prefetch_tmap(&tm_wb);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  pdl_wait();
+  const int np = a.hdr[kNumPrefill];
+  const int total = np > 0 ? P.m_tiles * a.tiles[np] : 0;
+  const int rows_total = GATEUP ? a.I : a.H;
+  const int K = GATEUP ? a.H : a.I;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+        int p, m, nt;
+        tile_coords(a, P.m_tiles, np, tile, p, m, nt);
+        const int e = a.pre_list[p];
+        const int wrow = e * rows_total + m * kBM;
+        const int brow = a.offsets[e] + nt * kBN;
+        for (int ks = 0; ks < P.k_steps; ++ks, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) break;
+          mbar_arrive_expect_tx(&full_c[s], C::kMats * C::kCTile);
+          tma_load_2d(sC + (s * C::kMats) * C::kCTile, &tm_wa, &full_c[s], ks * (kBK / 2), wrow);
+          if (GATEUP) tma_load_2d(sC + (s * C::kMats + 1) * C::kCTile, &tm_wb, &full_c[s], ks * (kBK / 2), wrow);
+          mbar_arrive_expect_tx(&full_b[s], C::kBTile);
+          tma_load_2d(sB + s * C::kBTile, &tm_b, &full_b[s], ks * kBK, brow);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_bf16(kBM, kBN);
+      uint32_t it = 0, tcount = 0;
+      for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
+        const int buf = tcount & 1;
+        if (!mbar_wait(&acc_empty[buf], ((tcount >> 1) & 1) ^ 1, abort_flag, kWaitLimitNs)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + buf * (C::kMats * kBN);
+        bool ok = true;
+        for (int ks = 0; ks < P.k_steps; ++ks, ++it) {
+          const int s = it % C::kStages;
+          const uint32_t ph = (it / C::kStages) & 1;
+          if (!mbar_wait(&full_b[s], ph, abort_flag, kWaitLimitNs) ||
+              !mbar_wait(&a_ready[s], ph, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t db = umma_desc_sw128(smem_u32(sB + s * C::kBTile));
+#pragma unroll
+          for (int mat = 0; mat < C::kMats; ++mat) {
+            const uint64_t da = umma_desc_sw128(smem_u32(sA + (s * C::kMats + mat) * C::kATile));
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes of K per MMA (>> 4 -> +2)
+              umma_bf16(d0 + mat * kBN, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[buf]);
+      }
+      // all MMAs issued by this thread complete before TMEM is released
+      umma_commit(drain);
+      mbar_wait(drain, 0, abort_flag, kWaitLimitNs);
+    }
+  } else if (warp < kEpiWarp0) {
+    // ---------------- dequantise ----------------
+    const int d = threadIdx.x - 64;           // 0..255
+    const int r = d & (kBM - 1);              // weight row in the tile
+    const int part = d >> 7;                  // gate/up: matrix; down: K half
+    uint32_t it = 0;
+    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+      int p, m, nt;
+      tile_coords(a, P.m_tiles, np, tile, p, m, nt);
+      const int e = a.pre_list[p];
+      const Planes PL = make_planes(tp.t[tp.id[e]]);
+      const int mat = GATEUP ? part : 0;
+      const uint8_t* srow = (GATEUP ? (part ? a.up_s : a.gate_s) : a.down_s) +
+                            ((size_t)e * rows_total + m * kBM + r) * (size_t)(K / 32);
+      uint4 sc = make_uint4(0, 0, 0, 0);
+      bool ok = true;
+      for (int ks = 0; ks < P.k_steps; ++ks, ++it) {
+        if ((ks & 7) == 0) sc = ldg_nc(srow + ks * 2);  // 16 scale bytes = 8 k-steps
+        const int s = it % C::kStages;
+        const uint32_t ph = (it / C::kStages) & 1;
+        if (!mbar_wait(&full_c[s], ph, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* ctile = sC + (s * C::kMats + mat) * C::kCTile;
+        uint8_t* arow = sA + (s * C::kMats + mat) * C::kATile + r * 128;
+        const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
+        // 32-byte swizzle of the codes tile: chunk c of row r at c ^ ((r >> 2) & 1)
+        const int sw = (r >> 2) & 1;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (!GATEUP && half != part) continue;
+          const uint4 cv = *reinterpret_cast<const uint4*>(ctile + r * 32 + ((half ^ sw) << 4));
+          const int blk = 2 * (ks & 7) + half;                     // block within the 16 loaded
+          const uint32_t sbyte = (scw[blk >> 2] >> ((blk & 3) * 8)) & 0xffu;
+          uint32_t w16[16];
+          const uint32_t s2 = scale_bf16x2(sbyte);
+          decode8(cv.x, PL, &w16[0]);
+          decode8(cv.y, PL, &w16[4]);
+          decode8(cv.z, PL, &w16[8]);
+          decode8(cv.w, PL, &w16[12]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {  // 16-byte chunks 4*half + q of the row, 128-byte swizzle
+            const int ch = 4 * half + q;
+            uint4 v = make_uint4(bf16x2_mul(w16[4 * q], s2), bf16x2_mul(w16[4 * q + 1], s2),
+                                 bf16x2_mul(w16[4 * q + 2], s2), bf16x2_mul(w16[4 * q + 3], s2));
+            *reinterpret_cast<uint4*>(arow + ((ch ^ (r & 7)) << 4)) = v;
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&a_ready[s]);
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int quad = warp & 3;          // TMEM lanes 32*quad .. +31
+    const int row = quad * 32 + lane;   // weight row in the tile
+    uint32_t tcount = 0;
+    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
+      int p, m, nt;
+      tile_coords(a, P.m_tiles, np, tile, p, m, nt);
+      const int e = a.pre_list[p];
+      const int n_e = a.counts[e];
+      const int row0 = a.offsets[e];
+      const int buf = tcount & 1;
+      if (!mbar_wait(&acc_full[buf], (tcount >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * (C::kMats * kBN);
+      const int wrow = m * kBM + row;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBN; c0 += 32) {
+        float g[32];
+        tmem_ld32(tb + c0, g);
+        if (GATEUP) {
+          float u[32];
+          tmem_ld32(tb + kBN + c0, u);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = nt * kBN + c0 + j;
+            if (n < n_e) a.h[(size_t)(row0 + n) * a.I + wrow] = __float2bfloat16_rn(silu_mul(g[j], u[j]));
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int n = nt * kBN + c0 + j;
+            if (n < n_e) a.y[(size_t)(row0 + n) * a.H + wrow] = g[j];
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  // ---------------- teardown ----------------
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) record_error(a.hdr + kStatus, MOE_Q4_ETIMEOUT);
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    // let any copy still in flight land before the CTA's smem goes away
+    for (int s = 0; s < C::kStages; ++s) {
+      volatile int quick = 0;
+      mbar_wait(&full_c[s], 0, &quick, 50000000ull);
+      quick = 0;
+      mbar_wait(&full_c[s], 1, &quick, 50000000ull);
+      quick = 0;
+      mbar_wait(&full_b[s], 0, &quick, 50000000ull);
+      quick = 0;
+      mbar_wait(&full_b[s], 1, &quick, 50000000ull);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+  pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major [rows][cols] array.
+static bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
+                     uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool GATEUP>
+static int launch_tc(const FwdArgs& a, const TableParams& tp, cudaStream_t s) {
+  using C = TcCfg<GATEUP>;
+  TcParams P;
+  P.a = a;
+  P.m_tiles = (GATEUP ? a.I : a.H) / kBM;
+  P.k_steps = (GATEUP ? a.H : a.I) / kBK;
+  const int R = a.T * a.k;
+  CUtensorMap tb, twa, twb;
+  bool ok;
+  if (GATEUP) {
+    ok = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.xg, a.H, R, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.gate_w, a.H / 2, (uint64_t)a.E * a.I, kBK / 2, kBM,
+                  CU_TENSOR_MAP_SWIZZLE_32B) &&
+         make_map(&twb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.up_w, a.H / 2, (uint64_t)a.E * a.I, kBK / 2, kBM,
+                  CU_TENSOR_MAP_SWIZZLE_32B);
+  } else {
+    ok = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.h, a.I, R, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         make_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.down_w, a.I / 2, (uint64_t)a.E * a.H, kBK / 2, kBM,
+                  CU_TENSOR_MAP_SWIZZLE_32B);
+    twb = twa;
+  }
+  if (!ok) return MOE_Q4_ECUDA;
+  if (cudaFuncSetAttribute(tc_gemm_kernel<GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+      cudaSuccess)
+    return MOE_Q4_ECUDA;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(sms);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<GATEUP>, P, tp, tb, twa, twb) == cudaSuccess ? MOE_Q4_OK
+                                                                                                  : MOE_Q4_ECUDA;
+}
+
+}  // namespace q4
+
+using namespace q4;
+
+int q4_prefill_tile_n() { return kBN; }
+
+int q4_launch_prefill(const FwdArgs& a, const TableParams& tp, bool gateup, cudaStream_t s) {
+  return gateup ? launch_tc<true>(a, tp, s) : launch_tc<false>(a, tp, s);
+}

@@ -28,7 +28,7 @@ struct FwdArgs {
   int32_t* inv;            // [T*k]
   int32_t* dec_list;       // [E]
   int32_t* pre_list;       // [E]
-  int32_t* tiles;          // [max_tiles][2] (expert, first row)
+  int32_t* tiles;          // [E+1] token-tile offsets of the tensor-core-path experts
   __nv_bfloat16* h;        // [T*k][I] bf16 rounding of silu(g)*u
   __nv_bfloat16* h_lo;     // [T*k][I] bf16 rounding of the remainder silu(g)*u - h
   float* y;                // [T*k][H]
@@ -49,3 +49,6 @@ int q4_fill_tables(q4::TableParams* tp, const float* tables, int n_tables, const
 int q4_launch_route(const q4::FwdArgs& a, cudaStream_t s);
 int q4_launch_decode(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, cudaStream_t s);
 int q4_launch_combine(const q4::FwdArgs& a, cudaStream_t s);
+int q4_launch_gather(const q4::FwdArgs& a, cudaStream_t s);
+int q4_launch_prefill(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, cudaStream_t s);
+int q4_prefill_tile_n();

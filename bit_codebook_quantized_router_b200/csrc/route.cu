@@ -151,6 +151,11 @@ __device__ void group_rows(const FwdArgs& a, int* sm) {
   int nd, np;
   const int pd = block_exclusive_scan(fd ? 1 : 0, warp_tot, nd);
   const int pp = block_exclusive_scan(fp ? 1 : 0, warp_tot, np);
+  // token tiles of each tensor-core-path expert, as an exclusive scan in
+  // pre_list order (tiles[p] .. tiles[p+1]-1 are expert pre_list[p]'s)
+  int ntot;
+  const int ntl = fp ? (c + a.tile_n - 1) / a.tile_n : 0;
+  const int ntoff = block_exclusive_scan(ntl, warp_tot, ntot);
   if (tid < E) {
     offs[tid] = off;
     a.offsets[tid] = off;
@@ -158,12 +163,15 @@ __device__ void group_rows(const FwdArgs& a, int* sm) {
     if (a.user_counts) a.user_counts[tid] = c;
     if (fd) a.dec_list[pd] = tid;
     if (fp) a.pre_list[pp] = tid;
+    if (fp && a.tiles) a.tiles[pp] = ntoff;
   }
   if (tid == 0) {
     offs[E] = total;
     a.offsets[E] = total;
     a.hdr[kNumDecode] = nd;
     a.hdr[kNumPrefill] = np;
+    a.hdr[kNumTiles] = ntot;
+    if (a.tiles) a.tiles[np] = ntot;
   }
   __syncthreads();
   // stable placement, kRouteThreads tokens per round

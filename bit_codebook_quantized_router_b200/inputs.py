@@ -148,7 +148,7 @@ def expert_weight(w: Workload, e: int, proj: str, device="cpu") -> torch.Tensor:
     comparison must take the same tensor.
     """
     N, K = proj_shape(w.shape, proj)
-    seed = (w.seed_weights * 1_000_003 + e * 17 + PROJECTIONS.index(proj)) * 2_654_435_761
+    seed = (int(w.seed_weights) * 1_000_003 + int(e) * 17 + PROJECTIONS.index(proj)) * 2_654_435_761
     g = _gen(seed, device)
     t = torch.randn((N, K), generator=g, device=device, dtype=torch.float32)
     return (t * WEIGHT_STD).to(torch.bfloat16)
