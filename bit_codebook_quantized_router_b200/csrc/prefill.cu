@@ -215,10 +215,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mat = GATEUP ? part : 0;
       const uint8_t* srow = (GATEUP ? (part ? a.up_s : a.gate_s) : a.down_s) +
                             ((size_t)e * rows_total + m * kBM + r) * (size_t)(K / 32);
-      uint4 sc = make_uint4(0, 0, 0, 0);
+      // scale bytes of blocks 2ks .. 2ks+3 (k-steps ks, ks+1): K % 128 == 0 keeps
+      // every 4-byte load inside the row and aligned
+      uint32_t sc = 0;
       bool ok = true;
       for (int ks = 0; ks < P.k_steps; ++ks, ++it) {
-        if ((ks & 7) == 0) sc = ldg_nc(srow + ks * 2);  // 16 scale bytes = 8 k-steps
+        if ((ks & 1) == 0) sc = *reinterpret_cast<const uint32_t*>(srow + ks * 2);
         const int s = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
         if (!mbar_wait(&full_c[s], ph, abort_flag, kWaitLimitNs)) {
@@ -227,15 +229,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const uint8_t* ctile = sC + (s * C::kMats + mat) * C::kCTile;
         uint8_t* arow = sA + (s * C::kMats + mat) * C::kATile + r * 128;
-        const uint32_t scw[4] = {sc.x, sc.y, sc.z, sc.w};
         // 32-byte swizzle of the codes tile: chunk c of row r at c ^ ((r >> 2) & 1)
         const int sw = (r >> 2) & 1;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           if (!GATEUP && half != part) continue;
           const uint4 cv = *reinterpret_cast<const uint4*>(ctile + r * 32 + ((half ^ sw) << 4));
-          const int blk = 2 * (ks & 7) + half;                     // block within the 16 loaded
-          const uint32_t sbyte = (scw[blk >> 2] >> ((blk & 3) * 8)) & 0xffu;
+          const int blk = 2 * (ks & 1) + half;  // block within the 4 loaded
+          const uint32_t sbyte = (sc >> (blk * 8)) & 0xffu;
           uint32_t w16[16];
           const uint32_t s2 = scale_bf16x2(sbyte);
           decode8(cv.x, PL, &w16[0]);
