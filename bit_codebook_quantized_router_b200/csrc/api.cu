@@ -332,3 +332,11 @@ extern "C" int moe_q4_route(const float* logits, int T, int E, int top_k, int32_
   a.inv = inv;
   return q4_launch_route(a, (cudaStream_t)stream);
 }
+
+// Validation + launch of one forward into a workspace the caller already
+// holds; used by the entry point that supplies its own static scratch.
+int q4_forward_in_workspace(const moe_q4_layer* layer, const void* x, const float* logits, int T, int top_k,
+                            void* out, float* out_f32, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return moe_q4_forward(layer, x, logits, T, top_k, out, out_f32, nullptr, nullptr, nullptr, ws, ws_bytes,
+                        (void*)stream);
+}

@@ -52,3 +52,5 @@ int q4_launch_combine(const q4::FwdArgs& a, cudaStream_t s);
 int q4_launch_gather(const q4::FwdArgs& a, cudaStream_t s);
 int q4_launch_prefill(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, cudaStream_t s);
 int q4_prefill_tile_n();
+int q4_forward_in_workspace(const moe_q4_layer* layer, const void* x, const float* logits, int T, int top_k,
+                            void* out, float* out_f32, void* ws, size_t ws_bytes, cudaStream_t stream);

@@ -227,6 +227,32 @@ MOE_Q4_API int moe_q4_forward_stages(const moe_q4_layer* layer, const void* x,
                                      void* ws, size_t ws_bytes, void* stream,
                                      void* const* events, int n_events);
 
+/* ---------------------------------------------------------------------------
+ * moe_q4_forward_noalloc -- moe_q4_forward for callers that cannot allocate
+ * device memory (no workspace argument).  The pages have no counterpart of
+ * this entry point; it exists for callers such as a serving loop that may not
+ * call cudaMalloc once running (an allocation can synchronise the device), or
+ * code that only holds raw device pointers from another framework's allocator.
+ *
+ * The workspace lives in a static device array of the library, 8 MiB, held on
+ * every GPU that loads the library until the process exits.  Sizes whose
+ * workspace (moe_q4_forward_workspace) exceeds it are rejected with
+ * MOE_Q4_ENOTSUP before anything is launched; at the GLM-5.2 layer shape
+ * (H 6144, I 2048, 256 experts, top-8) that admits T <= 23.  The first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress) and
+ * caches it: make that first call before any stream capture.  All calls share
+ * the array; calls that overlap on the GPU race on it, so serialise them.
+ * Arguments as for moe_q4_forward, plus:
+ *   status   optional device int32 (out), NULL to skip: receives the
+ *            forward's device status word (MOE_Q4_OK / MOE_Q4_EDEVICE /
+ *            MOE_Q4_ETIMEOUT) by a stream-ordered device-to-device copy.
+ * No allocation of any kind (no cudaMalloc/cudaFree, no allocating library
+ * routine); the call returns without waiting for the GPU.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API int moe_q4_forward_noalloc(const moe_q4_layer* layer, const void* x,
+                                      const float* logits, int T, int top_k, void* out,
+                                      float* out_f32, int32_t* status, void* stream);
+
 /* Synchronise `stream` and return the int32 at device address `status`
  * (as written by moe_q4_pack), or MOE_Q4_ECUDA. */
 MOE_Q4_API int moe_q4_read_status(const int32_t* status, void* stream);
