@@ -419,10 +419,16 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode_t1", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="layer with this many experts (same H, I, top-k) instead of the workload's; "
+                         "for small profiling captures")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = inputs.WORKLOADS[args.workload]
+    if args.experts:
+        import dataclasses
+        w = dataclasses.replace(w, shape=dataclasses.replace(w.shape, E=args.experts))
     if args.impl == "reference":
         run_reference(args, w)
     else:

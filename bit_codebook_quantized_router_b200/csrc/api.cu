@@ -20,6 +20,17 @@ constexpr int kDecodeMaxRows = 16;
 
 bool uses_prefill(int T) { return T > kDecodeMaxRows; }
 
+// Persistent small-M kernels run at most this many CTAs (one per SM); the
+// workspace holds two split-tile partial slots per CTA.
+constexpr int kDkMaxGrid = 160;
+
+int dk_grid() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 148;
+  return sms < kDkMaxGrid ? sms : kDkMaxGrid;
+}
+
 size_t align_up(size_t v) { return (v + kAlign - 1) & ~(kAlign - 1); }
 
 bool layer_ok(const moe_q4_layer* L) {
@@ -30,6 +41,9 @@ bool layer_ok(const moe_q4_layer* L) {
   const uint8_t* p[3] = {L->gate_w, L->up_w, L->down_w};
   for (auto q : p)
     if ((uintptr_t)q & 15) return false;
+  const uint8_t* sc[3] = {L->gate_s, L->up_s, L->down_s};
+  for (auto q : sc)
+    if ((uintptr_t)q & 7) return false;
   return true;
 }
 
@@ -44,10 +58,13 @@ bool shape_ok(const moe_q4_layer* L, int T, int top_k) {
 //   header int32[64] | ids int32[T*k] | w f32[T*k] | counts int32[E] |
 //   offsets int32[E+1] | row_token int32[T*k] | inv int32[T*k] |
 //   dec_list int32[E] | pre_list int32[E] | tiles int32[E+1] | h bf16[T*k][I] |
-//   h_lo bf16[T*k][I] | y f32[T*k][H] | xg bf16[T*k][H] (only when T > 16:
-//   activation rows in expert order for the tensor-core path)
+//   h_lo bf16[T*k][I] | y f32[T*k][H] | xg bf16[T*k][H] (activation rows in
+//   expert order) | split-tile counters int32[units] | partial sums of the
+//   small-M kernels f32[2*160][3][min(16,T)][128]
 struct Layout {
-  size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, tiles, h, h_lo, y, xg, end;
+  size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, tiles, h, h_lo, y, xg, dk_counter,
+      dk_partial, end;
+  int dk_units_gu, dk_units_dn, n_max;
 };
 
 Layout layout(const moe_q4_layer* L, int T, int k) {
@@ -81,7 +98,15 @@ Layout layout(const moe_q4_layer* L, int T, int k) {
   o.y = p;
   p = align_up(p + sizeof(float) * R * L->H);
   o.xg = p;
-  if (uses_prefill(T)) p = align_up(p + sizeof(__nv_bfloat16) * R * L->H);
+  p = align_up(p + sizeof(__nv_bfloat16) * R * L->H);
+  const int max_exp = (int)(R < (size_t)L->E ? R : (size_t)L->E);
+  o.dk_units_gu = max_exp * (L->I / 128);
+  o.dk_units_dn = max_exp * (L->H / 128);
+  o.n_max = T < 16 ? T : 16;
+  o.dk_counter = p;
+  p = align_up(p + sizeof(int32_t) * (size_t)(o.dk_units_gu + o.dk_units_dn));
+  o.dk_partial = p;
+  p = align_up(p + sizeof(float) * (size_t)2 * kDkMaxGrid * 3 * o.n_max * 128);
   o.end = p;
   return o;
 }
@@ -130,7 +155,9 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   a.dec_list = (int32_t*)(ws + o.dec_list);
   a.pre_list = (int32_t*)(ws + o.pre_list);
   a.tiles = (int32_t*)(ws + o.tiles);
-  a.xg = uses_prefill(T) ? (__nv_bfloat16*)(ws + o.xg) : nullptr;
+  a.xg = (__nv_bfloat16*)(ws + o.xg);
+  a.dk_counter = (int32_t*)(ws + o.dk_counter);
+  a.dk_counter_n = o.dk_units_gu + o.dk_units_dn;
   a.h = (__nv_bfloat16*)(ws + o.h);
   a.h_lo = (__nv_bfloat16*)(ws + o.h_lo);
   a.y = (float*)(ws + o.y);
@@ -154,12 +181,17 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   int rc = mark(0);
   if (rc == MOE_Q4_OK) rc = q4_launch_route(a, s);
   if (rc == MOE_Q4_OK) rc = mark(1);
-  if (rc == MOE_Q4_OK && pre) rc = q4_launch_gather(a, s);
+  const int grid = dk_grid();
+  float* part_gu = (float*)(ws + o.dk_partial);
+  float* part_dn = part_gu + (size_t)2 * kDkMaxGrid * 2 * o.n_max * 128;
+  int32_t* cnt_gu = a.dk_counter;
+  int32_t* cnt_dn = a.dk_counter + o.dk_units_gu;
+  if (rc == MOE_Q4_OK) rc = q4_launch_gather(a, s);
   if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, true, s);
-  if (rc == MOE_Q4_OK) rc = q4_launch_decode(a, tp, true, s);
+  if (rc == MOE_Q4_OK) rc = q4_launch_decode_tc(a, tp, true, part_gu, cnt_gu, grid, s);
   if (rc == MOE_Q4_OK) rc = mark(2);
   if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, false, s);
-  if (rc == MOE_Q4_OK) rc = q4_launch_decode(a, tp, false, s);
+  if (rc == MOE_Q4_OK) rc = q4_launch_decode_tc(a, tp, false, part_dn, cnt_dn, grid, s);
   if (rc == MOE_Q4_OK) rc = mark(3);
   if (rc == MOE_Q4_OK) rc = q4_launch_combine(a, s);
   if (rc == MOE_Q4_OK) rc = mark(4);

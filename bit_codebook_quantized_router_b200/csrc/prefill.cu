@@ -113,12 +113,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full_c[s], 1);
       mbar_init(&full_b[s], 1);
-      mbar_init(&a_ready[s], kDequantThreads);
+      mbar_init(&a_ready[s], kDequantThreads / 32);  // one arrival per dequant warp
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
+      mbar_init(&acc_empty[b], 4);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = d & (kBM - 1);              // weight row in the tile
     const int part = d >> 7;                  // gate/up: matrix; down: K half
     uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
+    for (int tile = blockIdx.x; tile < total && !warp_aborted(abort_flag); tile += gridDim.x) {
       int p, m, nt;
       tile_coords(a, P.m_tiles, np, tile, p, m, nt);
       const int e = a.pre_list[p];
@@ -223,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if ((ks & 1) == 0) sc = *reinterpret_cast<const uint32_t*>(srow + ks * 2);
         const int s = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
-        if (!mbar_wait(&full_c[s], ph, abort_flag, kWaitLimitNs)) {
+        if (!mbar_wait_warp(&full_c[s], ph, abort_flag, kWaitLimitNs)) {
           ok = false;
           break;
         }
@@ -252,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         fence_proxy_async_smem();
-        mbar_arrive(&a_ready[s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_ready[s]);
       }
       if (!ok) break;
     }
@@ -261,14 +262,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3;          // TMEM lanes 32*quad .. +31
     const int row = quad * 32 + lane;   // weight row in the tile
     uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
+    for (int tile = blockIdx.x; tile < total && !warp_aborted(abort_flag); tile += gridDim.x, ++tcount) {
       int p, m, nt;
       tile_coords(a, P.m_tiles, np, tile, p, m, nt);
       const int e = a.pre_list[p];
       const int n_e = a.counts[e];
       const int row0 = a.offsets[e];
       const int buf = tcount & 1;
-      if (!mbar_wait(&acc_full[buf], (tcount >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+      if (!mbar_wait_warp(&acc_full[buf], (tcount >> 1) & 1, abort_flag, kWaitLimitNs)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * (C::kMats * kBN);
       const int wrow = m * kBM + row;
@@ -293,7 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(&acc_empty[buf]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
     }
   }
 

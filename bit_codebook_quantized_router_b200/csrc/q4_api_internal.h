@@ -33,7 +33,9 @@ struct FwdArgs {
   __nv_bfloat16* h_lo;     // [T*k][I] bf16 rounding of the remainder silu(g)*u - h
   float* y;                // [T*k][H]
   float* out_f32;          // optional [T][H] fp32 combine result
-  __nv_bfloat16* xg;       // [T*k][H] expert-grouped activations (tensor-core path)
+  __nv_bfloat16* xg;       // [T*k][H] expert-grouped activations
+  int32_t* dk_counter;     // [dk_counter_n] split-tile arrival counters (small-M path)
+  int dk_counter_n;
   int32_t* user_ids;
   float* user_w;
   int32_t* user_counts;
@@ -47,10 +49,11 @@ int q4_fill_tables(q4::TableParams* tp, const float* tables, int n_tables, const
 
 // Kernel launchers (return MOE_Q4_OK or MOE_Q4_ECUDA).
 int q4_launch_route(const q4::FwdArgs& a, cudaStream_t s);
-int q4_launch_decode(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, cudaStream_t s);
 int q4_launch_combine(const q4::FwdArgs& a, cudaStream_t s);
 int q4_launch_gather(const q4::FwdArgs& a, cudaStream_t s);
 int q4_launch_prefill(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, cudaStream_t s);
 int q4_prefill_tile_n();
+int q4_launch_decode_tc(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, float* partial,
+                        int32_t* counter, int grid, cudaStream_t s);
 int q4_forward_in_workspace(const moe_q4_layer* layer, const void* x, const float* logits, int T, int top_k,
                             void* out, float* out_f32, void* ws, size_t ws_bytes, cudaStream_t stream);

@@ -132,6 +132,8 @@ __device__ void group_rows(const FwdArgs& a, int* sm) {
     counts[e] = 0;
     running[e] = 0;
   }
+  // per-tile arrival counters of the small-M kernels start at zero every call
+  for (int i = tid; i < a.dk_counter_n; i += kRouteThreads) a.dk_counter[i] = 0;
   __syncthreads();
   // ids come from topk_warp and are always < E; a value out of range would be
   // a library bug: record it and leave the row out rather than index past smem.
@@ -250,21 +252,17 @@ __global__ void __launch_bounds__(kRouteThreads) route_group_kernel(const __grid
 }
 
 // Gather the activation rows in expert-grouped order for the tensor-core
-// path: xg[row] = x[row_token[row]] (rows of experts on that path only).
+// GEMMs (both paths read activations by TMA from contiguous rows):
+// xg[row] = x[row_token[row]] for all T*k rows.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant__ FwdArgs a) {
   pdl_wait();
-  const int np = a.hdr[kNumPrefill];
   const int vec_per_row = a.H / 8;  // 16-byte vectors
-  for (int p = blockIdx.y; p < np; p += gridDim.y) {
-    const int e = a.pre_list[p];
-    const int r0 = a.offsets[e], r1 = a.offsets[e + 1];
-    for (int64_t v = blockIdx.x * 256 + threadIdx.x; v < (int64_t)(r1 - r0) * vec_per_row;
-         v += (int64_t)gridDim.x * 256) {
-      const int r = r0 + (int)(v / vec_per_row);
-      const int q = (int)(v % vec_per_row);
-      const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)a.row_token[r] * a.H) + q;
-      reinterpret_cast<uint4*>(a.xg + (size_t)r * a.H)[q] = *src;
-    }
+  const int64_t n = (int64_t)a.T * a.k * vec_per_row;
+  for (int64_t v = blockIdx.x * 256 + threadIdx.x; v < n; v += (int64_t)gridDim.x * 256) {
+    const int r = (int)(v / vec_per_row);
+    const int q = (int)(v % vec_per_row);
+    const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)a.row_token[r] * a.H) + q;
+    reinterpret_cast<uint4*>(a.xg + (size_t)r * a.H)[q] = *src;
   }
   pdl_trigger();
 }
@@ -317,7 +315,9 @@ int q4_launch_gather(const FwdArgs& a, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cfg.gridDim = dim3(64, 64);
+  const long long vecs = (long long)a.T * a.k * (a.H / 8);
+  const long long blocks = (vecs + 255) / 256;
+  cfg.gridDim = dim3((unsigned)(blocks < 148 * 8 ? blocks : 148 * 8));
   cfg.blockDim = dim3(256);
   return cudaLaunchKernelEx(&cfg, gather_rows_kernel, a) == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
 }

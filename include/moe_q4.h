@@ -125,12 +125,12 @@ typedef struct moe_q4_layer {
   int E;                    /* routed experts, 1..MOE_Q4_MAX_EXPERTS */
   int H;                    /* hidden size, % 128 == 0 */
   int I;                    /* expert intermediate size, % 128 == 0 */
-  const uint8_t* gate_w;    /* device [E][I][H/2] */
-  const uint8_t* gate_s;    /* device [E][I][H/32] */
-  const uint8_t* up_w;      /* device [E][I][H/2] */
-  const uint8_t* up_s;      /* device [E][I][H/32] */
-  const uint8_t* down_w;    /* device [E][H][I/2] */
-  const uint8_t* down_s;    /* device [E][H][I/32] */
+  const uint8_t* gate_w;    /* device [E][I][H/2], 16-byte aligned */
+  const uint8_t* gate_s;    /* device [E][I][H/32], 8-byte aligned */
+  const uint8_t* up_w;      /* device [E][I][H/2], 16-byte aligned */
+  const uint8_t* up_s;      /* device [E][I][H/32], 8-byte aligned */
+  const uint8_t* down_w;    /* device [E][H][I/2], 16-byte aligned */
+  const uint8_t* down_s;    /* device [E][H][I/32], 8-byte aligned */
   const float* tables;      /* host [n_tables][8] magnitudes */
   int n_tables;             /* 1..MOE_Q4_MAX_TABLES */
   const uint8_t* table_id;  /* host [E]: table of each expert */

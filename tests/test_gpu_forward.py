@@ -74,6 +74,21 @@ def test_small_layer_edge_counts(T, k, bias):
     gpu_support.check_out(out, ref, f"T={T} k={k}")
 
 
+# K a multiple of 128 but not of 256 (H = I = 384): the small-M path streams
+# 128-K stages of 64-byte code rows, several per tile; T <= 8 and T > 8 take
+# the two activation tile heights of the down projection.
+@pytest.mark.parametrize("T,k", [(1, 2), (5, 2), (9, 1), (24, 3)])
+def test_layer_k_not_multiple_of_256(T, k):
+    w = inputs.Workload("k384", 9, T, inputs.Shape(H=384, I=384, E=8, k=k))
+    L, dev = _small_device_layer(w)
+    x = inputs.activations(w)
+    lg = inputs.router_logits(w)
+    out, ids, _, _ = _run(dev, x.cuda(), lg.cuda(), k)
+    ref, rids, _ = oracle.moe_tokens(L, inputs.bf16_bits(x), lg.numpy(), k, return_routing=True)
+    assert np.array_equal(ids.cpu().numpy(), rids)
+    gpu_support.check_out(out, ref, f"H=I=384 T={T} k={k}")
+
+
 def test_identical_experts_equal_dense_ffn():
     w = inputs.Workload("ident", 8, 24, inputs.TINY)
     L, dev = _small_device_layer(w, identical_to=2)
