@@ -7,8 +7,10 @@ One step = one pass of the whole layer (route -> gate/up + SwiGLU -> down ->
 combine) over one batch of synthetic GLM-5.2-shaped input (hidden 6144,
 intermediate 2048, 256 experts, top-8; 4-bit Lloyd codebook + E8M0/32
 weights).  The default workload is decode at T=1.  Inputs rotate over 8
-seeded batches resident in HBM; L2 is flushed (a 256 MiB write) before every
-timed step, outside the step's own CUDA events.  Prints one JSON line (rank 0).
+seeded batches resident in HBM; L2 is flushed before every timed step, outside
+the step's own CUDA events: a 256 MiB write, then a 256 MiB read of a second
+buffer, so no dirty line of the flush is written back inside the timed region.
+Prints one JSON line (rank 0).
 
 --impl reference times the fp64 CPU oracle on the host cores on the same
 workload, each step a bounded sample (one expert's contribution for one
@@ -53,7 +55,8 @@ def workload_desc(w: inputs.Workload) -> dict:
          "routing": "zipf-skewed" if w.zipf else "uniform random",
          "tables": "lloyd + e2m1 (5 experts)" if w.mixed_tables else "lloyd",
          "inputs": f"{ROTATE} rotating seeded batches, resident in HBM",
-         "l2": "flushed (256 MiB write) before every timed step, outside its events"}
+         "l2": "flushed before every timed step, outside its events: 256 MiB write, then 256 MiB "
+               "read of another buffer (no dirty lines left to write back)"}
     return d
 
 
@@ -277,6 +280,61 @@ def build_device_layer(w):
     return q4.Layer(*parts["gate"], *parts["up"], *parts["down"], tables, tid)
 
 
+# kernels between the forward_stages events, in launch order
+KERNELS = [("route", "routing + grouping", None),
+           ("gather", "gather of activation rows", None),
+           ("gate_up_tc", "tc_gemm_kernel<gate/up> (tensor-core gate/up + SwiGLU)", "tensor"),
+           ("gate_up_small", "dk_kernel<gate/up> (small-M gate/up + SwiGLU)", "hbm"),
+           ("down_tc", "tc_gemm_kernel<down> (tensor-core down)", "tensor"),
+           ("down_small", "dk_kernel<down> (small-M down)", "hbm"),
+           ("combine", "combine", None)]
+SMALL_M_MAX_ROWS = 16
+
+
+def kernel_work(sh: inputs.Shape, T: int, counts) -> dict:
+    """Algorithmic work of each GEMM kernel for one batch, from its routing
+    counts: bytes for the small-M kernels (packed weights of their experts,
+    activation rows read, results written), FLOPs for the tensor-core ones."""
+    gu, dn = expert_bytes(sh)
+    c = np.asarray(counts)
+    small = (c > 0) & (c <= SMALL_M_MAX_ROWS)
+    big = c > SMALL_M_MAX_ROWS
+    rs, rb = int(c[small].sum()), int(c[big].sum())
+    return {"gate_up_small": small.sum() * gu + rs * sh.H * 2 + rs * sh.I * 2 * 2,
+            "down_small": small.sum() * dn + rs * sh.I * 2 * 2 + rs * sh.H * 4,
+            "gate_up_tc": 2.0 * rb * 2 * sh.I * sh.H,
+            "down_tc": 2.0 * rb * sh.H * sh.I}
+
+
+def roofline(work, kern_ms, n_prof, hbm_peak, tf_peak, peak_src):
+    """Achieved rate of every GEMM kernel (algorithmic work / event time,
+    summed over the profiled steps) and the roofline entry of the dominant
+    one (largest total time)."""
+    kernels = {}
+    for j, (key, name, bound) in enumerate(KERNELS):
+        ms = float(kern_ms[:, j].sum())
+        ent = {"name": name, "mean_ms": ms / n_prof}
+        if bound is not None:
+            tot = float(sum(work[i % ROTATE][key] for i in range(n_prof)))
+            if bound == "hbm":
+                ach = tot / (ms / 1e3) / 1e9 if ms > 0 else 0.0
+                ent.update(bound="hbm", achieved=ach, unit="GB/s", peak=hbm_peak, frac=ach / hbm_peak,
+                           algorithmic_per_launch=tot / n_prof)
+            else:
+                ach = tot / (ms / 1e3) / 1e12 if ms > 0 else 0.0
+                ent.update(bound="tensor", achieved=ach, unit="TFLOP/s", peak=tf_peak, frac=ach / tf_peak,
+                           algorithmic_per_launch=tot / n_prof)
+        kernels[key] = ent
+    gemms = [k for k, _, b in KERNELS if b is not None and kernels[k]["algorithmic_per_launch"] > 0]
+    dom = max(gemms, key=lambda k: kernels[k]["mean_ms"])
+    d = kernels[dom]
+    roof = {"kernel": d["name"], "bound": d["bound"], "achieved": d["achieved"], "peak": d["peak"],
+            "unit": d["unit"], "frac": d["frac"], "peak_source": peak_src,
+            "traffic": profile_traffic(dom), "algorithmic_per_launch": d["algorithmic_per_launch"],
+            "launch_ms": d["mean_ms"]}
+    return roof, kernels
+
+
 def run_ours(args, w):
     import torch.distributed as dist
 
@@ -295,14 +353,20 @@ def run_ours(args, w):
     xs = [inputs.activations(w, device="cuda", variant=v) for v in range(ROTATE)]
     lgs = [inputs.router_logits(w, device="cuda", variant=v) for v in range(ROTATE)]
     # distinct experts touched per batch (for the algorithmic bytes)
-    touched = []
+    touched, counts = [], []
     for lg in lgs:
         ids = torch.topk(lg, k, dim=1).indices
         touched.append(int(torch.unique(ids).numel()))
+        counts.append(torch.bincount(ids.reshape(-1), minlength=sh.E).cpu().numpy())
     ws = q4.alloc_workspace(q4.forward_workspace(layer, T, k))
     out = torch.empty((T, sh.H), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    scrub = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+
+    def flush_l2(i):
+        flush.fill_(i & 0xFF)
+        scrub.sum()
 
     def barrier():
         if world > 1:
@@ -319,7 +383,7 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         for i in range(args.steps):
-            flush.fill_(i & 0xFF)
+            flush_l2(i)
             starts[i].record(stream)
             q4.forward(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)
             ends[i].record(stream)
@@ -333,19 +397,18 @@ def run_ours(args, w):
     total_ms = float(tmax.item())
     value = T * args.steps * world / (total_ms / 1e3)
 
-    # stage times (separate pass, events between the kernels)
+    # per-kernel times (separate pass, events between the kernels)
     n_prof = min(args.steps, 100)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_prof)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(n_prof)]
     for row in evs:  # torch creates the CUDA event on first record
         for ev in row:
             ev.record(stream)
     torch.cuda.synchronize()
     for i in range(n_prof):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         q4.forward_stages(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out, ws, evs[i])
     torch.cuda.synchronize()
-    stage_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(4)] for i in range(n_prof)])
-    stage_mean = stage_ms.mean(0)
+    kern_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(7)] for i in range(n_prof)])
     assert q4.forward_status(ws) == 0
 
     # e2e through the host-buffer entry point (pinned host memory)
@@ -360,7 +423,7 @@ def run_ours(args, w):
     e_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e)]
     torch.cuda.synchronize()
     for i in range(n_e2e):
-        flush.fill_(i & 0xFF)
+        flush_l2(i)
         e_s[i].record(stream)
         st = q4.forward_host(layer, xh[i % ROTATE], lh[i % ROTATE], k, oh, wsh)
         e_e[i].record(stream)
@@ -372,31 +435,24 @@ def run_ours(args, w):
         dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
     e2e_value = T * n_e2e * world / (float(e2e_t.item()) / 1e3)
 
-    # roofline of the dominant kernel (gate/up + SwiGLU: the largest byte stream)
     hbm_peak, tf_peak, peak_src = load_peaks()
+    work = [kernel_work(sh, T, c) for c in counts]
+    roof, kernels = roofline(work, kern_ms, n_prof, hbm_peak, tf_peak, peak_src)
     gu, dn = expert_bytes(sh)
-    mean_touched = float(np.mean(touched))
-    R = T * k
-    gu_bytes = mean_touched * gu + T * sh.H * 2 + R * sh.I * 2 * 2
-    gu_ms = float(stage_mean[1])
-    achieved = gu_bytes / (gu_ms / 1e3) / 1e9
-    layer_bytes = mean_touched * (gu + dn) + T * sh.H * 2 * 2
-    kernels_per_step = (1 if T <= 256 else 2) + 3
+    layer_bytes = float(np.mean(touched)) * (gu + dn) + T * sh.H * 2 * 2
+    # our kernels per forward: route (1 fused for T <= 256, else 2), gather,
+    # small-M gate/up and down, combine, and the two tensor-core GEMMs for T > 16
+    kernels_per_step = (1 if T <= 256 else 2) + 4 + (2 if T > 16 else 0)
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_desc(w), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
-        "roofline": {"kernel": "decode gate/up + SwiGLU (packed 4-bit stream, mma.sync)", "bound": "hbm",
-                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
-                     "peak_source": peak_src, "traffic": profile_traffic("decode_gateup"),
-                     "algorithmic_bytes_per_launch": gu_bytes, "launch_ms": gu_ms},
-        "stages_ms": {"route": float(stage_mean[0]), "gate_up": float(stage_mean[1]),
-                      "down": float(stage_mean[2]), "combine": float(stage_mean[3])},
-        "layer_hbm": {"touched_experts": mean_touched, "bytes_per_step": layer_bytes,
+        "roofline": roof,
+        "kernels": kernels,
+        "layer_hbm": {"touched_experts": float(np.mean(touched)), "bytes_per_step": layer_bytes,
                       "gbs": layer_bytes / (total_ms / args.steps / 1e3) / 1e9,
-                      "frac_of_peak": layer_bytes / (total_ms / args.steps / 1e3) / 1e9 / hbm_peak,
-                      "frac_of_8tbs": layer_bytes / (total_ms / args.steps / 1e3) / 8e12},
+                      "frac_of_peak": layer_bytes / (total_ms / args.steps / 1e3) / 1e9 / hbm_peak},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * sh.H * 2 + T * sh.E * 4,
                 "d2h_bytes_per_step": T * sh.H * 2},
         "gpu_launches": kernels_per_step * args.steps,

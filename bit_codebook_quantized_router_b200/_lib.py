@@ -221,7 +221,7 @@ def route(logits: torch.Tensor, k: int, stream=None):
 
 
 def forward_stages(layer: Layer, x, logits, k: int, out, ws, events, stream=None) -> None:
-    """moe_q4_forward with torch.cuda.Event records at the 5 stage boundaries
+    """moe_q4_forward with torch.cuda.Event records at the 8 kernel boundaries
     (the events must have been recorded once: torch creates them lazily)."""
     arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
     st = layer.struct()

@@ -187,14 +187,17 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   int32_t* cnt_gu = a.dk_counter;
   int32_t* cnt_dn = a.dk_counter + o.dk_units_gu;
   if (rc == MOE_Q4_OK) rc = q4_launch_gather(a, s);
-  if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, true, s);
-  if (rc == MOE_Q4_OK) rc = q4_launch_decode_tc(a, tp, true, part_gu, cnt_gu, grid, s);
   if (rc == MOE_Q4_OK) rc = mark(2);
-  if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, false, s);
-  if (rc == MOE_Q4_OK) rc = q4_launch_decode_tc(a, tp, false, part_dn, cnt_dn, grid, s);
+  if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, true, s);
   if (rc == MOE_Q4_OK) rc = mark(3);
-  if (rc == MOE_Q4_OK) rc = q4_launch_combine(a, s);
+  if (rc == MOE_Q4_OK) rc = q4_launch_decode(a, tp, true, part_gu, cnt_gu, grid, s);
   if (rc == MOE_Q4_OK) rc = mark(4);
+  if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, false, s);
+  if (rc == MOE_Q4_OK) rc = mark(5);
+  if (rc == MOE_Q4_OK) rc = q4_launch_decode(a, tp, false, part_dn, cnt_dn, grid, s);
+  if (rc == MOE_Q4_OK) rc = mark(6);
+  if (rc == MOE_Q4_OK) rc = q4_launch_combine(a, s);
+  if (rc == MOE_Q4_OK) rc = mark(7);
   return rc;
 }
 
@@ -267,8 +270,8 @@ extern "C" int moe_q4_forward(const moe_q4_layer* layer, const void* x, const fl
 extern "C" int moe_q4_forward_stages(const moe_q4_layer* layer, const void* x, const float* logits,
                                      int T, int top_k, void* out, void* ws, size_t ws_bytes,
                                      void* stream, void* const* events, int n_events) {
-  if (!events || n_events < 5) return MOE_Q4_EINVAL;
-  for (int i = 0; i < 5; ++i)
+  if (!events || n_events < 8) return MOE_Q4_EINVAL;
+  for (int i = 0; i < 8; ++i)
     if (!events[i]) return MOE_Q4_EINVAL;
   if (!shape_ok(layer, T, top_k)) return MOE_Q4_EINVAL;
   TableParams tp;

@@ -1,0 +1,682 @@
+// Small-M ("decode") expert GEMMs: the packed weights of experts with at most
+// 16 rows, streamed from HBM once per call and decoded straight into MMA
+// operand registers.
+//
+//   gate/up: h[row] = silu(W_gate x) * (W_up x)
+//   down:    y[row] = W_down h[row]
+// ("Round 7 -- Rewrite the GLM-5.2 routed-expert encoder", "Owner-locked
+// decisions" 4 and 6.)
+//
+// * Work split.  A unit is (expert on this path, tile of 128 weight rows);
+//   the units' stages (256 weights of K each, 128 if K % 256 != 0) form one
+//   sequence that the persistent CTAs (one per SM) cut into equal contiguous
+//   ranges, so every SM streams the same number of bytes.  A tile whose K
+//   range spans several CTAs is finished by the last of them to arrive (a
+//   per-tile counter): it adds the partial sums in K order (deterministic)
+//   and writes the result.
+// * Data movement (warp 0): per stage and matrix one TMA brings 128 weight
+//   rows x 128 bytes of codes (a full 128-byte line per row: narrower boxes
+//   stream at a fraction of HBM bandwidth) with the 128-byte swizzle; TMA
+//   brings the expert's activation rows; the warp's lanes copy each row's
+//   scale bytes for the stage with cp.async, completing on the stage barrier.
+// * Decode + MMA (warps 1..16): warp (slab s, half J) owns weight rows
+//   16s..16s+15 of the tile and the J-th 128-K half of every stage.  Lane
+//   (g, t) reads the 16-byte code chunk t of rows g and g+8 (32 weights, one
+//   E8M0 block), decodes it to bf16 pairs ("aidendle94/GLM-5.2-NF4-Lloyd-
+//   Experts-GPTQ", "Codes are indices into the per-layer grid") and feeds
+//   them to mma.sync m16n8k16 as the A operand.  K is permuted inside each
+//   128-K half, the same way for weights and activations (a sum over K does
+//   not depend on its order): MMA m takes from lane t the pairs at K offsets
+//   32t + 2m and 32t + 16 + 2m, so every lane's operands come from its own
+//   code chunk and one 64-byte run of each activation row.  Decoding mixes a
+//   shared-memory table byte -> signed bf16 pair (one copy per lane: a warp's
+//   32 lookups hit 32 banks) with the in-register PRMT decode, balancing the
+//   integer pipe against shared-memory bandwidth; the block scale is one
+//   exact bf16x2 multiply.
+//   With N <= 16 token columns tcgen05.mma (A in TMEM) passes 2048 weights
+//   per instruction at about 50 cycles; mma.sync sustains 0.5 instructions
+//   per cycle per SM, 128 weights per cycle, and needs no copy of the decoded
+//   weights to TMEM or shared memory: this path is bound by HBM, not by
+//   tensor math, so it takes the faster of the two.
+// * Token columns: gate/up 8 per n-tile (NT = 1 or 2 tiles); down multiplies
+//   by h and by its low part h_lo (y = W h + W h_lo): with T <= 4 one n-tile
+//   holds h in columns 0..3 and h_lo in 4..7, else separate tiles accumulate
+//   into the same registers.
+// * The two K halves of a slab are added through shared memory (J = 0 + J =
+//   1), then warp (s, 0) finishes: SwiGLU and h / h_lo, or y, or a partial.
+//
+// Every wait is bounded (a timeout sets MOE_Q4_ETIMEOUT in the status word and
+// the CTA drains and exits); warps wait and leave together (vote).
+#include <cuda.h>
+
+#include "q4_api_internal.h"
+#include "q4_common.cuh"
+#include "sm100.cuh"
+
+namespace q4 {
+
+using namespace sm100;
+
+namespace dk {
+constexpr int kComputeWarps = 16;                    // 8 slabs x 2 K halves
+constexpr int kThreads = 32 * (1 + kComputeWarps);   // + the producer warp
+constexpr int kRows = 128;                           // weight rows per tile
+constexpr int kMaxRing = 6;                          // shared-memory stages, at most
+constexpr int kPrmtWords = 2;                        // of the 4 words of a chunk, decoded in registers
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint32_t kLutBytes = 65536;  // 256 entries x (2 table slots x 32 lanes x 4 B)
+constexpr uint32_t kScaleSlot = 8;     // scale bytes per row per stage (4 used for 128-K stages)
+constexpr uint32_t kBarBytes = 1024;   // barriers and flags
+}  // namespace dk
+
+template <bool GATEUP, int NT>
+struct DkCfg {
+  static constexpr int kMats = GATEUP ? 2 : 1;
+  // 1-KB activation atoms (8 rows x 128 B, 128-byte swizzle) per 64-K super-step
+  static constexpr int kAtoms = GATEUP ? NT : (NT == 4 ? 4 : 2);
+  // 8-token groups of the result
+  static constexpr int kTT = GATEUP ? NT : (NT == 4 ? 2 : 1);
+  static constexpr int kAcc = kMats * kTT * 4;  // accumulator floats per lane
+};
+
+// Shared-memory placement (addresses in the CTA's shared window).  The table
+// sits at a 64 KB boundary so its entry addresses can be formed by one PRMT;
+// the activation and scale rings, the exchange area and the barriers go below
+// it when the gap holds them, the code ring above it.  Host and device
+// compute the same placement from the window's start `raw`.
+struct DkLayout {
+  uint32_t lut, codes, x, scales, xch, bars, end;
+};
+
+__host__ __device__ inline DkLayout dk_layout(uint32_t raw, uint32_t code_stage, uint32_t x_stage,
+                                              uint32_t scale_stage, uint32_t xch_bytes, int ring) {
+  DkLayout L;
+  L.lut = (raw + 65535u) & ~65535u;
+  L.codes = L.lut + dk::kLutBytes;
+  const uint32_t codes_end = L.codes + (uint32_t)ring * code_stage;
+  const uint32_t others = (uint32_t)ring * (x_stage + scale_stage) + xch_bytes + dk::kBarBytes;
+  const uint32_t o = (raw + 1023u) & ~1023u;
+  if (o + others <= L.lut) {
+    L.x = o;
+    L.end = codes_end;
+  } else {
+    L.x = codes_end;
+    L.end = codes_end + others;
+  }
+  L.scales = L.x + (uint32_t)ring * x_stage;
+  L.xch = L.scales + (uint32_t)ring * scale_stage;
+  L.bars = L.xch + xch_bytes;
+  return L;
+}
+
+struct DkParams {
+  FwdArgs a;
+  int tiles_per_e;  // weight rows / 128
+  int subs;         // 64-K super-steps per stage: 4 (K % 256 == 0) or 2
+  int stages;       // stages per tile: K / (64 * subs)
+  int ring;         // shared-memory stages
+  int n_max;        // token columns kept in partial sums: min(16, T)
+  uint32_t code_stage, x_stage, scale_stage, xch_bytes;
+  float* partial;   // [2 * gridDim.x][mats][n_max][128]
+  int32_t* counter; // [units], zero at launch
+};
+
+__device__ __forceinline__ long long dk_range(int b, long long total, int G) { return (long long)b * total / G; }
+
+// CTA whose range holds stage g.
+__device__ __forceinline__ int dk_owner(long long g, long long total, int G) {
+  int b = (int)((g * G) / total);
+  while (b + 1 < G && dk_range(b + 1, total, G) <= g) ++b;
+  while (b > 0 && dk_range(b, total, G) > g) --b;
+  return b;
+}
+
+// CTAs holding part of [us, ue): the owners of its ends and every non-empty
+// range between them (with fewer stages than CTAs some ranges are empty).
+__device__ __forceinline__ int dk_contributors(long long us, long long ue, long long total, int G, int& c_first,
+                                               int& c_last) {
+  c_first = dk_owner(us, total, G);
+  c_last = dk_owner(ue - 1, total, G);
+  int n = 0;
+  for (int c = c_first; c <= c_last; ++c) n += dk_range(c + 1, total, G) > dk_range(c, total, G);
+  return n;
+}
+
+__device__ __forceinline__ void ring_next(int& s, uint32_t& ph, int n) {
+  if (++s == n) {
+    s = 0;
+    ph ^= 1u;
+  }
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  return v;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 v;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  return v;
+}
+
+// 16 bf16 pairs of one code chunk (4 words, pair 4w + b from byte b of word
+// w), scaled: words below kPrmtWords by the PRMT decode, the rest by table.
+__device__ __forceinline__ void decode_chunk(const uint4 c, const Planes& PL, uint32_t kreg, uint32_t scale2,
+                                             uint32_t p[16]) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (i < dk::kPrmtWords) {
+      decode8(w[i], PL, &p[4 * i]);
+    } else {
+      // table entry address = table | byte << 8 | slot << 7 | lane << 2
+      p[4 * i + 0] = lds32(prmt(w[i], kreg, 0x7604));
+      p[4 * i + 1] = lds32(prmt(w[i], kreg, 0x7614));
+      p[4 * i + 2] = lds32(prmt(w[i], kreg, 0x7624));
+      p[4 * i + 3] = lds32(prmt(w[i], kreg, 0x7634));
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) p[i] = bf16x2_mul(p[i], scale2);
+}
+
+template <bool GATEUP, int NT>
+__global__ void __launch_bounds__(dk::kThreads, 1)
+    dk_kernel(const __grid_constant__ DkParams P, const __grid_constant__ TableParams tp,
+              const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
+              const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xl) {
+  using C = DkCfg<GATEUP, NT>;
+  constexpr int kMats = C::kMats;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const DkLayout Ls = dk_layout(raw_s, P.code_stage, P.x_stage, P.scale_stage, P.xch_bytes, P.ring);
+  const FwdArgs& a = P.a;
+  if (Ls.end > raw_s + dynamic_smem_size()) {  // launched with less shared memory than the layout needs
+    if (threadIdx.x == 0) record_error(a.hdr + kStatus, MOE_Q4_ECUDA);
+    return;
+  }
+  uint8_t* lut = smem_raw + (Ls.lut - raw_s);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + (Ls.bars - raw_s));
+  uint64_t* full = bars;                          // [ring] codes + activations (TMA), scales (cp.async)
+  uint64_t* stage_empty = full + dk::kMaxRing;    // [ring] compute warps done with the stage
+  uint64_t* xfull = stage_empty + dk::kMaxRing;   // [8] K half 1 of slab s written to the exchange area
+  uint64_t* xfree = xfull + 8;                    // [8] ... and read by K half 0
+  uint64_t* lut_bar = xfree + 8;                  // compute threads rebuilding a table slot
+  uint64_t* epi_bar = lut_bar + 1;                // K-half-0 threads finishing a split tile
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(epi_bar + 1);
+  volatile int* last_flag = abort_flag + 1;
+
+  const int ring = P.ring;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ring; ++s) {
+      mbar_init(&full[s], 1 + 32);  // producer lane 0 (with the TMA bytes) + 32 cp.async arrivals
+      mbar_init(&stage_empty[s], dk::kComputeWarps);
+    }
+    for (int s = 0; s < 8; ++s) {
+      mbar_init(&xfull[s], 32);
+      mbar_init(&xfree[s], 32);
+    }
+    mbar_init(lut_bar, 32 * dk::kComputeWarps);
+    mbar_init(epi_bar, 32 * 8);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tmap(&tm_wa);
+    if (GATEUP) prefetch_tmap(&tm_wb);
+    prefetch_tmap(&tm_x);
+    if (!GATEUP) prefetch_tmap(&tm_xl);
+  }
+  __syncthreads();
+
+  pdl_wait();
+  const int n_dec = a.hdr[kNumDecode];
+  const int rows_total = GATEUP ? a.I : a.H;
+  const int K = GATEUP ? a.H : a.I;
+  const int subs = P.subs;
+  const int row_bytes = 32 * subs;  // code bytes per row per stage
+  const long long total = (long long)n_dec * P.tiles_per_e * P.stages;
+  const int G = gridDim.x, b = blockIdx.x;
+  const long long k0 = dk_range(b, total, G), k1 = dk_range(b + 1, total, G);
+
+  if (warp == 0) {
+    // ------------------------------ producer ------------------------------
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (long long g = k0; g < k1 && ok;) {
+      const int unit = (int)(g / P.stages);
+      const int st0 = (int)(g - (long long)unit * P.stages);
+      const long long seg_end = min(k1, (long long)(unit + 1) * P.stages);
+      const int e = a.dec_list[unit / P.tiles_per_e];
+      const int t = unit % P.tiles_per_e;
+      const int row0 = a.offsets[e];
+      const int wrow = e * rows_total + t * dk::kRows;
+      for (int st = st0; st < st0 + (int)(seg_end - g); ++st) {
+        if (!mbar_wait_warp(&stage_empty[s], ph ^ 1, abort_flag, dk::kWaitNs)) {
+          ok = false;
+          break;
+        }
+        // scale bytes of the stage (2 per 64-K super-step) for 4 rows per lane
+#pragma unroll
+        for (int m = 0; m < kMats; ++m) {
+          const uint8_t* sbase = (GATEUP ? (m ? a.up_s : a.gate_s) : a.down_s) + (size_t)wrow * (K / 32) +
+                                 (size_t)st * 2 * subs;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int r = lane + 32 * j;
+            const uint32_t dst =
+                Ls.scales + (uint32_t)s * P.scale_stage + (uint32_t)(m * dk::kRows + r) * dk::kScaleSlot;
+            if (subs == 4)
+              cp_async_small<8>(dst, sbase + (size_t)r * (K / 32));
+            else
+              cp_async_small<4>(dst, sbase + (size_t)r * (K / 32));
+          }
+        }
+        cp_async_arrive_noinc(&full[s]);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes + subs * C::kAtoms * 1024);
+          uint8_t* cdst = smem_raw + (Ls.codes - raw_s) + (size_t)s * P.code_stage;
+          tma_load_2d(cdst, &tm_wa, &full[s], st * row_bytes, wrow);
+          if (GATEUP) tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
+          // the expert's activation rows, grouped; rows past n_e belong to the next
+          // expert or lie outside the array: they only feed columns nobody writes
+          uint8_t* xdst = smem_raw + (Ls.x - raw_s) + (size_t)s * P.x_stage;
+          for (int j = 0; j < subs; ++j) {
+            const int kx = (st * subs + j) * 64;
+            uint8_t* d = xdst + j * C::kAtoms * 1024;
+            if (GATEUP) {
+              tma_load_2d(d, &tm_x, &full[s], kx, row0);  // 8 * NT rows
+            } else if (NT == 1) {
+              tma_load_2d(d, &tm_x, &full[s], kx, row0);             // h rows 0..3 at atom rows 0..3
+              tma_load_2d(d + 1024, &tm_xl, &full[s], kx, row0 - 4);  // h_lo rows 0..3 at atom rows 4..7
+            } else {
+              tma_load_2d(d, &tm_x, &full[s], kx, row0);                         // h: NT / 2 atoms
+              tma_load_2d(d + (NT / 2) * 1024, &tm_xl, &full[s], kx, row0);      // h_lo
+            }
+          }
+        }
+        __syncwarp();
+        ring_next(s, ph, ring);
+      }
+      g = seg_end;
+    }
+  } else {
+    // ------------------------------ compute ------------------------------
+    const int cw = warp - 1;       // 0..15
+    const int slab = cw & 7;       // rows 16 slab .. + 15 of the tile
+    const int J = cw >> 3;         // 128-K half of each stage
+    const int gq = lane >> 2;      // MMA group: rows gq, gq + 8; token column gq
+    const int tq = lane & 3;       // code chunk of the half; token columns 2tq, 2tq + 1
+    const int ctid = threadIdx.x - 32;
+    const bool active = 2 * J < subs;  // a 128-K stage has one half only
+    const int r0 = 16 * slab + gq, r1 = r0 + 8;
+    const int swz0 = subs == 4 ? (r0 & 7) : ((r0 >> 1) & 3);
+    const int swz1 = subs == 4 ? (r1 & 7) : ((r1 >> 1) & 3);
+    const int chunk = 4 * J + tq;  // 16-byte chunk of the stage row
+    const uint32_t coff0 = (uint32_t)(r0 * row_bytes + ((chunk ^ swz0) << 4));
+    const uint32_t coff1 = (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4));
+    // activation run of this lane: super-step 2J + (tq >> 1), chunks 4 (tq & 1) .. +3
+    const uint32_t xss = (uint32_t)(2 * J + (tq >> 1)) * C::kAtoms * 1024;
+    int slot_tab0 = -1, slot_tab1 = -1, victim = 0;
+    uint32_t lgen = 0, xgen = 0, egen = 0;
+    const uint32_t lane_k = (Ls.lut & 0xffff0000u) | ((uint32_t)lane << 2);
+    int s = 0;
+    uint32_t ph = 0;
+    bool ok = true;
+    for (long long g = k0; g < k1 && ok;) {
+      const int unit = (int)(g / P.stages);
+      const long long ustart = (long long)unit * P.stages, uend = ustart + P.stages;
+      const long long seg_end = min(k1, uend);
+      const int nst = (int)(seg_end - g);
+      const int e = a.dec_list[unit / P.tiles_per_e];
+      const int tile = unit % P.tiles_per_e;
+      const int tid = tp.id[e];
+      int slot = tid == slot_tab0 ? 0 : (tid == slot_tab1 ? 1 : -1);
+      if (slot < 0) {
+        // (re)build a slot: entry c -> bf16 pair of codes (c & 15, c >> 4), signed,
+        // unscaled, one copy per lane.  Bounded barriers on both sides: every
+        // compute thread is done with the old contents before any write, and all
+        // writes land before anyone reads.
+        mbar_arrive(lut_bar);
+        if (!mbar_wait_warp(lut_bar, lgen & 1, abort_flag, dk::kWaitNs)) break;
+        ++lgen;
+        slot = victim;
+        victim ^= 1;
+        if (slot == 0)
+          slot_tab0 = tid;
+        else
+          slot_tab1 = tid;
+        const float* tv = tp.t[tid];
+        const uint32_t ent = ctid & 255, half = ctid >> 8;
+        const uint32_t lo = ent & 15, hi = ent >> 4;
+        const uint32_t blo = (uint32_t)bf16_bits_rn(tv[lo & 7]) ^ ((lo & 8) ? 0x8000u : 0u);
+        const uint32_t bhi = (uint32_t)bf16_bits_rn(tv[hi & 7]) ^ ((hi & 8) ? 0x8000u : 0u);
+        const uint32_t word = blo | (bhi << 16);
+        uint4* dst = reinterpret_cast<uint4*>(lut + ent * 256 + slot * 128 + half * 64);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(word, word, word, word);
+        mbar_arrive(lut_bar);
+        if (!mbar_wait_warp(lut_bar, lgen & 1, abort_flag, dk::kWaitNs)) break;
+        ++lgen;
+      }
+      const uint32_t kreg = lane_k | ((uint32_t)slot << 7);
+      const Planes PL = make_planes(tp.t[tid]);
+
+      float acc[kMats][C::kTT][4];
+#pragma unroll
+      for (int m = 0; m < kMats; ++m)
+#pragma unroll
+        for (int tt = 0; tt < C::kTT; ++tt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[m][tt][i] = 0.0f;
+
+      for (int j = 0; j < nst && ok; ++j) {
+        if (!mbar_wait_warp(&full[s], ph, abort_flag, dk::kWaitNs)) {
+          ok = false;
+          break;
+        }
+        if (active) {
+          const uint32_t cbase = Ls.codes + (uint32_t)s * P.code_stage;
+          const uint32_t sbase = Ls.scales + (uint32_t)s * P.scale_stage;
+          const uint32_t xbase = Ls.x + (uint32_t)s * P.x_stage + xss;
+          // activation operands: 16 pairs per n-tile, pair m at K offset 32 tq + 2m
+          uint32_t xr[NT][16];
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            int atom, row;
+            if (GATEUP) {
+              atom = nt;
+              row = gq;
+            } else if (NT == 1) {
+              atom = gq >> 2;  // h at rows 0..3 of atom 0, h_lo at rows 4..7 of atom 1
+              row = gq;
+            } else {
+              atom = nt;
+              row = gq;
+            }
+            const uint32_t rb = xbase + (uint32_t)atom * 1024 + (uint32_t)row * 128;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint4 v = lds128(rb + ((((tq & 1) * 4 + c) ^ row) << 4));
+              xr[nt][4 * c + 0] = v.x;
+              xr[nt][4 * c + 1] = v.y;
+              xr[nt][4 * c + 2] = v.z;
+              xr[nt][4 * c + 3] = v.w;
+            }
+          }
+#pragma unroll
+          for (int m = 0; m < kMats; ++m) {
+            const uint32_t mb = cbase + (uint32_t)(m * dk::kRows * row_bytes);
+            const uint4 c0 = lds128(mb + coff0);
+            const uint4 c1 = lds128(mb + coff1);
+            const uint2 s0 = lds64(sbase + (uint32_t)((m * dk::kRows + r0) * dk::kScaleSlot));
+            const uint2 s1 = lds64(sbase + (uint32_t)((m * dk::kRows + r1) * dk::kScaleSlot));
+            // E8M0 byte of block 4J + tq
+            const uint32_t e0 = ((J ? s0.y : s0.x) >> (8 * tq)) & 0xffu;
+            const uint32_t e1 = ((J ? s1.y : s1.x) >> (8 * tq)) & 0xffu;
+            uint32_t pa[16], pb[16];
+            decode_chunk(c0, PL, kreg, scale_bf16x2(e0), pa);
+            decode_chunk(c1, PL, kreg, scale_bf16x2(e1), pb);
+#pragma unroll
+            for (int mm = 0; mm < 8; ++mm) {
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                const int tt = GATEUP ? nt : (NT == 4 ? (nt & 1) : 0);
+                mma_16816(acc[m][tt], pa[mm], pb[mm], pa[mm + 8], pb[mm + 8], xr[nt][mm], xr[nt][mm + 8]);
+              }
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&stage_empty[s]);
+        ring_next(s, ph, ring);
+      }
+      if (!ok) break;
+
+      // ---- segment end: add the K halves (J = 1 into J = 0) ----
+      float* xch = reinterpret_cast<float*>(smem_raw + (Ls.xch - raw_s)) + (size_t)slab * C::kAcc * 32;
+      if (J == 1) {
+        if (xgen > 0 && !mbar_wait_warp(&xfree[slab], (xgen - 1) & 1, abort_flag, dk::kWaitNs)) break;
+#pragma unroll
+        for (int m = 0; m < kMats; ++m)
+#pragma unroll
+          for (int tt = 0; tt < C::kTT; ++tt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xch[((m * C::kTT + tt) * 4 + i) * 32 + lane] = acc[m][tt][i];
+        mbar_arrive(&xfull[slab]);
+        ++xgen;
+        g = seg_end;
+        continue;
+      }
+      if (!mbar_wait_warp(&xfull[slab], xgen & 1, abort_flag, dk::kWaitNs)) break;
+#pragma unroll
+      for (int m = 0; m < kMats; ++m)
+#pragma unroll
+        for (int tt = 0; tt < C::kTT; ++tt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[m][tt][i] += xch[((m * C::kTT + tt) * 4 + i) * 32 + lane];
+      mbar_arrive(&xfree[slab]);
+      ++xgen;
+      if (!GATEUP && NT == 1) {
+        // columns 4..7 hold W h_lo for tokens 0..3: add them to columns 0..3
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[0][0][i] += __shfl_xor_sync(0xffffffffu, acc[0][0][i], 2);
+      }
+
+      // ---- K half 0 finishes the slab: token n = 8 tt + 2 tq + (i & 1), row r0 / r1 ----
+      const int row0 = a.offsets[e], n_e = a.counts[e];
+      const bool final_here = (g == ustart && seg_end == uend);
+      if (!final_here) {
+        // partial: slot 2b (segment starts this CTA's range) or 2b+1 (its last)
+        const int pslot = (g == k0) ? 2 * b : 2 * b + 1;
+        float* pp = P.partial + (size_t)pslot * kMats * P.n_max * dk::kRows;
+#pragma unroll
+        for (int m = 0; m < kMats; ++m)
+#pragma unroll
+          for (int tt = 0; tt < C::kTT; ++tt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int n = 8 * tt + 2 * tq + (i & 1);
+              if (n < P.n_max) pp[(m * P.n_max + n) * dk::kRows + ((i >> 1) ? r1 : r0)] = acc[m][tt][i];
+            }
+        __threadfence();
+        mbar_arrive(epi_bar);
+        if (!mbar_wait_warp(epi_bar, egen & 1, abort_flag, dk::kWaitNs)) break;
+        ++egen;
+        if (slab == 0 && lane == 0) {
+          int c_first, c_last;
+          const int n_contrib = dk_contributors(ustart, uend, total, G, c_first, c_last);
+          const int old = atomicAdd(&P.counter[unit], 1);
+          *last_flag = (old == n_contrib - 1) ? 1 : 0;
+        }
+        mbar_arrive(epi_bar);
+        if (!mbar_wait_warp(epi_bar, egen & 1, abort_flag, dk::kWaitNs)) break;
+        ++egen;
+        if (!*last_flag) {
+          g = seg_end;
+          continue;
+        }
+        __threadfence();
+        // last arrival: add the partials of every CTA on this tile in K order
+        int c_first, c_last;
+        dk_contributors(ustart, uend, total, G, c_first, c_last);
+#pragma unroll
+        for (int m = 0; m < kMats; ++m)
+#pragma unroll
+          for (int tt = 0; tt < C::kTT; ++tt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[m][tt][i] = 0.0f;
+        for (int c = c_first; c <= c_last; ++c) {
+          if (dk_range(c + 1, total, G) == dk_range(c, total, G)) continue;  // empty range
+          const int sl = (c == c_first && dk_range(c, total, G) != ustart) ? 2 * c + 1 : 2 * c;
+          const float* qp = P.partial + (size_t)sl * kMats * P.n_max * dk::kRows;
+#pragma unroll
+          for (int m = 0; m < kMats; ++m)
+#pragma unroll
+            for (int tt = 0; tt < C::kTT; ++tt)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int n = 8 * tt + 2 * tq + (i & 1);
+                if (n < P.n_max) acc[m][tt][i] += __ldcg(qp + (m * P.n_max + n) * dk::kRows + ((i >> 1) ? r1 : r0));
+              }
+        }
+      }
+      // finished slab: h (gate/up, as the bf16 pair h, h_lo) or y (down)
+#pragma unroll
+      for (int tt = 0; tt < C::kTT; ++tt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int n = 8 * tt + 2 * tq + (i & 1);
+          if (n >= n_e) continue;
+          const size_t row = (size_t)row0 + n;
+          const int wr = tile * dk::kRows + ((i >> 1) ? r1 : r0);
+          if (GATEUP) {
+            const float hv = silu_mul(acc[0][tt][i], acc[kMats - 1][tt][i]);
+            const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
+            a.h[row * a.I + wr] = hb;
+            a.h_lo[row * a.I + wr] = __float2bfloat16_rn(hv - __bfloat162float(hb));
+          } else {
+            a.y[row * a.H + wr] = acc[0][tt][i];
+          }
+        }
+      g = seg_end;
+    }
+  }
+
+  // ------------------------------ teardown ------------------------------
+  __syncthreads();
+  if (threadIdx.x == 0 && *abort_flag) record_error(a.hdr + kStatus, MOE_Q4_ETIMEOUT);
+  if (warp == 0 && *abort_flag) {
+    // copies still in flight land before the CTA's shared memory goes away
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (lane == 0)
+      for (int s = 0; s < ring; ++s)
+        for (uint32_t par = 0; par < 2; ++par) {
+          volatile int quick = 0;
+          mbar_wait(&full[s], par, &quick, 20000000ull);
+        }
+  }
+  __syncthreads();
+  pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn dk_encode() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+static bool dk_map(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t cols,
+                   uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = dk_encode();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool GATEUP, int NT>
+static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, int32_t* counter, int grid,
+                     cudaStream_t s) {
+  using C = DkCfg<GATEUP, NT>;
+  DkParams P;
+  P.a = a;
+  const int K = GATEUP ? a.H : a.I;
+  P.tiles_per_e = (GATEUP ? a.I : a.H) / dk::kRows;
+  P.subs = (K % 256 == 0) ? 4 : 2;  // K % 128 == 0 always
+  P.stages = K / (64 * P.subs);
+  P.n_max = a.T < 16 ? a.T : 16;
+  P.code_stage = (uint32_t)(C::kMats * dk::kRows * 32 * P.subs);
+  P.x_stage = (uint32_t)(P.subs * C::kAtoms * 1024);
+  P.scale_stage = (uint32_t)(C::kMats * dk::kRows * dk::kScaleSlot);
+  P.xch_bytes = (uint32_t)(8 * C::kAcc * 32 * sizeof(float));
+  P.partial = partial;
+  P.counter = counter;
+
+  // deepest ring that fits; the dynamic window starts after the reserved bytes
+  // (the kernel has no static shared memory)
+  int dev = 0, reserved = 1024, optin = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  P.ring = 0;
+  uint32_t smem = 0;
+  for (int rs = dk::kMaxRing; rs >= 2 && !P.ring; --rs) {
+    const DkLayout L = dk_layout((uint32_t)reserved, P.code_stage, P.x_stage, P.scale_stage, P.xch_bytes, rs);
+    if (L.end - (uint32_t)reserved <= (uint32_t)optin) {
+      P.ring = rs;
+      smem = L.end - (uint32_t)reserved;
+    }
+  }
+  if (!P.ring) return MOE_Q4_ECUDA;
+
+  const int R = a.T * a.k;
+  const CUtensorMapSwizzle csw = P.subs == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const uint32_t cbox = 32u * P.subs;
+  const uint32_t xrows = GATEUP ? 8u * NT : (NT == 4 ? 16u : 8u);
+  CUtensorMap twa, twb, tx, txl;
+  bool ok;
+  if (GATEUP) {
+    ok = dk_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.gate_w, a.H / 2, (uint64_t)a.E * a.I, cbox, dk::kRows, csw) &&
+         dk_map(&twb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.up_w, a.H / 2, (uint64_t)a.E * a.I, cbox, dk::kRows, csw) &&
+         dk_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.xg, a.H, R, 64, xrows, CU_TENSOR_MAP_SWIZZLE_128B);
+    txl = tx;
+  } else {
+    ok = dk_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.down_w, a.I / 2, (uint64_t)a.E * a.H, cbox, dk::kRows,
+                csw) &&
+         dk_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.h, a.I, R, 64, xrows, CU_TENSOR_MAP_SWIZZLE_128B) &&
+         dk_map(&txl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.h_lo, a.I, R, 64, xrows, CU_TENSOR_MAP_SWIZZLE_128B);
+    twb = twa;
+  }
+  if (!ok) return MOE_Q4_ECUDA;
+  if (cudaFuncSetAttribute(dk_kernel<GATEUP, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return MOE_Q4_ECUDA;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(dk::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, dk_kernel<GATEUP, NT>, P, tp, twa, twb, tx, txl) == cudaSuccess ? MOE_Q4_OK
+                                                                                                 : MOE_Q4_ECUDA;
+}
+
+}  // namespace q4
+
+using namespace q4;
+
+// Token columns per launch follow from T: an expert holds at most min(T, 16)
+// rows on this path.
+int q4_launch_decode(const FwdArgs& a, const TableParams& tp, bool gateup, float* partial, int32_t* counter,
+                     int grid, cudaStream_t s) {
+  if (a.T * a.k == 0) return MOE_Q4_OK;
+  if (gateup)
+    return a.T <= 8 ? launch_dk<true, 1>(a, tp, partial, counter, grid, s)
+                    : launch_dk<true, 2>(a, tp, partial, counter, grid, s);
+  if (a.T <= 4) return launch_dk<false, 1>(a, tp, partial, counter, grid, s);
+  if (a.T <= 8) return launch_dk<false, 2>(a, tp, partial, counter, grid, s);
+  return launch_dk<false, 4>(a, tp, partial, counter, grid, s);
+}

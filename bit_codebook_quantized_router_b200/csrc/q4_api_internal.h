@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/moe_q4.h"
+#include "moe_q4.h"
 
 namespace q4 {
 struct TableParams;
@@ -53,7 +53,7 @@ int q4_launch_combine(const q4::FwdArgs& a, cudaStream_t s);
 int q4_launch_gather(const q4::FwdArgs& a, cudaStream_t s);
 int q4_launch_prefill(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, cudaStream_t s);
 int q4_prefill_tile_n();
-int q4_launch_decode_tc(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, float* partial,
+int q4_launch_decode(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, float* partial,
                         int32_t* counter, int grid, cudaStream_t s);
 int q4_forward_in_workspace(const moe_q4_layer* layer, const void* x, const float* logits, int T, int top_k,
                             void* out, float* out_f32, void* ws, size_t ws_bytes, cudaStream_t stream);

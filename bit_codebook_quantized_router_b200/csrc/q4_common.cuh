@@ -10,7 +10,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/moe_q4.h"
+#include "moe_q4.h"
 
 namespace q4 {
 

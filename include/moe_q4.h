@@ -215,10 +215,14 @@ MOE_Q4_API int moe_q4_route(const float* logits, int T, int E, int top_k, int32_
 
 /* ---------------------------------------------------------------------------
  * moe_q4_forward_stages -- moe_q4_forward with cudaEvent_t records at the
- * stage boundaries, for timing each kernel on the launching stream:
- *   events[0] before routing, [1] after routing/grouping, [2] after
- *   gate/up + SwiGLU, [3] after the down projection, [4] after the combine.
- * events: host array of n_events (>= 5) cudaEvent_t handles created by the
+ * kernel boundaries, for timing each kernel on the launching stream:
+ *   events[0] before routing, [1] after routing/grouping, [2] after the
+ *   gather of activation rows, [3] after the tensor-core gate/up + SwiGLU,
+ *   [4] after the small-M gate/up + SwiGLU, [5] after the tensor-core down
+ *   projection, [6] after the small-M down projection, [7] after the combine
+ *   (a kernel with no rows to take, e.g. the tensor-core ones for T <= 16,
+ *   is not launched: its two events are recorded back to back).
+ * events: host array of n_events (>= 8) cudaEvent_t handles created by the
  * caller.  The records separate the stages (no programmatic overlap across
  * them), so throughput is measured with moe_q4_forward itself.
  * ------------------------------------------------------------------------- */
