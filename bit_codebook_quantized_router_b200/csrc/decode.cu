@@ -19,10 +19,9 @@
 //   stream at a fraction of HBM bandwidth) with the 128-byte swizzle; TMA
 //   brings the expert's activation rows; the warp's lanes copy each row's
 //   scale bytes for the stage with cp.async, completing on the stage barrier.
-// * Decode + MMA (warps 1..16): warp (slab s, half J) owns weight rows
-//   16s..16s+15 of the tile and the J-th 128-K half of every stage.  Lane
-//   (g, t) reads the 16-byte code chunk t of rows g and g+8 (32 weights, one
-//   E8M0 block), decodes it to bf16 pairs ("aidendle94/GLM-5.2-NF4-Lloyd-
+// * Decode + MMA (warps 1..8): warp s owns weight rows 16s..16s+15 of the
+//   tile.  In each 128-K half of a stage, lane (g, t) reads the 16-byte code
+//   chunk t of rows g and g+8 (32 weights, one E8M0 block), decodes it to bf16 pairs ("aidendle94/GLM-5.2-NF4-Lloyd-
 //   Experts-GPTQ", "Codes are indices into the per-layer grid") and feeds
 //   them to mma.sync m16n8k16 as the A operand.  K is permuted inside each
 //   128-K half, the same way for weights and activations (a sum over K does
@@ -42,8 +41,8 @@
 //   by h and by its low part h_lo (y = W h + W h_lo): with T <= 4 one n-tile
 //   holds h in columns 0..3 and h_lo in 4..7, else separate tiles accumulate
 //   into the same registers.
-// * The two K halves of a slab are added through shared memory (J = 0 + J =
-//   1), then warp (s, 0) finishes: SwiGLU and h / h_lo, or y, or a partial.
+// * At the end of a segment the warp finishes its rows: SwiGLU and h / h_lo,
+//   or y, or a partial sum for a tile shared with other CTAs.
 //
 // Every wait is bounded (a timeout sets MOE_Q4_ETIMEOUT in the status word and
 // the CTA drains and exits); warps wait and leave together (vote).
@@ -58,11 +57,11 @@ namespace q4 {
 using namespace sm100;
 
 namespace dk {
-constexpr int kComputeWarps = 16;                    // 8 slabs x 2 K halves
+constexpr int kComputeWarps = 8;                     // one 16-row slab each
 constexpr int kThreads = 32 * (1 + kComputeWarps);   // + the producer warp
 constexpr int kRows = 128;                           // weight rows per tile
 constexpr int kMaxRing = 6;                          // shared-memory stages, at most
-constexpr int kPrmtWords = 2;                        // of the 4 words of a chunk, decoded in registers
+constexpr int kPrmtWords = 1;                        // of the 4 words of a chunk, decoded in registers
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kLutBytes = 65536;  // 256 entries x (2 table slots x 32 lanes x 4 B)
 constexpr uint32_t kScaleSlot = 8;     // scale bytes per row per stage (4 used for 128-K stages)
@@ -76,25 +75,28 @@ struct DkCfg {
   static constexpr int kAtoms = GATEUP ? NT : (NT == 4 ? 4 : 2);
   // 8-token groups of the result
   static constexpr int kTT = GATEUP ? NT : (NT == 4 ? 2 : 1);
-  static constexpr int kAcc = kMats * kTT * 4;  // accumulator floats per lane
+  // independent accumulators per (matrix, token group): MMA mm of K half J adds
+  // into chain 2J + (mm & 1) (or J), so no MMA waits on the one before it for
+  // long; the chains are added in a fixed order at the end
+  static constexpr int kChains = (kMats * kTT <= 2 && NT <= 2) ? 4 : 2;
 };
 
 // Shared-memory placement (addresses in the CTA's shared window).  The table
 // sits at a 64 KB boundary so its entry addresses can be formed by one PRMT;
-// the activation and scale rings, the exchange area and the barriers go below
-// it when the gap holds them, the code ring above it.  Host and device
+// the activation and scale rings and the barriers go below it when the gap
+// holds them, the code ring above it.  Host and device
 // compute the same placement from the window's start `raw`.
 struct DkLayout {
-  uint32_t lut, codes, x, scales, xch, bars, end;
+  uint32_t lut, codes, x, scales, bars, end;
 };
 
 __host__ __device__ inline DkLayout dk_layout(uint32_t raw, uint32_t code_stage, uint32_t x_stage,
-                                              uint32_t scale_stage, uint32_t xch_bytes, int ring) {
+                                              uint32_t scale_stage, int ring) {
   DkLayout L;
   L.lut = (raw + 65535u) & ~65535u;
   L.codes = L.lut + dk::kLutBytes;
   const uint32_t codes_end = L.codes + (uint32_t)ring * code_stage;
-  const uint32_t others = (uint32_t)ring * (x_stage + scale_stage) + xch_bytes + dk::kBarBytes;
+  const uint32_t others = (uint32_t)ring * (x_stage + scale_stage) + dk::kBarBytes;
   const uint32_t o = (raw + 1023u) & ~1023u;
   if (o + others <= L.lut) {
     L.x = o;
@@ -104,8 +106,7 @@ __host__ __device__ inline DkLayout dk_layout(uint32_t raw, uint32_t code_stage,
     L.end = codes_end + others;
   }
   L.scales = L.x + (uint32_t)ring * x_stage;
-  L.xch = L.scales + (uint32_t)ring * scale_stage;
-  L.bars = L.xch + xch_bytes;
+  L.bars = L.scales + (uint32_t)ring * scale_stage;
   return L;
 }
 
@@ -116,7 +117,7 @@ struct DkParams {
   int stages;       // stages per tile: K / (64 * subs)
   int ring;         // shared-memory stages
   int n_max;        // token columns kept in partial sums: min(16, T)
-  uint32_t code_stage, x_stage, scale_stage, xch_bytes;
+  uint32_t code_stage, x_stage, scale_stage;
   float* partial;   // [2 * gridDim.x][mats][n_max][128]
   int32_t* counter; // [units], zero at launch
 };
@@ -149,16 +150,49 @@ __device__ __forceinline__ void ring_next(int& s, uint32_t& ph, int n) {
   }
 }
 
+// Shared-memory loads and MMAs of the inner loop are plain (not volatile)
+// asm, so the compiler may interleave the independent chains of a stage.
+// Their order against the stage barriers comes from data dependencies:
+// every address is derived from `after_wait(base)`, issued after the wait,
+// and the release takes the loaded words as inputs (`arrive_after`).
+__device__ __forceinline__ uint32_t after_wait(uint32_t v) {
+  uint32_t r;
+  asm volatile("mov.b32 %0, %1;" : "=r"(r) : "r"(v) : "memory");
+  return r;
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+  asm("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
   return v;
 }
 
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
-  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+  asm("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
   return v;
+}
+
+__device__ __forceinline__ uint32_t lds32_nv(uint32_t addr) {
+  uint32_t v;
+  asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
+// Arrive on `bar` once `dep` (a value computed from every shared-memory word
+// the warp read from the stage) is available.
+__device__ __forceinline__ void arrive_after(uint64_t* bar, uint32_t dep) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar)), "r"(dep)
+               : "memory");
+}
+
+// D += A(16x16, bf16, row) * B(16x8, bf16, col), fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float c[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // 16 bf16 pairs of one code chunk (4 words, pair 4w + b from byte b of word
@@ -172,10 +206,10 @@ __device__ __forceinline__ void decode_chunk(const uint4 c, const Planes& PL, ui
       decode8(w[i], PL, &p[4 * i]);
     } else {
       // table entry address = table | byte << 8 | slot << 7 | lane << 2
-      p[4 * i + 0] = lds32(prmt(w[i], kreg, 0x7604));
-      p[4 * i + 1] = lds32(prmt(w[i], kreg, 0x7614));
-      p[4 * i + 2] = lds32(prmt(w[i], kreg, 0x7624));
-      p[4 * i + 3] = lds32(prmt(w[i], kreg, 0x7634));
+      p[4 * i + 0] = lds32_nv(prmt(w[i], kreg, 0x7604));
+      p[4 * i + 1] = lds32_nv(prmt(w[i], kreg, 0x7614));
+      p[4 * i + 2] = lds32_nv(prmt(w[i], kreg, 0x7624));
+      p[4 * i + 3] = lds32_nv(prmt(w[i], kreg, 0x7634));
     }
   }
 #pragma unroll
@@ -191,7 +225,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   constexpr int kMats = C::kMats;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
-  const DkLayout Ls = dk_layout(raw_s, P.code_stage, P.x_stage, P.scale_stage, P.xch_bytes, P.ring);
+  const DkLayout Ls = dk_layout(raw_s, P.code_stage, P.x_stage, P.scale_stage, P.ring);
   const FwdArgs& a = P.a;
   if (Ls.end > raw_s + dynamic_smem_size()) {  // launched with less shared memory than the layout needs
     if (threadIdx.x == 0) record_error(a.hdr + kStatus, MOE_Q4_ECUDA);
@@ -201,10 +235,8 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + (Ls.bars - raw_s));
   uint64_t* full = bars;                          // [ring] codes + activations (TMA), scales (cp.async)
   uint64_t* stage_empty = full + dk::kMaxRing;    // [ring] compute warps done with the stage
-  uint64_t* xfull = stage_empty + dk::kMaxRing;   // [8] K half 1 of slab s written to the exchange area
-  uint64_t* xfree = xfull + 8;                    // [8] ... and read by K half 0
-  uint64_t* lut_bar = xfree + 8;                  // compute threads rebuilding a table slot
-  uint64_t* epi_bar = lut_bar + 1;                // K-half-0 threads finishing a split tile
+  uint64_t* lut_bar = stage_empty + dk::kMaxRing; // compute threads rebuilding a table slot
+  uint64_t* epi_bar = lut_bar + 1;                // compute threads finishing a split tile
   volatile int* abort_flag = reinterpret_cast<volatile int*>(epi_bar + 1);
   volatile int* last_flag = abort_flag + 1;
 
@@ -215,12 +247,8 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       mbar_init(&full[s], 1 + 32);  // producer lane 0 (with the TMA bytes) + 32 cp.async arrivals
       mbar_init(&stage_empty[s], dk::kComputeWarps);
     }
-    for (int s = 0; s < 8; ++s) {
-      mbar_init(&xfull[s], 32);
-      mbar_init(&xfree[s], 32);
-    }
     mbar_init(lut_bar, 32 * dk::kComputeWarps);
-    mbar_init(epi_bar, 32 * 8);
+    mbar_init(epi_bar, 32 * dk::kComputeWarps);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_wa);
@@ -304,23 +332,16 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     }
   } else {
     // ------------------------------ compute ------------------------------
-    const int cw = warp - 1;       // 0..15
-    const int slab = cw & 7;       // rows 16 slab .. + 15 of the tile
-    const int J = cw >> 3;         // 128-K half of each stage
+    const int slab = warp - 1;     // rows 16 slab .. + 15 of the tile
     const int gq = lane >> 2;      // MMA group: rows gq, gq + 8; token column gq
-    const int tq = lane & 3;       // code chunk of the half; token columns 2tq, 2tq + 1
+    const int tq = lane & 3;       // code chunk of a half; token columns 2tq, 2tq + 1
     const int ctid = threadIdx.x - 32;
-    const bool active = 2 * J < subs;  // a 128-K stage has one half only
+    const int n_halves = subs / 2; // 128-K halves per stage
     const int r0 = 16 * slab + gq, r1 = r0 + 8;
     const int swz0 = subs == 4 ? (r0 & 7) : ((r0 >> 1) & 3);
     const int swz1 = subs == 4 ? (r1 & 7) : ((r1 >> 1) & 3);
-    const int chunk = 4 * J + tq;  // 16-byte chunk of the stage row
-    const uint32_t coff0 = (uint32_t)(r0 * row_bytes + ((chunk ^ swz0) << 4));
-    const uint32_t coff1 = (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4));
-    // activation run of this lane: super-step 2J + (tq >> 1), chunks 4 (tq & 1) .. +3
-    const uint32_t xss = (uint32_t)(2 * J + (tq >> 1)) * C::kAtoms * 1024;
     int slot_tab0 = -1, slot_tab1 = -1, victim = 0;
-    uint32_t lgen = 0, xgen = 0, egen = 0;
+    uint32_t lgen = 0, egen = 0;
     const uint32_t lane_k = (Ls.lut & 0xffff0000u) | ((uint32_t)lane << 2);
     int s = 0;
     uint32_t ph = 0;
@@ -349,57 +370,82 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         else
           slot_tab1 = tid;
         const float* tv = tp.t[tid];
-        const uint32_t ent = ctid & 255, half = ctid >> 8;
+        const uint32_t ent = ctid;  // 0..255
         const uint32_t lo = ent & 15, hi = ent >> 4;
         const uint32_t blo = (uint32_t)bf16_bits_rn(tv[lo & 7]) ^ ((lo & 8) ? 0x8000u : 0u);
         const uint32_t bhi = (uint32_t)bf16_bits_rn(tv[hi & 7]) ^ ((hi & 8) ? 0x8000u : 0u);
         const uint32_t word = blo | (bhi << 16);
-        uint4* dst = reinterpret_cast<uint4*>(lut + ent * 256 + slot * 128 + half * 64);
+        uint4* dst = reinterpret_cast<uint4*>(lut + ent * 256 + slot * 128);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(word, word, word, word);
+        for (int i = 0; i < 8; ++i) dst[i] = make_uint4(word, word, word, word);
         mbar_arrive(lut_bar);
         if (!mbar_wait_warp(lut_bar, lgen & 1, abort_flag, dk::kWaitNs)) break;
         ++lgen;
       }
       const uint32_t kreg = lane_k | ((uint32_t)slot << 7);
       const Planes PL = make_planes(tp.t[tid]);
+      // token column of this lane in n-tile nt exists (else its operand is zero and
+      // its shared-memory read is skipped)
+      const int n_e_seg = a.counts[e];
+      bool col_ok[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        int tok;
+        if (GATEUP)
+          tok = 8 * nt + gq;
+        else if (NT == 1)
+          tok = gq & 3;
+        else if (NT == 2)
+          tok = gq;
+        else
+          tok = 8 * (nt & 1) + gq;
+        col_ok[nt] = tok < n_e_seg;
+      }
 
-      float acc[kMats][C::kTT][4];
+      float accc[kMats][C::kTT][C::kChains][4];
 #pragma unroll
       for (int m = 0; m < kMats; ++m)
 #pragma unroll
         for (int tt = 0; tt < C::kTT; ++tt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) acc[m][tt][i] = 0.0f;
+          for (int c = 0; c < C::kChains; ++c)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) accc[m][tt][c][i] = 0.0f;
 
       for (int j = 0; j < nst && ok; ++j) {
         if (!mbar_wait_warp(&full[s], ph, abort_flag, dk::kWaitNs)) {
           ok = false;
           break;
         }
-        if (active) {
-          const uint32_t cbase = Ls.codes + (uint32_t)s * P.code_stage;
-          const uint32_t sbase = Ls.scales + (uint32_t)s * P.scale_stage;
-          const uint32_t xbase = Ls.x + (uint32_t)s * P.x_stage + xss;
+        const uint32_t cbase = after_wait(Ls.codes + (uint32_t)s * P.code_stage);
+        const uint32_t sbase = after_wait(Ls.scales + (uint32_t)s * P.scale_stage);
+        const uint32_t xstage = after_wait(Ls.x + (uint32_t)s * P.x_stage);
+        uint32_t dep = 0;  // every word read from the stage, folded
+#pragma unroll
+        for (int J = 0; J < 2; ++J) {
+          if (J >= n_halves) break;
+          const int chunk = 4 * J + tq;  // 16-byte chunk of the stage row
+          const uint32_t coff0 = (uint32_t)(r0 * row_bytes + ((chunk ^ swz0) << 4));
+          const uint32_t coff1 = (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4));
+          // activation run of this lane: super-step 2J + (tq >> 1), chunks 4 (tq & 1) .. +3
+          const uint32_t xbase = xstage + (uint32_t)(2 * J + (tq >> 1)) * C::kAtoms * 1024;
           // activation operands: 16 pairs per n-tile, pair m at K offset 32 tq + 2m
           uint32_t xr[NT][16];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            int atom, row;
-            if (GATEUP) {
+            int atom;
+            if (GATEUP)
               atom = nt;
-              row = gq;
-            } else if (NT == 1) {
+            else if (NT == 1)
               atom = gq >> 2;  // h at rows 0..3 of atom 0, h_lo at rows 4..7 of atom 1
-              row = gq;
-            } else {
+            else
               atom = nt;
-              row = gq;
-            }
-            const uint32_t rb = xbase + (uint32_t)atom * 1024 + (uint32_t)row * 128;
+            const uint32_t rb = xbase + (uint32_t)atom * 1024 + (uint32_t)gq * 128;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              const uint4 v = lds128(rb + ((((tq & 1) * 4 + c) ^ row) << 4));
+              uint4 v = make_uint4(0u, 0u, 0u, 0u);
+              if (col_ok[nt]) v = lds128(rb + ((((tq & 1) * 4 + c) ^ gq) << 4));
+              dep ^= v.x ^ v.w;
               xr[nt][4 * c + 0] = v.x;
               xr[nt][4 * c + 1] = v.y;
               xr[nt][4 * c + 2] = v.z;
@@ -413,6 +459,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
             const uint4 c1 = lds128(mb + coff1);
             const uint2 s0 = lds64(sbase + (uint32_t)((m * dk::kRows + r0) * dk::kScaleSlot));
             const uint2 s1 = lds64(sbase + (uint32_t)((m * dk::kRows + r1) * dk::kScaleSlot));
+            dep ^= c0.x ^ c0.w ^ c1.x ^ c1.w ^ s0.x ^ s1.y;
             // E8M0 byte of block 4J + tq
             const uint32_t e0 = ((J ? s0.y : s0.x) >> (8 * tq)) & 0xffu;
             const uint32_t e1 = ((J ? s1.y : s1.x) >> (8 * tq)) & 0xffu;
@@ -424,48 +471,39 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
 #pragma unroll
               for (int nt = 0; nt < NT; ++nt) {
                 const int tt = GATEUP ? nt : (NT == 4 ? (nt & 1) : 0);
-                mma_16816(acc[m][tt], pa[mm], pb[mm], pa[mm + 8], pb[mm + 8], xr[nt][mm], xr[nt][mm + 8]);
+                const int ch = C::kChains == 4 ? 2 * J + (mm & 1) : J;
+                mma_bf16_16816(accc[m][tt][ch], pa[mm], pb[mm], pa[mm + 8], pb[mm + 8], xr[nt][mm], xr[nt][mm + 8]);
               }
             }
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&stage_empty[s]);
+        // the table lookups read only the table, not the stage: the stage is free
+        // once the loads above have returned (their values feed `dep`)
+        dep = __reduce_xor_sync(0xffffffffu, dep);
+        if (lane == 0) arrive_after(&stage_empty[s], dep);
         ring_next(s, ph, ring);
       }
       if (!ok) break;
 
-      // ---- segment end: add the K halves (J = 1 into J = 0) ----
-      float* xch = reinterpret_cast<float*>(smem_raw + (Ls.xch - raw_s)) + (size_t)slab * C::kAcc * 32;
-      if (J == 1) {
-        if (xgen > 0 && !mbar_wait_warp(&xfree[slab], (xgen - 1) & 1, abort_flag, dk::kWaitNs)) break;
-#pragma unroll
-        for (int m = 0; m < kMats; ++m)
-#pragma unroll
-          for (int tt = 0; tt < C::kTT; ++tt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) xch[((m * C::kTT + tt) * 4 + i) * 32 + lane] = acc[m][tt][i];
-        mbar_arrive(&xfull[slab]);
-        ++xgen;
-        g = seg_end;
-        continue;
-      }
-      if (!mbar_wait_warp(&xfull[slab], xgen & 1, abort_flag, dk::kWaitNs)) break;
+      float acc[kMats][C::kTT][4];
 #pragma unroll
       for (int m = 0; m < kMats; ++m)
 #pragma unroll
         for (int tt = 0; tt < C::kTT; ++tt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) acc[m][tt][i] += xch[((m * C::kTT + tt) * 4 + i) * 32 + lane];
-      mbar_arrive(&xfree[slab]);
-      ++xgen;
+          for (int i = 0; i < 4; ++i) {
+            float v = accc[m][tt][0][i];
+#pragma unroll
+            for (int c = 1; c < C::kChains; ++c) v += accc[m][tt][c][i];
+            acc[m][tt][i] = v;
+          }
       if (!GATEUP && NT == 1) {
         // columns 4..7 hold W h_lo for tokens 0..3: add them to columns 0..3
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[0][0][i] += __shfl_xor_sync(0xffffffffu, acc[0][0][i], 2);
       }
 
-      // ---- K half 0 finishes the slab: token n = 8 tt + 2 tq + (i & 1), row r0 / r1 ----
+      // ---- the warp finishes its rows: token n = 8 tt + 2 tq + (i & 1), row r0 / r1 ----
       const int row0 = a.offsets[e], n_e = a.counts[e];
       const bool final_here = (g == ustart && seg_end == uend);
       if (!final_here) {
@@ -607,7 +645,6 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
   P.code_stage = (uint32_t)(C::kMats * dk::kRows * 32 * P.subs);
   P.x_stage = (uint32_t)(P.subs * C::kAtoms * 1024);
   P.scale_stage = (uint32_t)(C::kMats * dk::kRows * dk::kScaleSlot);
-  P.xch_bytes = (uint32_t)(8 * C::kAcc * 32 * sizeof(float));
   P.partial = partial;
   P.counter = counter;
 
@@ -620,7 +657,7 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
   P.ring = 0;
   uint32_t smem = 0;
   for (int rs = dk::kMaxRing; rs >= 2 && !P.ring; --rs) {
-    const DkLayout L = dk_layout((uint32_t)reserved, P.code_stage, P.x_stage, P.scale_stage, P.xch_bytes, rs);
+    const DkLayout L = dk_layout((uint32_t)reserved, P.code_stage, P.x_stage, P.scale_stage, rs);
     if (L.end - (uint32_t)reserved <= (uint32_t)optin) {
       P.ring = rs;
       smem = L.end - (uint32_t)reserved;
