@@ -186,7 +186,9 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   float* part_dn = part_gu + (size_t)2 * kDkMaxGrid * 2 * o.n_max * 128;
   int32_t* cnt_gu = a.dk_counter;
   int32_t* cnt_dn = a.dk_counter + o.dk_units_gu;
-  if (rc == MOE_Q4_OK) rc = q4_launch_gather(a, s);
+  // grouped activation rows feed the tensor-core path only (the small-M kernels
+  // copy their rows from x themselves)
+  if (rc == MOE_Q4_OK && pre) rc = q4_launch_gather(a, s);
   if (rc == MOE_Q4_OK) rc = mark(2);
   if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, true, s);
   if (rc == MOE_Q4_OK) rc = mark(3);

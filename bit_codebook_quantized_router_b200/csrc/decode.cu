@@ -16,9 +16,11 @@
 //   and writes the result.
 // * Data movement (warp 0): per stage and matrix one TMA brings 128 weight
 //   rows x 128 bytes of codes (a full 128-byte line per row: narrower boxes
-//   stream at a fraction of HBM bandwidth) with the 128-byte swizzle; TMA
-//   brings the expert's activation rows; the warp's lanes copy each row's
-//   scale bytes for the stage with cp.async, completing on the stage barrier.
+//   stream at a fraction of HBM bandwidth) with the 128-byte swizzle; the
+//   warp's lanes copy each row's scale bytes for the stage and (gate/up) the
+//   expert's activation rows, straight from x through the row -> token map,
+//   with cp.async, completing on the stage barrier; the down projection's h
+//   rows come by TMA.
 // * Decode + MMA (warps 1..8): warp s owns weight rows 16s..16s+15 of the
 //   tile.  In each 128-K half of a stage, lane (g, t) reads the 16-byte code
 //   chunk t of rows g and g+8 (32 weights, one E8M0 block), decodes it to bf16 pairs ("aidendle94/GLM-5.2-NF4-Lloyd-
@@ -26,8 +28,9 @@
 //   them to mma.sync m16n8k16 as the A operand.  K is permuted inside each
 //   128-K half, the same way for weights and activations (a sum over K does
 //   not depend on its order): MMA m takes from lane t the pairs at K offsets
-//   32t + 2m and 32t + 16 + 2m, so every lane's operands come from its own
-//   code chunk and one 64-byte run of each activation row.  Decoding mixes a
+//   32t + 4m and 32t + 4m + 2, so every lane's operands come from its own
+//   code chunk and one 64-byte run of each activation row, and each MMA's two
+//   activation registers are adjacent words of one 16-byte load.  Decoding mixes a
 //   shared-memory table byte -> signed bf16 pair (one copy per lane: a warp's
 //   32 lookups hit 32 banks) with the in-register PRMT decode, balancing the
 //   integer pipe against shared-memory bandwidth; the block scale is one
@@ -81,33 +84,58 @@ struct DkCfg {
   static constexpr int kChains = (kMats * kTT <= 2 && NT <= 2) ? 4 : 2;
 };
 
-// Shared-memory placement (addresses in the CTA's shared window).  The table
-// sits at a 64 KB boundary so its entry addresses can be formed by one PRMT;
-// the activation and scale rings and the barriers go below it when the gap
-// holds them, the code ring above it.  Host and device
-// compute the same placement from the window's start `raw`.
+// Shared-memory placement, as offsets from the start of the CTA's dynamic
+// window.  The table sits at a 64 KB boundary so its entry addresses can be
+// formed by one PRMT; that leaves a region below it and one above.  The
+// activation and scale rings and the barriers go low, the code stages high
+// and, when the low region has room left, one or more of them low too (a
+// deeper ring keeps more bytes in flight per SM).  The host computes it for
+// the window start it expects; the kernel checks alignment and size.
 struct DkLayout {
-  uint32_t lut, codes, x, scales, bars, end;
+  uint32_t lut, code_hi, code_lo, x, scales, bars, end;
+  int n_hi;  // code stages at code_hi; stages n_hi.. at code_lo
 };
 
-__host__ __device__ inline DkLayout dk_layout(uint32_t raw, uint32_t code_stage, uint32_t x_stage,
-                                              uint32_t scale_stage, int ring) {
-  DkLayout L;
-  L.lut = (raw + 65535u) & ~65535u;
-  L.codes = L.lut + dk::kLutBytes;
-  const uint32_t codes_end = L.codes + (uint32_t)ring * code_stage;
-  const uint32_t others = (uint32_t)ring * (x_stage + scale_stage) + dk::kBarBytes;
+static bool dk_layout(uint32_t raw, uint32_t limit, uint32_t code_stage, uint32_t x_stage, uint32_t scale_stage,
+                      int ring, DkLayout& L) {
+  const uint32_t lut = (raw + 65535u) & ~65535u;
   const uint32_t o = (raw + 1023u) & ~1023u;
-  if (o + others <= L.lut) {
-    L.x = o;
-    L.end = codes_end;
+  const uint32_t hi = lut + dk::kLutBytes;
+  if (hi > limit) return false;
+  const uint32_t others = (uint32_t)ring * (x_stage + scale_stage) + dk::kBarBytes;
+  const int fit_hi = (int)((limit - hi) / code_stage);
+  uint32_t x;
+  if (o + others <= lut) {
+    // low: others, then the code stages that do not fit high
+    const int n_hi = fit_hi < ring ? fit_hi : ring;
+    const uint32_t lo = (o + others + 1023u) & ~1023u;
+    if (lo + (uint32_t)(ring - n_hi) * code_stage > lut) return false;
+    x = o;
+    L.n_hi = n_hi;
+    L.code_hi = hi;
+    L.code_lo = lo;
+    L.end = hi + (uint32_t)n_hi * code_stage;
   } else {
-    L.x = codes_end;
-    L.end = codes_end + others;
+    // all high: code stages, then the others
+    if (fit_hi < ring || hi + (uint32_t)ring * code_stage + others > limit) return false;
+    L.n_hi = ring;
+    L.code_hi = L.code_lo = hi;
+    x = hi + (uint32_t)ring * code_stage;
+    L.end = x + others;
   }
-  L.scales = L.x + (uint32_t)ring * x_stage;
+  L.lut = lut;
+  L.x = x;
+  L.scales = x + (uint32_t)ring * x_stage;
   L.bars = L.scales + (uint32_t)ring * scale_stage;
-  return L;
+  // offsets from the window start
+  L.lut -= raw;
+  L.code_hi -= raw;
+  L.code_lo -= raw;
+  L.x -= raw;
+  L.scales -= raw;
+  L.bars -= raw;
+  L.end -= raw;
+  return true;
 }
 
 struct DkParams {
@@ -116,6 +144,7 @@ struct DkParams {
   int subs;         // 64-K super-steps per stage: 4 (K % 256 == 0) or 2
   int stages;       // stages per tile: K / (64 * subs)
   int ring;         // shared-memory stages
+  DkLayout lay;     // shared-memory placement (offsets)
   int n_max;        // token columns kept in partial sums: min(16, T)
   uint32_t code_stage, x_stage, scale_stage;
   float* partial;   // [2 * gridDim.x][mats][n_max][128]
@@ -195,6 +224,19 @@ __device__ __forceinline__ void mma_bf16_16816(float c[4], uint32_t a0, uint32_t
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// Table slot `slot`: entry c -> bf16 pair of codes (c & 15, c >> 4), signed,
+// unscaled, one copy per lane (entry c of lane l at c * 256 + slot * 128 +
+// l * 4).  Thread ent (0..255) writes entry ent.
+__device__ __forceinline__ void build_lut_slot(uint8_t* lut, const float* tv, int slot, int ent) {
+  const uint32_t lo = ent & 15, hi = ent >> 4;
+  const uint32_t blo = (uint32_t)bf16_bits_rn(tv[lo & 7]) ^ ((lo & 8) ? 0x8000u : 0u);
+  const uint32_t bhi = (uint32_t)bf16_bits_rn(tv[hi & 7]) ^ ((hi & 8) ? 0x8000u : 0u);
+  const uint32_t word = blo | (bhi << 16);
+  uint4* dst = reinterpret_cast<uint4*>(lut + ent * 256 + slot * 128);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dst[i] = make_uint4(word, word, word, word);
+}
+
 // 16 bf16 pairs of one code chunk (4 words, pair 4w + b from byte b of word
 // w), scaled: words below kPrmtWords by the PRMT decode, the rest by table.
 __device__ __forceinline__ void decode_chunk(const uint4 c, const Planes& PL, uint32_t kreg, uint32_t scale2,
@@ -225,15 +267,26 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   constexpr int kMats = C::kMats;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
-  const DkLayout Ls = dk_layout(raw_s, P.code_stage, P.x_stage, P.scale_stage, P.ring);
+  // absolute shared addresses of the placement
+  DkLayout Ls = P.lay;
+  Ls.lut += raw_s;
+  Ls.code_hi += raw_s;
+  Ls.code_lo += raw_s;
+  Ls.x += raw_s;
+  Ls.scales += raw_s;
+  Ls.bars += raw_s;
   const FwdArgs& a = P.a;
-  if (Ls.end > raw_s + dynamic_smem_size()) {  // launched with less shared memory than the layout needs
+  if (P.lay.end > dynamic_smem_size() || (Ls.lut & 0xffffu) != 0u) {
+    // the window is smaller or starts elsewhere than the host planned for
     if (threadIdx.x == 0) record_error(a.hdr + kStatus, MOE_Q4_ECUDA);
     return;
   }
+  const auto code_base = [&](int s) -> uint32_t {
+    return s < Ls.n_hi ? Ls.code_hi + (uint32_t)s * P.code_stage : Ls.code_lo + (uint32_t)(s - Ls.n_hi) * P.code_stage;
+  };
   uint8_t* lut = smem_raw + (Ls.lut - raw_s);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + (Ls.bars - raw_s));
-  uint64_t* full = bars;                          // [ring] codes + activations (TMA), scales (cp.async)
+  uint64_t* full = bars;                          // [ring] codes (+ h: TMA), scales (+ x: cp.async)
   uint64_t* stage_empty = full + dk::kMaxRing;    // [ring] compute warps done with the stage
   uint64_t* lut_bar = stage_empty + dk::kMaxRing; // compute threads rebuilding a table slot
   uint64_t* epi_bar = lut_bar + 1;                // compute threads finishing a split tile
@@ -253,9 +306,14 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     fence_mbar_init();
     prefetch_tmap(&tm_wa);
     if (GATEUP) prefetch_tmap(&tm_wb);
-    prefetch_tmap(&tm_x);
-    if (!GATEUP) prefetch_tmap(&tm_xl);
+    if (!GATEUP) {
+      prefetch_tmap(&tm_x);
+      prefetch_tmap(&tm_xl);
+    }
   }
+  // with a single table every expert uses table 0: its table slot is built
+  // before waiting for the previous kernel
+  if (tp.n == 1 && warp >= 1) build_lut_slot(lut, tp.t[0], 0, threadIdx.x - 32);
   __syncthreads();
 
   pdl_wait();
@@ -279,12 +337,30 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       const long long seg_end = min(k1, (long long)(unit + 1) * P.stages);
       const int e = a.dec_list[unit / P.tiles_per_e];
       const int t = unit % P.tiles_per_e;
-      const int row0 = a.offsets[e];
       const int wrow = e * rows_total + t * dk::kRows;
+      const int row0 = a.offsets[e];
+      // gate/up: the tokens of the activation rows this lane copies (rows
+      // (lane >> 3) + 4q of the expert, absent ones zero-filled)
+      int tok[2 * NT];
+      int n_e = 0;
+      if (GATEUP) {
+        n_e = a.counts[e];
+#pragma unroll
+        for (int q = 0; q < 2 * NT; ++q) {
+          const int n = (lane >> 3) + 4 * q;
+          tok[q] = n < n_e ? a.row_token[row0 + n] : 0;
+        }
+      }
       for (int st = st0; st < st0 + (int)(seg_end - g); ++st) {
         if (!mbar_wait_warp(&stage_empty[s], ph ^ 1, abort_flag, dk::kWaitNs)) {
           ok = false;
           break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes + (GATEUP ? 0 : subs * C::kAtoms * 1024));
+          uint8_t* cdst = smem_raw + (code_base(s) - raw_s);
+          tma_load_2d(cdst, &tm_wa, &full[s], st * row_bytes, wrow);
+          if (GATEUP) tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
         }
         // scale bytes of the stage (2 per 64-K super-step) for 4 rows per lane
 #pragma unroll
@@ -302,26 +378,37 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
               cp_async_small<4>(dst, sbase + (size_t)r * (K / 32));
           }
         }
-        cp_async_arrive_noinc(&full[s]);
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes + subs * C::kAtoms * 1024);
-          uint8_t* cdst = smem_raw + (Ls.codes - raw_s) + (size_t)s * P.code_stage;
-          tma_load_2d(cdst, &tm_wa, &full[s], st * row_bytes, wrow);
-          if (GATEUP) tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
-          // the expert's activation rows, grouped; rows past n_e belong to the next
-          // expert or lie outside the array: they only feed columns nobody writes
-          uint8_t* xdst = smem_raw + (Ls.x - raw_s) + (size_t)s * P.x_stage;
+        const uint32_t xdst = Ls.x + (uint32_t)s * P.x_stage;
+        if (GATEUP) {
+          // activation rows: 8 NT rows x 8 chunks of 16 B per 64-K super-step, in
+          // the 128-byte swizzle the compute warps read (chunk c of row n at c ^ n)
           for (int j = 0; j < subs; ++j) {
             const int kx = (st * subs + j) * 64;
-            uint8_t* d = xdst + j * C::kAtoms * 1024;
-            if (GATEUP) {
-              tma_load_2d(d, &tm_x, &full[s], kx, row0);  // 8 * NT rows
-            } else if (NT == 1) {
+#pragma unroll
+            for (int q = 0; q < 2 * NT; ++q) {
+              const int idx = lane + 32 * q;
+              const int n = idx >> 3, c = idx & 7;
+              const uint32_t dst = xdst + (uint32_t)(j * C::kAtoms * 1024 + (n >> 3) * 1024 + (n & 7) * 128 +
+                                                     ((c ^ (n & 7)) << 4));
+              const bool have = n < n_e;
+              const __nv_bfloat16* src = have ? a.x + (size_t)tok[q] * a.H + kx + 8 * c : a.x;
+              cp_async_16_zfill(dst, src, have ? 16u : 0u);
+            }
+          }
+        }
+        cp_async_arrive_noinc(&full[s]);
+        if (!GATEUP && lane == 0) {
+          // the expert's h rows, grouped; rows past n_e belong to the next expert or
+          // lie outside the array: they only feed columns nobody writes
+          for (int j = 0; j < subs; ++j) {
+            const int kx = (st * subs + j) * 64;
+            uint8_t* d = smem_raw + (xdst - raw_s) + j * C::kAtoms * 1024;
+            if (NT == 1) {
               tma_load_2d(d, &tm_x, &full[s], kx, row0);             // h rows 0..3 at atom rows 0..3
               tma_load_2d(d + 1024, &tm_xl, &full[s], kx, row0 - 4);  // h_lo rows 0..3 at atom rows 4..7
             } else {
-              tma_load_2d(d, &tm_x, &full[s], kx, row0);                         // h: NT / 2 atoms
-              tma_load_2d(d + (NT / 2) * 1024, &tm_xl, &full[s], kx, row0);      // h_lo
+              tma_load_2d(d, &tm_x, &full[s], kx, row0);                     // h: NT / 2 atoms
+              tma_load_2d(d + (NT / 2) * 1024, &tm_xl, &full[s], kx, row0);  // h_lo
             }
           }
         }
@@ -340,7 +427,20 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     const int r0 = 16 * slab + gq, r1 = r0 + 8;
     const int swz0 = subs == 4 ? (r0 & 7) : ((r0 >> 1) & 3);
     const int swz1 = subs == 4 ? (r1 & 7) : ((r1 >> 1) & 3);
-    int slot_tab0 = -1, slot_tab1 = -1, victim = 0;
+    // per-lane offsets inside a stage: code chunk 4J + tq of rows r0 / r1, and
+    // this lane's activation run (super-step 2J + (tq >> 1), row gq, chunks
+    // 4 (tq & 1) .. +3 in the 128-byte swizzle)
+    uint32_t coff[2][2], xoff[2][4];
+#pragma unroll
+    for (int J = 0; J < 2; ++J) {
+      const int chunk = 4 * J + tq;
+      coff[J][0] = (uint32_t)(r0 * row_bytes + ((chunk ^ swz0) << 4));
+      coff[J][1] = (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4));
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        xoff[J][c] = (uint32_t)((2 * J + (tq >> 1)) * C::kAtoms * 1024 + gq * 128 + ((((tq & 1) * 4 + c) ^ gq) << 4));
+    }
+    int slot_tab0 = tp.n == 1 ? 0 : -1, slot_tab1 = -1, victim = tp.n == 1 ? 1 : 0;
     uint32_t lgen = 0, egen = 0;
     const uint32_t lane_k = (Ls.lut & 0xffff0000u) | ((uint32_t)lane << 2);
     int s = 0;
@@ -369,39 +469,13 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           slot_tab0 = tid;
         else
           slot_tab1 = tid;
-        const float* tv = tp.t[tid];
-        const uint32_t ent = ctid;  // 0..255
-        const uint32_t lo = ent & 15, hi = ent >> 4;
-        const uint32_t blo = (uint32_t)bf16_bits_rn(tv[lo & 7]) ^ ((lo & 8) ? 0x8000u : 0u);
-        const uint32_t bhi = (uint32_t)bf16_bits_rn(tv[hi & 7]) ^ ((hi & 8) ? 0x8000u : 0u);
-        const uint32_t word = blo | (bhi << 16);
-        uint4* dst = reinterpret_cast<uint4*>(lut + ent * 256 + slot * 128);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) dst[i] = make_uint4(word, word, word, word);
+        build_lut_slot(lut, tp.t[tid], slot, ctid);
         mbar_arrive(lut_bar);
         if (!mbar_wait_warp(lut_bar, lgen & 1, abort_flag, dk::kWaitNs)) break;
         ++lgen;
       }
       const uint32_t kreg = lane_k | ((uint32_t)slot << 7);
       const Planes PL = make_planes(tp.t[tid]);
-      // token column of this lane in n-tile nt exists (else its operand is zero and
-      // its shared-memory read is skipped)
-      const int n_e_seg = a.counts[e];
-      bool col_ok[NT];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        int tok;
-        if (GATEUP)
-          tok = 8 * nt + gq;
-        else if (NT == 1)
-          tok = gq & 3;
-        else if (NT == 2)
-          tok = gq;
-        else
-          tok = 8 * (nt & 1) + gq;
-        col_ok[nt] = tok < n_e_seg;
-      }
-
       float accc[kMats][C::kTT][C::kChains][4];
 #pragma unroll
       for (int m = 0; m < kMats; ++m)
@@ -417,19 +491,14 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           ok = false;
           break;
         }
-        const uint32_t cbase = after_wait(Ls.codes + (uint32_t)s * P.code_stage);
+        const uint32_t cbase = after_wait(code_base(s));
         const uint32_t sbase = after_wait(Ls.scales + (uint32_t)s * P.scale_stage);
         const uint32_t xstage = after_wait(Ls.x + (uint32_t)s * P.x_stage);
         uint32_t dep = 0;  // every word read from the stage, folded
 #pragma unroll
         for (int J = 0; J < 2; ++J) {
           if (J >= n_halves) break;
-          const int chunk = 4 * J + tq;  // 16-byte chunk of the stage row
-          const uint32_t coff0 = (uint32_t)(r0 * row_bytes + ((chunk ^ swz0) << 4));
-          const uint32_t coff1 = (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4));
-          // activation run of this lane: super-step 2J + (tq >> 1), chunks 4 (tq & 1) .. +3
-          const uint32_t xbase = xstage + (uint32_t)(2 * J + (tq >> 1)) * C::kAtoms * 1024;
-          // activation operands: 16 pairs per n-tile, pair m at K offset 32 tq + 2m
+          // activation operands: 16 pairs per n-tile, pair p at K offset 32 tq + 2p
           uint32_t xr[NT][16];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
@@ -440,26 +509,24 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
               atom = gq >> 2;  // h at rows 0..3 of atom 0, h_lo at rows 4..7 of atom 1
             else
               atom = nt;
-            const uint32_t rb = xbase + (uint32_t)atom * 1024 + (uint32_t)gq * 128;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              uint4 v = make_uint4(0u, 0u, 0u, 0u);
-              if (col_ok[nt]) v = lds128(rb + ((((tq & 1) * 4 + c) ^ gq) << 4));
-              dep ^= v.x ^ v.w;
+              const uint4 v = lds128(xstage + (uint32_t)atom * 1024 + xoff[J][c]);
               xr[nt][4 * c + 0] = v.x;
               xr[nt][4 * c + 1] = v.y;
               xr[nt][4 * c + 2] = v.z;
               xr[nt][4 * c + 3] = v.w;
+              dep ^= v.x;
             }
           }
 #pragma unroll
           for (int m = 0; m < kMats; ++m) {
             const uint32_t mb = cbase + (uint32_t)(m * dk::kRows * row_bytes);
-            const uint4 c0 = lds128(mb + coff0);
-            const uint4 c1 = lds128(mb + coff1);
+            const uint4 c0 = lds128(mb + coff[J][0]);
+            const uint4 c1 = lds128(mb + coff[J][1]);
             const uint2 s0 = lds64(sbase + (uint32_t)((m * dk::kRows + r0) * dk::kScaleSlot));
             const uint2 s1 = lds64(sbase + (uint32_t)((m * dk::kRows + r1) * dk::kScaleSlot));
-            dep ^= c0.x ^ c0.w ^ c1.x ^ c1.w ^ s0.x ^ s1.y;
+            dep ^= c0.x ^ c1.x ^ s0.x ^ s1.x;
             // E8M0 byte of block 4J + tq
             const uint32_t e0 = ((J ? s0.y : s0.x) >> (8 * tq)) & 0xffu;
             const uint32_t e1 = ((J ? s1.y : s1.x) >> (8 * tq)) & 0xffu;
@@ -472,7 +539,8 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
               for (int nt = 0; nt < NT; ++nt) {
                 const int tt = GATEUP ? nt : (NT == 4 ? (nt & 1) : 0);
                 const int ch = C::kChains == 4 ? 2 * J + (mm & 1) : J;
-                mma_bf16_16816(accc[m][tt][ch], pa[mm], pb[mm], pa[mm + 8], pb[mm + 8], xr[nt][mm], xr[nt][mm + 8]);
+                mma_bf16_16816(accc[m][tt][ch], pa[2 * mm], pb[2 * mm], pa[2 * mm + 1], pb[2 * mm + 1],
+                               xr[nt][2 * mm], xr[nt][2 * mm + 1]);
               }
             }
           }
@@ -655,15 +723,12 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
   cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev);
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   P.ring = 0;
-  uint32_t smem = 0;
-  for (int rs = dk::kMaxRing; rs >= 2 && !P.ring; --rs) {
-    const DkLayout L = dk_layout((uint32_t)reserved, P.code_stage, P.x_stage, P.scale_stage, rs);
-    if (L.end - (uint32_t)reserved <= (uint32_t)optin) {
+  for (int rs = dk::kMaxRing; rs >= 2 && !P.ring; --rs)
+    if (dk_layout((uint32_t)reserved, (uint32_t)reserved + (uint32_t)optin, P.code_stage, P.x_stage, P.scale_stage,
+                  rs, P.lay))
       P.ring = rs;
-      smem = L.end - (uint32_t)reserved;
-    }
-  }
   if (!P.ring) return MOE_Q4_ECUDA;
+  const uint32_t smem = P.lay.end;
 
   const int R = a.T * a.k;
   const CUtensorMapSwizzle csw = P.subs == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -673,9 +738,8 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
   bool ok;
   if (GATEUP) {
     ok = dk_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.gate_w, a.H / 2, (uint64_t)a.E * a.I, cbox, dk::kRows, csw) &&
-         dk_map(&twb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.up_w, a.H / 2, (uint64_t)a.E * a.I, cbox, dk::kRows, csw) &&
-         dk_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.xg, a.H, R, 64, xrows, CU_TENSOR_MAP_SWIZZLE_128B);
-    txl = tx;
+         dk_map(&twb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.up_w, a.H / 2, (uint64_t)a.E * a.I, cbox, dk::kRows, csw);
+    tx = txl = twa;  // unused: activation rows come by cp.async
   } else {
     ok = dk_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.down_w, a.I / 2, (uint64_t)a.E * a.H, cbox, dk::kRows,
                 csw) &&
