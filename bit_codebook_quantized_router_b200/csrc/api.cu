@@ -59,7 +59,7 @@ bool shape_ok(const moe_q4_layer* L, int T, int top_k) {
 //   offsets int32[E+1] | row_token int32[T*k] | inv int32[T*k] |
 //   dec_list int32[E] | pre_list int32[E] | tiles int32[E+1] | h bf16[T*k][I] |
 //   h_lo bf16[T*k][I] | y f32[T*k][H] | xg bf16[T*k][H] (activation rows in
-//   expert order) | split-tile counters int32[units] | partial sums of the
+//   expert order, T > 16 only) | split-tile counters int32[units] | partial sums of the
 //   small-M kernels f32[2*160][3][min(16,T)][128]
 struct Layout {
   size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, tiles, h, h_lo, y, xg, dk_counter,
@@ -97,8 +97,12 @@ Layout layout(const moe_q4_layer* L, int T, int k) {
   p = align_up(p + sizeof(__nv_bfloat16) * R * L->I);
   o.y = p;
   p = align_up(p + sizeof(float) * R * L->H);
-  o.xg = p;
-  p = align_up(p + sizeof(__nv_bfloat16) * R * L->H);
+  // grouped activation rows: read by the tensor-core path only (T > 16)
+  o.xg = 0;
+  if (uses_prefill(T)) {
+    o.xg = p;
+    p = align_up(p + sizeof(__nv_bfloat16) * R * L->H);
+  }
   const int max_exp = (int)(R < (size_t)L->E ? R : (size_t)L->E);
   o.dk_units_gu = max_exp * (L->I / 128);
   o.dk_units_dn = max_exp * (L->H / 128);
@@ -155,7 +159,7 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   a.dec_list = (int32_t*)(ws + o.dec_list);
   a.pre_list = (int32_t*)(ws + o.pre_list);
   a.tiles = (int32_t*)(ws + o.tiles);
-  a.xg = (__nv_bfloat16*)(ws + o.xg);
+  a.xg = o.xg ? (__nv_bfloat16*)(ws + o.xg) : nullptr;
   a.dk_counter = (int32_t*)(ws + o.dk_counter);
   a.dk_counter_n = o.dk_units_gu + o.dk_units_dn;
   a.h = (__nv_bfloat16*)(ws + o.h);
