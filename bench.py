@@ -335,6 +335,74 @@ def roofline(work, kern_ms, n_prof, hbm_peak, tf_peak, peak_src):
     return roof, kernels
 
 
+
+def measure_graph(q4, layer, xs, lgs, k, out, ws, flush_l2, steps, stream):
+    """The same forward replayed from CUDA graphs (one per rotating batch):
+    launch gaps between the kernels disappear.  Returns (ms_per_step, None) or
+    (None, reason)."""
+    try:
+        graphs = []
+        for v in range(ROTATE):
+            q4.forward(layer, xs[v], lgs[v], k, out=out, ws=ws)  # warm (host-side lookups)
+        torch.cuda.synchronize()
+        for v in range(ROTATE):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                q4.forward(layer, xs[v], lgs[v], k, out=out, ws=ws)
+            graphs.append(g)
+        for v in range(ROTATE):
+            graphs[v].replay()
+        torch.cuda.synchronize()
+        if q4.forward_status(ws) != 0:
+            return None, "device status after graph replay"
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps):
+            flush_l2(i)
+            st[i].record(stream)
+            graphs[i % ROTATE].replay()
+            en[i].record(stream)
+        torch.cuda.synchronize()
+        ms = sum(a.elapsed_time(b) for a, b in zip(st, en)) / steps
+        del graphs
+        return ms, None
+    except Exception as exc:  # capture unsupported here: report, do not fail the run
+        torch.cuda.synchronize()
+        return None, f"{type(exc).__name__}: {exc}"[:200]
+
+
+def measure_dequant(q4, layer, hbm_peak, flush_l2, stream, reps=5):
+    """Standalone full-layer dequant: every expert's gate, up and down to bf16
+    (three calls, preallocated outputs).  Algorithmic bytes = packed codes +
+    scales read + bf16 written."""
+    parts = [(layer.gate_w, layer.gate_s), (layer.up_w, layer.up_s), (layer.down_w, layer.down_s)]
+    outs = [torch.empty((c.shape[0], c.shape[1], c.shape[2] * 2), dtype=torch.bfloat16, device=c.device)
+            for c, _ in parts]
+    nbytes = sum(c.numel() + s.numel() + o.numel() * 2 for (c, s), o in zip(parts, outs))
+
+    def run():
+        for (c, s), o in zip(parts, outs):
+            q4.dequant(c, s, layer.tables, layer.table_id, out=o)
+
+    for _ in range(3):
+        run()
+    torch.cuda.synchronize()
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    for i in range(reps):
+        flush_l2(i)
+        st[i].record(stream)
+        run()
+        en[i].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in zip(st, en)) / reps
+    del outs
+    torch.cuda.empty_cache()
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"kernel": "dequant_kernel (all 256 x 3 projections -> bf16)", "bytes": nbytes, "ms": ms,
+            "gbs": gbs, "frac": gbs / hbm_peak, "frac_of_8tbs": gbs / 8000.0}
+
+
 def run_ours(args, w):
     import torch.distributed as dist
 
@@ -436,6 +504,8 @@ def run_ours(args, w):
     e2e_value = T * n_e2e * world / (float(e2e_t.item()) / 1e3)
 
     hbm_peak, tf_peak, peak_src = load_peaks()
+    graph_ms, graph_why = measure_graph(q4, layer, xs, lgs, k, out, ws, flush_l2, min(args.steps, 200), stream)
+    dq = measure_dequant(q4, layer, hbm_peak, flush_l2, stream) if not args.no_dequant else None
     work = [kernel_work(sh, T, c) for c in counts]
     roof, kernels = roofline(work, kern_ms, n_prof, hbm_peak, tf_peak, peak_src)
     gu, dn = expert_bytes(sh)
@@ -455,6 +525,10 @@ def run_ours(args, w):
                       "frac_of_peak": layer_bytes / (total_ms / args.steps / 1e3) / 1e9 / hbm_peak},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * sh.H * 2 + T * sh.E * 4,
                 "d2h_bytes_per_step": T * sh.H * 2},
+        "graph": ({"value": T * world / (graph_ms / 1e3), "unit": UNIT, "ms_per_step": graph_ms,
+                   "note": "same forward replayed from CUDA graphs, L2 flushed outside the events"}
+                  if graph_ms else {"value": None, "unavailable": graph_why}),
+        "dequant": dq,
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk.summary(),
     }
@@ -475,6 +549,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode_t1", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dequant", action="store_true", help="skip the standalone full-layer dequant measurement")
     ap.add_argument("--experts", type=int, default=0,
                     help="layer with this many experts (same H, I, top-k) instead of the workload's; "
                          "for small profiling captures")

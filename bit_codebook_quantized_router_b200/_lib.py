@@ -145,12 +145,16 @@ def pack(w: torch.Tensor, tables, table_id, status: torch.Tensor | None = None, 
     return codes, scales
 
 
-def dequant(codes: torch.Tensor, scales: torch.Tensor, tables, table_id, stream=None) -> torch.Tensor:
-    """uint8 codes [E, N, K/2] + scales [E, N, K/32] -> bf16 [E, N, K]."""
+def dequant(codes: torch.Tensor, scales: torch.Tensor, tables, table_id, stream=None,
+            out: torch.Tensor | None = None) -> torch.Tensor:
+    """uint8 codes [E, N, K/2] + scales [E, N, K/32] -> bf16 [E, N, K] (into `out` if given)."""
     E, N, Kh = codes.shape
     K = Kh * 2
     t, tid = _host_tables(tables, table_id, E)
-    out = torch.empty((E, N, K), dtype=torch.bfloat16, device=codes.device)
+    if out is None:
+        out = torch.empty((E, N, K), dtype=torch.bfloat16, device=codes.device)
+    elif out.shape != (E, N, K) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 tensor [E, N, K]")
     _check(lib().moe_q4_dequant(_ptr(codes.contiguous()), _ptr(scales.contiguous()), t.ctypes.data,
                                 t.shape[0], tid.ctypes.data, E, N, K, _ptr(out), _stream(stream)),
            "moe_q4_dequant")
