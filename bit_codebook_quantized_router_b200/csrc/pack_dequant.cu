@@ -91,13 +91,16 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
 }
 
 // ---------------------------------------------------------------------------
-// Dequantisation: one thread per 32-weight block, 64 bytes of bf16 out.
+// Dequantisation: one thread per 32-bit code word (8 weights, 16 bytes of
+// bf16 out), so a warp's loads cover 128 contiguous code bytes and its stores
+// 512 contiguous output bytes; each thread takes kDqWords words a grid stride
+// apart, loads first, so several loads are in flight per thread.
 // Fast path (the block's scale keeps every non-zero level a normal bf16):
-// the bf16-rounded levels get the exponent added once per block, then PRMT
-// byte-plane lookups decode 8 codes per 32-bit word.  Rounding commutes with
-// a power-of-two scale in the normal range, so this equals "fp32 multiply,
-// then RNE to bf16" bit for bit.  Otherwise (subnormal / overflowing
-// results, scale byte 0xFF) every weight takes the literal fp32 path.
+// the bf16-rounded levels get the exponent added, then PRMT byte-plane
+// lookups decode the 8 codes.  Rounding commutes with a power-of-two scale in
+// the normal range, so this equals "fp32 multiply, then RNE to bf16" bit for
+// bit.  Otherwise (subnormal / overflowing results, scale byte 0xFF) every
+// weight takes the literal fp32 path.
 // ---------------------------------------------------------------------------
 struct DequantTable {
   uint32_t b[8];     // bf16 bits of each level (RNE)
@@ -105,9 +108,42 @@ struct DequantTable {
   int has_sub;       // a non-zero level that is a bf16 subnormal
 };
 
+constexpr int kDqWords = 4;
+
+__device__ __forceinline__ void dequant_word(uint32_t cw, uint32_t s, const DequantTable& d, const float* t,
+                                             uint32_t res[4]) {
+  const int e = (int)s - 127;
+  // emin + e >= 2 keeps even the unrounded fp32 level times 2^e normal.
+  if (!d.has_sub && s != 255u && d.emin + e >= 2 && d.emax + e <= 254) {
+    uint32_t bb[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bb[i] = d.b[i] ? (uint32_t)((int)d.b[i] + e * 128) : 0u;
+    const uint32_t w01 = bb[0] | (bb[1] << 16), w23 = bb[2] | (bb[3] << 16);
+    const uint32_t w45 = bb[4] | (bb[5] << 16), w67 = bb[6] | (bb[7] << 16);
+    Planes p;
+    p.l0 = prmt(w01, w23, 0x6420);
+    p.h0 = prmt(w01, w23, 0x7531);
+    p.l1 = prmt(w45, w67, 0x6420);
+    p.h1 = prmt(w45, w67, 0x7531);
+    decode8(cw, p, res);
+  } else {
+    const float mult = __uint_as_float(s == 0u ? 0x00400000u : (s << 23));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t code = (cw >> (4 * i)) & 0xfu;
+      uint32_t bits = (s == 255u) ? 0x7fc0u : (uint32_t)bf16_bits_rn(__fmul_rn(t[code & 7], mult));
+      if (code & 8u) bits ^= 0x8000u;
+      if (i & 1)
+        res[i >> 1] |= bits << 16;
+      else
+        res[i >> 1] = bits;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict__ codes,
                                                       const uint8_t* __restrict__ scales,
-                                                      int64_t n_blocks, int N, int K,
+                                                      int64_t n_words, int N, int K,
                                                       const __grid_constant__ TableParams tp,
                                                       uint16_t* __restrict__ out) {
   __shared__ DequantTable st[kMaxTables];
@@ -131,49 +167,27 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
     st[threadIdx.x] = d;
   }
   __syncthreads();
-  const int bpr = K / kBlockK;
-  for (int64_t b = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; b < n_blocks;
-       b += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = b / bpr;
-    const int tid = tp.id[(int)(row / N)];
-    const uint32_t s = scales[b];
-    const uint4 c = ldg_stream(codes + b * 16);
-    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-    uint32_t res[16];
-    const DequantTable& d = st[tid];
-    const int e = (int)s - 127;
-    // emin + e >= 2 keeps even the unrounded fp32 level times 2^e normal.
-    if (!d.has_sub && s != 255u && d.emin + e >= 2 && d.emax + e <= 254) {
-      uint32_t bb[8];
+  const uint64_t words_per_expert = (uint64_t)N * (uint64_t)(K / 8);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t w0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; w0 < n_words; w0 += stride * kDqWords) {
+    uint32_t cw[kDqWords], sc[kDqWords];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) bb[i] = d.b[i] ? (uint32_t)((int)d.b[i] + e * 128) : 0u;
-      const uint32_t w01 = bb[0] | (bb[1] << 16), w23 = bb[2] | (bb[3] << 16);
-      const uint32_t w45 = bb[4] | (bb[5] << 16), w67 = bb[6] | (bb[7] << 16);
-      Planes p;
-      p.l0 = prmt(w01, w23, 0x6420);
-      p.h0 = prmt(w01, w23, 0x7531);
-      p.l1 = prmt(w45, w67, 0x6420);
-      p.h1 = prmt(w45, w67, 0x7531);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) decode8(cw[q], p, &res[4 * q]);
-    } else {
-      const float* t = tp.t[tid];
-      const float mult = __uint_as_float(s == 0u ? 0x00400000u : (s << 23));
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const uint32_t code = (cw[i >> 3] >> ((i & 7) * 4)) & 0xfu;
-        uint32_t bits = (s == 255u) ? 0x7fc0u : (uint32_t)bf16_bits_rn(__fmul_rn(t[code & 7], mult));
-        if (code & 8u) bits ^= 0x8000u;
-        if (i & 1)
-          res[i >> 1] |= bits << 16;
-        else
-          res[i >> 1] = bits;
+    for (int u = 0; u < kDqWords; ++u) {
+      const int64_t w = w0 + u * stride;
+      if (w < n_words) {
+        cw[u] = __ldcs(reinterpret_cast<const unsigned int*>(codes) + w);
+        sc[u] = __ldg(scales + (w >> 2));  // 4 words per 32-weight block
       }
     }
-    uint4* dst = reinterpret_cast<uint4*>(out + b * kBlockK);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      dst[q] = make_uint4(res[4 * q], res[4 * q + 1], res[4 * q + 2], res[4 * q + 3]);
+    for (int u = 0; u < kDqWords; ++u) {
+      const int64_t w = w0 + u * stride;
+      if (w >= n_words) break;
+      const int tid = tp.n == 1 ? 0 : tp.id[(int)((uint64_t)w / words_per_expert)];
+      uint32_t res[4];
+      dequant_word(cw[u], sc[u], st[tid], tp.t[tid], res);
+      __stcs(reinterpret_cast<uint4*>(out) + w, make_uint4(res[0], res[1], res[2], res[3]));
+    }
   }
 }
 
@@ -210,11 +224,11 @@ extern "C" int moe_q4_dequant(const uint8_t* weight, const uint8_t* weight_scale
   int rc = q4_fill_tables(&tp, tables, n_tables, table_id, E);
   if (rc != MOE_Q4_OK) return rc;
   if (((uintptr_t)weight & 15) || ((uintptr_t)out & 15)) return MOE_Q4_EINVAL;
-  const int64_t n_blocks = (int64_t)E * N * (K / kBlockK);
+  const int64_t n_words = (int64_t)E * N * (K / 8);
   const int threads = 256;
-  const int64_t want = (n_blocks + threads - 1) / threads;
-  const int grid = (int)(want < 148 * 16 ? want : 148 * 16);
-  dequant_kernel<<<grid, threads, 0, (cudaStream_t)stream>>>(weight, weight_scale, n_blocks, N, K,
+  const int64_t want = (n_words + threads * kDqWords - 1) / (threads * kDqWords);
+  const int grid = (int)(want < 148 * 8 ? want : 148 * 8);
+  dequant_kernel<<<grid, threads, 0, (cudaStream_t)stream>>>(weight, weight_scale, n_words, N, K,
                                                               tp, (uint16_t*)out);
   return cudaGetLastError() == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
 }
