@@ -21,11 +21,9 @@
 //   expert's activation rows, straight from x through the row -> token map,
 //   with cp.async, completing on the stage barrier; the down projection's h
 //   rows come by TMA.
-// * Decode + MMA (warps 1..16): warp (s, part) owns weight rows 16s..16s+15
-//   of the tile and, for gate/up, one matrix (part 0 gate, part 1 up) over
-//   the whole stage, for down one 128-K half of each stage.  In a 128-K half,
-//   lane (g, t) reads the 16-byte code chunk t of rows g and g+8 (32 weights,
-//   one E8M0 block), decodes it to bf16 pairs ("aidendle94/GLM-5.2-NF4-Lloyd-
+// * Decode + MMA (warps 1..8): warp s owns weight rows 16s..16s+15 of the
+//   tile.  In each 128-K half of a stage, lane (g, t) reads the 16-byte code
+//   chunk t of rows g and g+8 (32 weights, one E8M0 block), decodes it to bf16 pairs ("aidendle94/GLM-5.2-NF4-Lloyd-
 //   Experts-GPTQ", "Codes are indices into the per-layer grid") and feeds
 //   them to mma.sync m16n8k16 as the A operand.  K is permuted inside each
 //   128-K half, the same way for weights and activations (a sum over K does
@@ -46,11 +44,8 @@
 //   by h and by its low part h_lo (y = W h + W h_lo): with T <= 4 one n-tile
 //   holds h in columns 0..3 and h_lo in 4..7, else separate tiles accumulate
 //   into the same registers.
-// * At the end of a segment part 1 hands its sums to part 0 through shared
-//   memory (up -> gate; the second K half -> the first, added in a fixed
-//   order), and part 0 finishes the rows: SwiGLU and h / h_lo, or y, or a
-//   partial sum for a tile shared with other CTAs.  Sixteen compute warps
-//   (four per scheduler) hide the latencies of the decode chains.
+// * At the end of a segment the warp finishes its rows: SwiGLU and h / h_lo,
+//   or y, or a partial sum for a tile shared with other CTAs.
 //
 // Every wait is bounded (a timeout sets MOE_Q4_ETIMEOUT in the status word and
 // the CTA drains and exits); warps wait and leave together (vote).
@@ -65,7 +60,7 @@ namespace q4 {
 using namespace sm100;
 
 namespace dk {
-constexpr int kComputeWarps = 16;                    // 8 row slabs x 2 parts
+constexpr int kComputeWarps = 8;                     // one 16-row slab each
 constexpr int kThreads = 32 * (1 + kComputeWarps);   // + the producer warp
 constexpr int kRows = 128;                           // weight rows per tile
 constexpr int kMaxRing = 6;                          // shared-memory stages, at most
@@ -83,11 +78,10 @@ struct DkCfg {
   static constexpr int kAtoms = GATEUP ? NT : (NT == 4 ? 4 : 2);
   // 8-token groups of the result
   static constexpr int kTT = GATEUP ? NT : (NT == 4 ? 2 : 1);
-  // independent accumulators per token group, so no MMA waits on the one
-  // before it for long: gate/up MMA mm of K half J adds into chain 2J + (mm & 1)
-  // (or J), down into mm & 3 (or mm & 1); added in a fixed order at the end
-  static constexpr int kChains = kTT == 1 ? 4 : 2;
-  static constexpr int kXch = kTT * 4;  // floats per lane handed from part 1 to part 0
+  // independent accumulators per (matrix, token group): MMA mm of K half J adds
+  // into chain 2J + (mm & 1) (or J), so no MMA waits on the one before it for
+  // long; the chains are added in a fixed order at the end
+  static constexpr int kChains = (kMats * kTT <= 2 && NT <= 2) ? 4 : 2;
 };
 
 // Shared-memory placement, as offsets from the start of the CTA's dynamic
@@ -98,17 +92,17 @@ struct DkCfg {
 // deeper ring keeps more bytes in flight per SM).  The host computes it for
 // the window start it expects; the kernel checks alignment and size.
 struct DkLayout {
-  uint32_t lut, code_hi, code_lo, x, scales, xch, bars, end;
+  uint32_t lut, code_hi, code_lo, x, scales, bars, end;
   int n_hi;  // code stages at code_hi; stages n_hi.. at code_lo
 };
 
 static bool dk_layout(uint32_t raw, uint32_t limit, uint32_t code_stage, uint32_t x_stage, uint32_t scale_stage,
-                      uint32_t xch_bytes, int ring, DkLayout& L) {
+                      int ring, DkLayout& L) {
   const uint32_t lut = (raw + 65535u) & ~65535u;
   const uint32_t o = (raw + 1023u) & ~1023u;
   const uint32_t hi = lut + dk::kLutBytes;
   if (hi > limit) return false;
-  const uint32_t others = (uint32_t)ring * (x_stage + scale_stage) + xch_bytes + dk::kBarBytes;
+  const uint32_t others = (uint32_t)ring * (x_stage + scale_stage) + dk::kBarBytes;
   const int fit_hi = (int)((limit - hi) / code_stage);
   uint32_t x;
   if (o + others <= lut) {
@@ -132,15 +126,13 @@ static bool dk_layout(uint32_t raw, uint32_t limit, uint32_t code_stage, uint32_
   L.lut = lut;
   L.x = x;
   L.scales = x + (uint32_t)ring * x_stage;
-  L.xch = L.scales + (uint32_t)ring * scale_stage;
-  L.bars = L.xch + xch_bytes;
+  L.bars = L.scales + (uint32_t)ring * scale_stage;
   // offsets from the window start
   L.lut -= raw;
   L.code_hi -= raw;
   L.code_lo -= raw;
   L.x -= raw;
   L.scales -= raw;
-  L.xch -= raw;
   L.bars -= raw;
   L.end -= raw;
   return true;
@@ -204,6 +196,17 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
   return v;
 }
 
+// 16-byte shared load by the lanes with `pred` set; the others get zeros and
+// touch no shared memory.
+__device__ __forceinline__ void lds128_if(uint32_t addr, uint32_t pred, uint32_t& x, uint32_t& y, uint32_t& z,
+                                          uint32_t& w) {
+  asm("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %5, 0;\n\t"
+      "mov.b32 %0, 0;\n\tmov.b32 %1, 0;\n\tmov.b32 %2, 0;\n\tmov.b32 %3, 0;\n\t"
+      "@p ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];\n\t}"
+      : "=&r"(x), "=&r"(y), "=&r"(z), "=&r"(w)
+      : "r"(addr), "r"(pred));
+}
+
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
   asm("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
@@ -234,15 +237,15 @@ __device__ __forceinline__ void mma_bf16_16816(float c[4], uint32_t a0, uint32_t
 
 // Table slot `slot`: entry c -> bf16 pair of codes (c & 15, c >> 4), signed,
 // unscaled, one copy per lane (entry c of lane l at c * 256 + slot * 128 +
-// l * 4).  Thread (ent, half) writes the copies of lanes 16 half .. + 15.
-__device__ __forceinline__ void build_lut_slot(uint8_t* lut, const float* tv, int slot, int ent, int half) {
+// l * 4).  Thread ent (0..255) writes entry ent.
+__device__ __forceinline__ void build_lut_slot(uint8_t* lut, const float* tv, int slot, int ent) {
   const uint32_t lo = ent & 15, hi = ent >> 4;
   const uint32_t blo = (uint32_t)bf16_bits_rn(tv[lo & 7]) ^ ((lo & 8) ? 0x8000u : 0u);
   const uint32_t bhi = (uint32_t)bf16_bits_rn(tv[hi & 7]) ^ ((hi & 8) ? 0x8000u : 0u);
   const uint32_t word = blo | (bhi << 16);
-  uint4* dst = reinterpret_cast<uint4*>(lut + ent * 256 + slot * 128 + half * 64);
+  uint4* dst = reinterpret_cast<uint4*>(lut + ent * 256 + slot * 128);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) dst[i] = make_uint4(word, word, word, word);
+  for (int i = 0; i < 8; ++i) dst[i] = make_uint4(word, word, word, word);
 }
 
 // 16 bf16 pairs of one code chunk (4 words, pair 4w + b from byte b of word
@@ -282,7 +285,6 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   Ls.code_lo += raw_s;
   Ls.x += raw_s;
   Ls.scales += raw_s;
-  Ls.xch += raw_s;
   Ls.bars += raw_s;
   const FwdArgs& a = P.a;
   if (P.lay.end > dynamic_smem_size() || (Ls.lut & 0xffffu) != 0u) {
@@ -297,10 +299,8 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + (Ls.bars - raw_s));
   uint64_t* full = bars;                          // [ring] codes (+ h: TMA), scales (+ x: cp.async)
   uint64_t* stage_empty = full + dk::kMaxRing;    // [ring] compute warps done with the stage
-  uint64_t* xfull = stage_empty + dk::kMaxRing;   // [8] part 1 of slab s wrote its sums
-  uint64_t* xfree = xfull + 8;                    // [8] part 0 of slab s read them
-  uint64_t* lut_bar = xfree + 8;                  // compute threads rebuilding a table slot
-  uint64_t* epi_bar = lut_bar + 1;                // part-0 threads finishing a split tile
+  uint64_t* lut_bar = stage_empty + dk::kMaxRing; // compute threads rebuilding a table slot
+  uint64_t* epi_bar = lut_bar + 1;                // compute threads finishing a split tile
   volatile int* abort_flag = reinterpret_cast<volatile int*>(epi_bar + 1);
   volatile int* last_flag = abort_flag + 1;
 
@@ -311,12 +311,8 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       mbar_init(&full[s], 1 + 32);  // producer lane 0 (with the TMA bytes) + 32 cp.async arrivals
       mbar_init(&stage_empty[s], dk::kComputeWarps);
     }
-    for (int i = 0; i < 8; ++i) {
-      mbar_init(&xfull[i], 32);
-      mbar_init(&xfree[i], 32);
-    }
     mbar_init(lut_bar, 32 * dk::kComputeWarps);
-    mbar_init(epi_bar, 32 * 8);
+    mbar_init(epi_bar, 32 * dk::kComputeWarps);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_wa);
@@ -328,7 +324,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   }
   // with a single table every expert uses table 0: its table slot is built
   // before waiting for the previous kernel
-  if (tp.n == 1 && warp >= 1) build_lut_slot(lut, tp.t[0], 0, (threadIdx.x - 32) & 255, (threadIdx.x - 32) >> 8);
+  if (tp.n == 1 && warp >= 1) build_lut_slot(lut, tp.t[0], 0, threadIdx.x - 32);
   __syncthreads();
 
   pdl_wait();
@@ -434,27 +430,29 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     }
   } else {
     // ------------------------------ compute ------------------------------
-    const int cw = warp - 1;        // 0..15
-    const int slab = cw & 7;        // rows 16 slab .. + 15 of the tile
-    const int part = cw >> 3;       // gate/up: matrix (0 gate, 1 up); down: K half of a stage
-    const int mat = GATEUP ? part : 0;
-    const int gq = lane >> 2;       // MMA group: rows gq, gq + 8; token column gq
-    const int tq = lane & 3;        // code chunk of a half; token columns 2tq, 2tq + 1
-    const int ctid = threadIdx.x - 32;  // 0..511
-    const int n_halves = subs / 2;  // 128-K halves per stage
-    // the halves this warp reads: gate/up all, down its own (none when a
-    // 128-K stage has no second half)
-    const int J_lo = GATEUP ? 0 : part;
-    const int J_hi = GATEUP ? n_halves : (part < n_halves ? part + 1 : part);
+    const int slab = warp - 1;     // rows 16 slab .. + 15 of the tile
+    const int gq = lane >> 2;      // MMA group: rows gq, gq + 8; token column gq
+    const int tq = lane & 3;       // code chunk of a half; token columns 2tq, 2tq + 1
+    const int ctid = threadIdx.x - 32;
+    const int n_halves = subs / 2; // 128-K halves per stage
     const int r0 = 16 * slab + gq, r1 = r0 + 8;
     const int swz0 = subs == 4 ? (r0 & 7) : ((r0 >> 1) & 3);
     const int swz1 = subs == 4 ? (r1 & 7) : ((r1 >> 1) & 3);
-    const uint32_t moff = (uint32_t)(mat * dk::kRows * row_bytes);                  // this matrix's codes
-    const uint32_t soff0 = (uint32_t)((mat * dk::kRows + r0) * dk::kScaleSlot);      // its scale rows
-    const uint32_t soff1 = (uint32_t)((mat * dk::kRows + r1) * dk::kScaleSlot);
-    float* xch = reinterpret_cast<float*>(smem_raw + (Ls.xch - raw_s)) + (size_t)slab * C::kXch * 32;
+    // per-lane offsets inside a stage: code chunk 4J + tq of rows r0 / r1, and
+    // this lane's activation run (super-step 2J + (tq >> 1), row gq, chunks
+    // 4 (tq & 1) .. +3 in the 128-byte swizzle)
+    uint32_t coff[2][2], xoff[2][4];
+#pragma unroll
+    for (int J = 0; J < 2; ++J) {
+      const int chunk = 4 * J + tq;
+      coff[J][0] = (uint32_t)(r0 * row_bytes + ((chunk ^ swz0) << 4));
+      coff[J][1] = (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4));
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        xoff[J][c] = (uint32_t)((2 * J + (tq >> 1)) * C::kAtoms * 1024 + gq * 128 + ((((tq & 1) * 4 + c) ^ gq) << 4));
+    }
     int slot_tab0 = tp.n == 1 ? 0 : -1, slot_tab1 = -1, victim = tp.n == 1 ? 1 : 0;
-    uint32_t lgen = 0, egen = 0, xgen = 0;
+    uint32_t lgen = 0, egen = 0;
     const uint32_t lane_k = (Ls.lut & 0xffff0000u) | ((uint32_t)lane << 2);
     int s = 0;
     uint32_t ph = 0;
@@ -469,9 +467,10 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       const int tid = tp.id[e];
       int slot = tid == slot_tab0 ? 0 : (tid == slot_tab1 ? 1 : -1);
       if (slot < 0) {
-        // (re)build a slot.  Bounded barriers on both sides: every compute
-        // thread is done with the old contents before any write, and all writes
-        // land before anyone reads.
+        // (re)build a slot: entry c -> bf16 pair of codes (c & 15, c >> 4), signed,
+        // unscaled, one copy per lane.  Bounded barriers on both sides: every
+        // compute thread is done with the old contents before any write, and all
+        // writes land before anyone reads.
         mbar_arrive(lut_bar);
         if (!mbar_wait_warp(lut_bar, lgen & 1, abort_flag, dk::kWaitNs)) break;
         ++lgen;
@@ -481,39 +480,53 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           slot_tab0 = tid;
         else
           slot_tab1 = tid;
-        build_lut_slot(lut, tp.t[tid], slot, ctid & 255, ctid >> 8);
+        build_lut_slot(lut, tp.t[tid], slot, ctid);
         mbar_arrive(lut_bar);
         if (!mbar_wait_warp(lut_bar, lgen & 1, abort_flag, dk::kWaitNs)) break;
         ++lgen;
       }
       const uint32_t kreg = lane_k | ((uint32_t)slot << 7);
       const Planes PL = make_planes(tp.t[tid]);
-
-      float accc[C::kTT][C::kChains][4];
+      // activation rows of absent tokens are not read (their operands are zero;
+      // their MMA columns are never written)
+      const int n_e_seg = a.counts[e];
+      uint32_t col_ok[NT];
 #pragma unroll
-      for (int tt = 0; tt < C::kTT; ++tt)
+      for (int nt = 0; nt < NT; ++nt) {
+        int tok;
+        if (GATEUP)
+          tok = 8 * nt + gq;
+        else if (NT == 1)
+          tok = gq & 3;
+        else if (NT == 2)
+          tok = gq;
+        else
+          tok = 8 * (nt & 1) + gq;
+        col_ok[nt] = tok < n_e_seg ? 1u : 0u;
+      }
+      float accc[kMats][C::kTT][C::kChains][4];
 #pragma unroll
-        for (int c = 0; c < C::kChains; ++c)
+      for (int m = 0; m < kMats; ++m)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) accc[tt][c][i] = 0.0f;
+        for (int tt = 0; tt < C::kTT; ++tt)
+#pragma unroll
+          for (int c = 0; c < C::kChains; ++c)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) accc[m][tt][c][i] = 0.0f;
 
       for (int j = 0; j < nst && ok; ++j) {
         if (!mbar_wait_warp(&full[s], ph, abort_flag, dk::kWaitNs)) {
           ok = false;
           break;
         }
-        const uint32_t cbase = after_wait(code_base(s)) + moff;
+        const uint32_t cbase = after_wait(code_base(s));
         const uint32_t sbase = after_wait(Ls.scales + (uint32_t)s * P.scale_stage);
         const uint32_t xstage = after_wait(Ls.x + (uint32_t)s * P.x_stage);
         uint32_t dep = 0;  // every word read from the stage, folded
-        const uint2 s0 = lds64(sbase + soff0);
-        const uint2 s1 = lds64(sbase + soff1);
-        dep ^= s0.x ^ s1.x;
 #pragma unroll
         for (int J = 0; J < 2; ++J) {
-          if (J < J_lo || J >= J_hi) continue;
+          if (J >= n_halves) break;
           // activation operands: 16 pairs per n-tile, pair p at K offset 32 tq + 2p
-          const uint32_t xrow = xstage + (uint32_t)(2 * J + (tq >> 1)) * C::kAtoms * 1024 + (uint32_t)gq * 128;
           uint32_t xr[NT][16];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
@@ -526,33 +539,34 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
               atom = nt;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              const uint4 v = lds128(xrow + (uint32_t)atom * 1024 + ((((tq & 1) * 4 + c) ^ gq) << 4));
-              xr[nt][4 * c + 0] = v.x;
-              xr[nt][4 * c + 1] = v.y;
-              xr[nt][4 * c + 2] = v.z;
-              xr[nt][4 * c + 3] = v.w;
-              dep ^= v.x;
+              lds128_if(xstage + (uint32_t)atom * 1024 + xoff[J][c], col_ok[nt], xr[nt][4 * c + 0],
+                        xr[nt][4 * c + 1], xr[nt][4 * c + 2], xr[nt][4 * c + 3]);
+              dep ^= xr[nt][4 * c + 0];
             }
           }
-          const int chunk = 4 * J + tq;  // 16-byte chunk of the stage row
-          const uint4 c0 = lds128(cbase + (uint32_t)(r0 * row_bytes + ((chunk ^ swz0) << 4)));
-          const uint4 c1 = lds128(cbase + (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4)));
-          dep ^= c0.x ^ c1.x;
-          // E8M0 byte of block 4J + tq
-          const uint32_t e0 = ((J ? s0.y : s0.x) >> (8 * tq)) & 0xffu;
-          const uint32_t e1 = ((J ? s1.y : s1.x) >> (8 * tq)) & 0xffu;
-          uint32_t pa[16], pb[16];
-          decode_chunk(c0, PL, kreg, scale_bf16x2(e0), pa);
-          decode_chunk(c1, PL, kreg, scale_bf16x2(e1), pb);
 #pragma unroll
-          for (int mm = 0; mm < 8; ++mm) {
+          for (int m = 0; m < kMats; ++m) {
+            const uint32_t mb = cbase + (uint32_t)(m * dk::kRows * row_bytes);
+            const uint4 c0 = lds128(mb + coff[J][0]);
+            const uint4 c1 = lds128(mb + coff[J][1]);
+            const uint2 s0 = lds64(sbase + (uint32_t)((m * dk::kRows + r0) * dk::kScaleSlot));
+            const uint2 s1 = lds64(sbase + (uint32_t)((m * dk::kRows + r1) * dk::kScaleSlot));
+            dep ^= c0.x ^ c1.x ^ s0.x ^ s1.x;
+            // E8M0 byte of block 4J + tq
+            const uint32_t e0 = ((J ? s0.y : s0.x) >> (8 * tq)) & 0xffu;
+            const uint32_t e1 = ((J ? s1.y : s1.x) >> (8 * tq)) & 0xffu;
+            uint32_t pa[16], pb[16];
+            decode_chunk(c0, PL, kreg, scale_bf16x2(e0), pa);
+            decode_chunk(c1, PL, kreg, scale_bf16x2(e1), pb);
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-              const int tt = GATEUP ? nt : (NT == 4 ? (nt & 1) : 0);
-              const int ch = C::kChains == 4 ? (GATEUP ? 2 * J + (mm & 1) : (mm & 3))
-                                             : (GATEUP ? J : (mm & 1));
-              mma_bf16_16816(accc[tt][ch], pa[2 * mm], pb[2 * mm], pa[2 * mm + 1], pb[2 * mm + 1],
-                             xr[nt][2 * mm], xr[nt][2 * mm + 1]);
+            for (int mm = 0; mm < 8; ++mm) {
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) {
+                const int tt = GATEUP ? nt : (NT == 4 ? (nt & 1) : 0);
+                const int ch = C::kChains == 4 ? 2 * J + (mm & 1) : J;
+                mma_bf16_16816(accc[m][tt][ch], pa[2 * mm], pb[2 * mm], pa[2 * mm + 1], pb[2 * mm + 1],
+                               xr[nt][2 * mm], xr[nt][2 * mm + 1]);
+              }
             }
           }
         }
@@ -564,45 +578,18 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       }
       if (!ok) break;
 
-      float mine[C::kTT][4];
+      float acc[kMats][C::kTT][4];
 #pragma unroll
-      for (int tt = 0; tt < C::kTT; ++tt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          float v = accc[tt][0][i];
-#pragma unroll
-          for (int c = 1; c < C::kChains; ++c) v += accc[tt][c][i];
-          mine[tt][i] = v;
-        }
-
-      // ---- segment end: part 1 hands its sums to part 0 ----
-      if (part == 1) {
-        if (xgen > 0 && !mbar_wait_warp(&xfree[slab], (xgen - 1) & 1, abort_flag, dk::kWaitNs)) break;
+      for (int m = 0; m < kMats; ++m)
 #pragma unroll
         for (int tt = 0; tt < C::kTT; ++tt)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) xch[(tt * 4 + i) * 32 + lane] = mine[tt][i];
-        mbar_arrive(&xfull[slab]);
-        ++xgen;
-        g = seg_end;
-        continue;
-      }
-      if (!mbar_wait_warp(&xfull[slab], xgen & 1, abort_flag, dk::kWaitNs)) break;
-      float acc[kMats][C::kTT][4];  // gate/up: [0] gate (own), [1] up (part 1); down: own + second half
+          for (int i = 0; i < 4; ++i) {
+            float v = accc[m][tt][0][i];
 #pragma unroll
-      for (int tt = 0; tt < C::kTT; ++tt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float other = xch[(tt * 4 + i) * 32 + lane];
-          if (GATEUP) {
-            acc[0][tt][i] = mine[tt][i];
-            acc[kMats - 1][tt][i] = other;
-          } else {
-            acc[0][tt][i] = mine[tt][i] + other;
+            for (int c = 1; c < C::kChains; ++c) v += accc[m][tt][c][i];
+            acc[m][tt][i] = v;
           }
-        }
-      mbar_arrive(&xfree[slab]);
-      ++xgen;
       if (!GATEUP && NT == 1) {
         // columns 4..7 hold W h_lo for tokens 0..3: add them to columns 0..3
 #pragma unroll
@@ -751,7 +738,6 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
   P.code_stage = (uint32_t)(C::kMats * dk::kRows * 32 * P.subs);
   P.x_stage = (uint32_t)(P.subs * C::kAtoms * 1024);
   P.scale_stage = (uint32_t)(C::kMats * dk::kRows * dk::kScaleSlot);
-  const uint32_t xch_bytes = (uint32_t)(8 * C::kXch * 32 * sizeof(float));
   P.partial = partial;
   P.counter = counter;
 
@@ -764,7 +750,7 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
   P.ring = 0;
   for (int rs = dk::kMaxRing; rs >= 2 && !P.ring; --rs)
     if (dk_layout((uint32_t)reserved, (uint32_t)reserved + (uint32_t)optin, P.code_stage, P.x_stage, P.scale_stage,
-                  xch_bytes, rs, P.lay))
+                  rs, P.lay))
       P.ring = rs;
   if (!P.ring) return MOE_Q4_ECUDA;
   const uint32_t smem = P.lay.end;
