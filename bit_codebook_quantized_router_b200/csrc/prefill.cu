@@ -6,10 +6,13 @@
 // decisions" 4 and 6), for the experts whose row count exceeds the streaming
 // path's limit.
 //
-// Swap-AB grouped GEMM: the MMA's M = 128 weight rows, N = a tile of BN
-// tokens of one expert, K streamed in steps of 64.  A persistent CTA per SM
-// walks tiles ordered (expert, weight m-tile, token tile) so the token tiles
-// of one weight tile run back to back and re-read it from L2.
+// Swap-AB grouped GEMM: the MMA's M = 128 weight rows, N = a tile of up to
+// BN = 256 tokens of one expert (the expert's last tile takes N = its
+// remaining rows rounded up to 16), K streamed in steps of 64.  Each decoded
+// 128 x 64 weight tile feeds N = 256 columns of MMA work, so the tensor core,
+// not the decode, sets the pace.  A persistent CTA per SM walks tiles ordered
+// (expert, weight m-tile, token tile) so the token tiles of one weight tile
+// run back to back and re-read it from L2.
 //
 // Warp roles (448 threads):
 //   warp 0       TMA producer: packed codes of the m-tile (128 rows x 32 B per
@@ -17,7 +20,8 @@
 //                128-byte swizzle) into a 3-4 stage ring;
 //   warp 1       allocates TMEM and issues tcgen05.mma (one thread): for each
 //                k-step, 4 MMAs of K=16 per weight matrix into fp32 TMEM
-//                accumulators, double-buffered across tiles;
+//                accumulators (gate + up fill all 512 columns: one buffer;
+//                down: double-buffered across tiles);
 //   warps 2..9   dequantise: codes -> bf16 through the PRMT byte-plane lookup
 //                of the expert's table, E8M0 scale by an exact bf16x2
 //                multiply, stored to smem in the canonical 128-byte-swizzle
@@ -39,7 +43,7 @@ namespace q4 {
 
 using namespace sm100;
 
-constexpr int kBN = 128;          // token tile (MMA N)
+constexpr int kBN = 256;          // token tile (largest MMA N)
 constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBK = 64;           // K per pipeline stage (128 bytes of bf16)
 constexpr int kThreads = 448;
@@ -55,7 +59,8 @@ struct TcCfg {
   static constexpr int kBTile = kBN * kBK * 2;        // 16 KB
   static constexpr int kCTile = kBM * kBK / 2;        // 4 KB codes per matrix
   static constexpr int kStageBytes = kMats * kATile + kBTile + kMats * kCTile;
-  static constexpr int kTmemCols = 2 * kMats * kBN;   // double-buffered accumulators
+  static constexpr int kAccBufs = GATEUP ? 1 : 2;     // TMEM holds 512 columns
+  static constexpr int kTmemCols = kAccBufs * kMats * kBN;
   static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 1024 /*barriers*/;
 };
 
@@ -116,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&a_ready[s], kDequantThreads / 32);  // one arrival per dequant warp
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 4);
     }
@@ -167,11 +172,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idesc = umma_idesc_bf16(kBM, kBN);
       uint32_t it = 0, tcount = 0;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
-        const int buf = tcount & 1;
-        if (!mbar_wait(&acc_empty[buf], ((tcount >> 1) & 1) ^ 1, abort_flag, kWaitLimitNs)) break;
+        int p, m, nt;
+        tile_coords(a, P.m_tiles, np, tile, p, m, nt);
+        const int left = a.counts[a.pre_list[p]] - nt * kBN;  // tokens in this tile and after
+        const int n_cols = left >= kBN ? kBN : ((left + 15) & ~15);
+        const uint32_t idesc = umma_idesc_bf16(kBM, n_cols);
+        const int buf = (int)(tcount % C::kAccBufs);
+        const uint32_t use = tcount / C::kAccBufs;  // earlier uses of this buffer
+        if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1, abort_flag, kWaitLimitNs)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + buf * (C::kMats * kBN);
         bool ok = true;
@@ -268,13 +278,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int e = a.pre_list[p];
       const int n_e = a.counts[e];
       const int row0 = a.offsets[e];
-      const int buf = tcount & 1;
-      if (!mbar_wait_warp(&acc_full[buf], (tcount >> 1) & 1, abort_flag, kWaitLimitNs)) break;
+      const int buf = (int)(tcount % C::kAccBufs);
+      const uint32_t use = tcount / C::kAccBufs;
+      if (!mbar_wait_warp(&acc_full[buf], use & 1, abort_flag, kWaitLimitNs)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * (C::kMats * kBN);
       const int wrow = m * kBM + row;
+      const int n_hi = n_e - nt * kBN < kBN ? n_e - nt * kBN : kBN;  // tokens of this tile
 #pragma unroll 1
-      for (int c0 = 0; c0 < kBN; c0 += 32) {
+      for (int c0 = 0; c0 < n_hi; c0 += 32) {
         float g[32];
         tmem_ld32(tb + c0, g);
         if (GATEUP) {
