@@ -46,14 +46,16 @@ using namespace sm100;
 constexpr int kBN = 256;          // token tile (largest MMA N)
 constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBK = 64;           // K per pipeline stage (128 bytes of bf16)
-constexpr int kThreads = 448;
-constexpr int kDequantThreads = 256;
-constexpr int kEpiWarp0 = 10;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 template <bool GATEUP>
 struct TcCfg {
   static constexpr int kMats = GATEUP ? 2 : 1;
+  // dequant warps: one 16-byte code chunk (32 weights) per thread per k-step:
+  // gate/up 2 matrices x 128 rows x 2 chunks, down 128 rows x 2 chunks
+  static constexpr int kDequantThreads = kMats * 256;
+  static constexpr int kEpiWarp0 = 2 + kDequantThreads / 32;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
   static constexpr int kStages = GATEUP ? 3 : 4;
   static constexpr int kATile = kBM * kBK * 2;        // 16 KB bf16 per matrix
   static constexpr int kBTile = kBN * kBK * 2;        // 16 KB
@@ -90,7 +92,7 @@ __device__ __forceinline__ void tile_coords(const FwdArgs& a, int m_tiles, int n
 }
 
 template <bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ TcParams P, const __grid_constant__ TableParams tp,
                    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_wa,
                    const __grid_constant__ CUtensorMap tm_wb) {
@@ -118,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full_c[s], 1);
       mbar_init(&full_b[s], 1);
-      mbar_init(&a_ready[s], kDequantThreads / 32);  // one arrival per dequant warp
+      mbar_init(&a_ready[s], C::kDequantThreads / 32);  // one arrival per dequant warp
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
@@ -211,26 +213,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(drain);
       mbar_wait(drain, 0, abort_flag, kWaitLimitNs);
     }
-  } else if (warp < kEpiWarp0) {
+  } else if (warp < C::kEpiWarp0) {
     // ---------------- dequantise ----------------
-    const int d = threadIdx.x - 64;           // 0..255
+    const int d = threadIdx.x - 64;           // 0 .. kDequantThreads - 1
     const int r = d & (kBM - 1);              // weight row in the tile
-    const int part = d >> 7;                  // gate/up: matrix; down: K half
+    const int my_half = (d >> 7) & 1;         // 32-weight half of the row's 64 K
+    const int mat = GATEUP ? (d >> 8) : 0;    // gate / up
     uint32_t it = 0;
     for (int tile = blockIdx.x; tile < total && !warp_aborted(abort_flag); tile += gridDim.x) {
       int p, m, nt;
       tile_coords(a, P.m_tiles, np, tile, p, m, nt);
       const int e = a.pre_list[p];
       const Planes PL = make_planes(tp.t[tp.id[e]]);
-      const int mat = GATEUP ? part : 0;
-      const uint8_t* srow = (GATEUP ? (part ? a.up_s : a.gate_s) : a.down_s) +
+      const uint8_t* srow = (GATEUP ? (mat ? a.up_s : a.gate_s) : a.down_s) +
                             ((size_t)e * rows_total + m * kBM + r) * (size_t)(K / 32);
-      // scale bytes of blocks 2ks .. 2ks+3 (k-steps ks, ks+1): K % 128 == 0 keeps
-      // every 4-byte load inside the row and aligned
+      // scale bytes of blocks 2ks .. 2ks+3 (k-steps ks, ks+1) as one 4-byte word
+      // (K % 128 == 0 keeps every word inside the row and aligned), loaded three
+      // words ahead of use so the loads' latency hides behind the decode
+      const uint32_t* sw32 = reinterpret_cast<const uint32_t*>(srow);
+      const int n_sw = P.k_steps / 2;
+      uint32_t q0 = sw32[0], q1 = n_sw > 1 ? sw32[1] : 0u, q2 = n_sw > 2 ? sw32[2] : 0u;
       uint32_t sc = 0;
       bool ok = true;
       for (int ks = 0; ks < P.k_steps; ++ks, ++it) {
-        if ((ks & 1) == 0) sc = *reinterpret_cast<const uint32_t*>(srow + ks * 2);
+        if ((ks & 1) == 0) {
+          sc = q0;
+          q0 = q1;
+          q1 = q2;
+          q2 = (ks >> 1) + 3 < n_sw ? sw32[(ks >> 1) + 3] : 0u;
+        }
         const int s = it % C::kStages;
         const uint32_t ph = (it / C::kStages) & 1;
         if (!mbar_wait_warp(&full_c[s], ph, abort_flag, kWaitLimitNs)) {
@@ -243,7 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sw = (r >> 2) & 1;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          if (!GATEUP && half != part) continue;
+          if (half != my_half) continue;
           const uint4 cv = *reinterpret_cast<const uint4*>(ctile + r * 32 + ((half ^ sw) << 4));
           const int blk = 2 * (ks & 1) + half;  // block within the 4 loaded
           const uint32_t sbyte = (sc >> (blk * 8)) & 0xffu;
@@ -286,20 +297,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int wrow = m * kBM + row;
       const int n_hi = n_e - nt * kBN < kBN ? n_e - nt * kBN : kBN;  // tokens of this tile
 #pragma unroll 1
-      for (int c0 = 0; c0 < n_hi; c0 += 32) {
-        float g[32];
-        tmem_ld32(tb + c0, g);
+      for (int c0 = 0; c0 < n_hi; c0 += 16) {
+        float g[16];
+        tmem_ld16(tb + c0, g);
         if (GATEUP) {
-          float u[32];
-          tmem_ld32(tb + kBN + c0, u);
+          float u[16];
+          tmem_ld16(tb + kBN + c0, u);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const int n = nt * kBN + c0 + j;
             if (n < n_e) a.h[(size_t)(row0 + n) * a.I + wrow] = __float2bfloat16_rn(silu_mul(g[j], u[j]));
           }
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
+          for (int j = 0; j < 16; ++j) {
             const int n = nt * kBN + c0 + j;
             if (n < n_e) a.y[(size_t)(row0 + n) * a.H + wrow] = g[j];
           }
@@ -401,7 +412,7 @@ static int launch_tc(const FwdArgs& a, const TableParams& tp, cudaStream_t s) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = s;
   cfg.attrs = attr;
