@@ -23,6 +23,7 @@ bool uses_prefill(int T) { return T > kDecodeMaxRows; }
 // Persistent small-M kernels run at most this many CTAs (one per SM); the
 // workspace holds two split-tile partial slots per CTA.
 constexpr int kDkMaxGrid = 160;
+constexpr int kDkSlabs = 8;  // small-M row slabs per 128-row tile (one split-tile counter each)
 
 int dk_grid() {
   int dev = 0, sms = 148;
@@ -108,7 +109,7 @@ Layout layout(const moe_q4_layer* L, int T, int k) {
   o.dk_units_dn = max_exp * (L->H / 128);
   o.n_max = T < 16 ? T : 16;
   o.dk_counter = p;
-  p = align_up(p + sizeof(int32_t) * (size_t)(o.dk_units_gu + o.dk_units_dn));
+  p = align_up(p + sizeof(int32_t) * (size_t)(o.dk_units_gu + o.dk_units_dn) * kDkSlabs);
   o.dk_partial = p;
   p = align_up(p + sizeof(float) * (size_t)2 * kDkMaxGrid * 3 * o.n_max * 128);
   o.end = p;
@@ -161,7 +162,7 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   a.tiles = (int32_t*)(ws + o.tiles);
   a.xg = o.xg ? (__nv_bfloat16*)(ws + o.xg) : nullptr;
   a.dk_counter = (int32_t*)(ws + o.dk_counter);
-  a.dk_counter_n = o.dk_units_gu + o.dk_units_dn;
+  a.dk_counter_n = (o.dk_units_gu + o.dk_units_dn) * kDkSlabs;
   a.h = (__nv_bfloat16*)(ws + o.h);
   a.h_lo = (__nv_bfloat16*)(ws + o.h_lo);
   a.y = (float*)(ws + o.y);
@@ -189,7 +190,7 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   float* part_gu = (float*)(ws + o.dk_partial);
   float* part_dn = part_gu + (size_t)2 * kDkMaxGrid * 2 * o.n_max * 128;
   int32_t* cnt_gu = a.dk_counter;
-  int32_t* cnt_dn = a.dk_counter + o.dk_units_gu;
+  int32_t* cnt_dn = a.dk_counter + (size_t)o.dk_units_gu * kDkSlabs;
   // grouped activation rows feed the tensor-core path only (the small-M kernels
   // copy their rows from x themselves)
   if (rc == MOE_Q4_OK && pre) rc = q4_launch_gather(a, s);

@@ -148,7 +148,7 @@ struct DkParams {
   int n_max;        // token columns kept in partial sums: min(16, T)
   uint32_t code_stage, x_stage, scale_stage;
   float* partial;   // [2 * gridDim.x][mats][n_max][128]
-  int32_t* counter; // [units], zero at launch
+  int32_t* counter; // [units][8 slabs], zero at launch
 };
 
 __device__ __forceinline__ long long dk_range(int b, long long total, int G) { return (long long)b * total / G; }
@@ -170,6 +170,12 @@ __device__ __forceinline__ int dk_contributors(long long us, long long ue, long 
   int n = 0;
   for (int c = c_first; c <= c_last; ++c) n += dk_range(c + 1, total, G) > dk_range(c, total, G);
   return n;
+}
+
+__device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 
 __device__ __forceinline__ void ring_next(int& s, uint32_t& ph, int n) {
@@ -300,9 +306,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   uint64_t* full = bars;                          // [ring] codes (+ h: TMA), scales (+ x: cp.async)
   uint64_t* stage_empty = full + dk::kMaxRing;    // [ring] compute warps done with the stage
   uint64_t* lut_bar = stage_empty + dk::kMaxRing; // compute threads rebuilding a table slot
-  uint64_t* epi_bar = lut_bar + 1;                // compute threads finishing a split tile
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(epi_bar + 1);
-  volatile int* last_flag = abort_flag + 1;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(lut_bar + 1);
 
   const int ring = P.ring;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -312,7 +316,6 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       mbar_init(&stage_empty[s], dk::kComputeWarps);
     }
     mbar_init(lut_bar, 32 * dk::kComputeWarps);
-    mbar_init(epi_bar, 32 * dk::kComputeWarps);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_wa);
@@ -452,7 +455,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         xoff[J][c] = (uint32_t)((2 * J + (tq >> 1)) * C::kAtoms * 1024 + gq * 128 + ((((tq & 1) * 4 + c) ^ gq) << 4));
     }
     int slot_tab0 = tp.n == 1 ? 0 : -1, slot_tab1 = -1, victim = tp.n == 1 ? 1 : 0;
-    uint32_t lgen = 0, egen = 0;
+    uint32_t lgen = 0;
     const uint32_t lane_k = (Ls.lut & 0xffff0000u) | ((uint32_t)lane << 2);
     int s = 0;
     uint32_t ph = 0;
@@ -612,24 +615,22 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
               const int n = 8 * tt + 2 * tq + (i & 1);
               if (n < P.n_max) pp[(m * P.n_max + n) * dk::kRows + ((i >> 1) ? r1 : r0)] = acc[m][tt][i];
             }
-        __threadfence();
-        mbar_arrive(epi_bar);
-        if (!mbar_wait_warp(epi_bar, egen & 1, abort_flag, dk::kWaitNs)) break;
-        ++egen;
-        if (slab == 0 && lane == 0) {
+        // each slab warp signs in on its own counter (release: its lanes' partial
+        // stores, ordered before lane 0's atomic by the warp barrier); the last
+        // warp of a slab to sign in (acquire) finishes those rows
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
           int c_first, c_last;
           const int n_contrib = dk_contributors(ustart, uend, total, G, c_first, c_last);
-          const int old = atomicAdd(&P.counter[unit], 1);
-          *last_flag = (old == n_contrib - 1) ? 1 : 0;
+          last = atom_add_acq_rel(&P.counter[(size_t)unit * 8 + slab], 1) == n_contrib - 1;
         }
-        mbar_arrive(epi_bar);
-        if (!mbar_wait_warp(epi_bar, egen & 1, abort_flag, dk::kWaitNs)) break;
-        ++egen;
-        if (!*last_flag) {
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (!last) {
           g = seg_end;
           continue;
         }
-        __threadfence();
+        __syncwarp();
         // last arrival: add the partials of every CTA on this tile in K order
         int c_first, c_last;
         dk_contributors(ustart, uend, total, G, c_first, c_last);
