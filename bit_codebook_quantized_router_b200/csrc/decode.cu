@@ -76,6 +76,10 @@ struct DkCfg {
   static constexpr int kMats = GATEUP ? 2 : 1;
   // 1-KB activation atoms (8 rows x 128 B, 128-byte swizzle) per 64-K super-step
   static constexpr int kAtoms = GATEUP ? NT : (NT == 4 ? 4 : 2);
+  // gate/up activation rows: unswizzled 128-byte rows at a 144-byte pitch (the
+  // odd 16-byte multiple spreads rows over the banks); bytes per super-step
+  static constexpr int kXRowPitch = 144;
+  static constexpr int kXSuper = GATEUP ? 8 * NT * kXRowPitch : kAtoms * 1024;
   // 8-token groups of the result
   static constexpr int kTT = GATEUP ? NT : (NT == 4 ? 2 : 1);
   // independent accumulators per (matrix, token group): MMA mm of K half J adds
@@ -353,17 +357,18 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       const int t = unit % P.tiles_per_e;
       const int wrow = e * rows_total + t * dk::kRows;
       const int row0 = a.offsets[e];
-      // gate/up: the tokens of the activation rows this lane copies (rows
-      // (lane >> 3) + 4q of the expert, absent ones zero-filled)
-      int tok[2 * NT];
-      int n_e = 0;
+      // gate/up: activation rows by untiled bulk copies (128 B of x[token] per
+      // 64 K; a tiled TMA would need a 128-byte-aligned destination),
+      // n_e rows x subs super-steps per stage spread over the lanes: lane l
+      // copies items l and l + 32 (row item % n_e, super-step item / n_e).
+      // Rows past n_e are not written: the compute lanes never read them.
+      int n_e = 0, tok_a = 0, tok_b = 0;
       if (GATEUP) {
         n_e = a.counts[e];
-#pragma unroll
-        for (int q = 0; q < 2 * NT; ++q) {
-          const int n = (lane >> 3) + 4 * q;
-          tok[q] = n < n_e ? a.row_token[row0 + n] : 0;
-        }
+        const int my_tok = lane < n_e ? a.row_token[row0 + lane] : 0;  // n_e <= 16
+        const int ne = n_e > 0 ? n_e : 1;
+        tok_a = __shfl_sync(0xffffffffu, my_tok, lane % ne);
+        tok_b = __shfl_sync(0xffffffffu, my_tok, (lane + 32) % ne);
       }
       for (int st = st0; st < st0 + (int)(seg_end - g); ++st) {
         if (!mbar_wait_warp(&stage_empty[s], ph ^ 1, abort_flag, dk::kWaitNs)) {
@@ -371,11 +376,13 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           break;
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes + (GATEUP ? 0 : subs * C::kAtoms * 1024));
+          mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes +
+                                              (GATEUP ? n_e * subs * 128 : subs * C::kAtoms * 1024));
           uint8_t* cdst = smem_raw + (code_base(s) - raw_s);
           tma_load_2d(cdst, &tm_wa, &full[s], st * row_bytes, wrow);
           if (GATEUP) tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
         }
+        __syncwarp();  // the expected bytes are registered before any row copy can land
         // scale bytes of the stage (2 per 64-K super-step) for 4 rows per lane
 #pragma unroll
         for (int m = 0; m < kMats; ++m) {
@@ -394,19 +401,15 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         }
         const uint32_t xdst = Ls.x + (uint32_t)s * P.x_stage;
         if (GATEUP) {
-          // activation rows: 8 NT rows x 8 chunks of 16 B per 64-K super-step, in
-          // the 128-byte swizzle the compute warps read (chunk c of row n at c ^ n)
-          for (int j = 0; j < subs; ++j) {
-            const int kx = (st * subs + j) * 64;
+          // row n of super-step j lands at j * kXSuper + n * kXRowPitch (16-byte
+          // aligned: x-ring and stage sizes are multiples of 16, the pitch is 144)
 #pragma unroll
-            for (int q = 0; q < 2 * NT; ++q) {
-              const int idx = lane + 32 * q;
-              const int n = idx >> 3, c = idx & 7;
-              const uint32_t dst = xdst + (uint32_t)(j * C::kAtoms * 1024 + (n >> 3) * 1024 + (n & 7) * 128 +
-                                                     ((c ^ (n & 7)) << 4));
-              const bool have = n < n_e;
-              const __nv_bfloat16* src = have ? a.x + (size_t)tok[q] * a.H + kx + 8 * c : a.x;
-              cp_async_16_zfill(dst, src, have ? 16u : 0u);
+          for (int h = 0; h < 2; ++h) {
+            const int item = lane + 32 * h;
+            if (item < n_e * subs) {
+              const int n = item % n_e, j = item / n_e;
+              uint8_t* d = smem_raw + (xdst - raw_s) + j * C::kXSuper + n * C::kXRowPitch;
+              bulk_load(d, a.x + (size_t)(h ? tok_b : tok_a) * a.H + (st * subs + j) * 64, 128u, &full[s]);
             }
           }
         }
@@ -416,7 +419,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           // lie outside the array: they only feed columns nobody writes
           for (int j = 0; j < subs; ++j) {
             const int kx = (st * subs + j) * 64;
-            uint8_t* d = smem_raw + (xdst - raw_s) + j * C::kAtoms * 1024;
+            uint8_t* d = smem_raw + (xdst - raw_s) + j * C::kXSuper;
             if (NT == 1) {
               tma_load_2d(d, &tm_x, &full[s], kx, row0);             // h rows 0..3 at atom rows 0..3
               tma_load_2d(d + 1024, &tm_xl, &full[s], kx, row0 - 4);  // h_lo rows 0..3 at atom rows 4..7
@@ -452,7 +455,8 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       coff[J][1] = (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4));
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        xoff[J][c] = (uint32_t)((2 * J + (tq >> 1)) * C::kAtoms * 1024 + gq * 128 + ((((tq & 1) * 4 + c) ^ gq) << 4));
+        xoff[J][c] = GATEUP ? (uint32_t)((2 * J + (tq >> 1)) * C::kXSuper + gq * C::kXRowPitch + ((tq & 1) * 4 + c) * 16)
+                            : (uint32_t)((2 * J + (tq >> 1)) * C::kXSuper + gq * 128 + ((((tq & 1) * 4 + c) ^ gq) << 4));
     }
     int slot_tab0 = tp.n == 1 ? 0 : -1, slot_tab1 = -1, victim = tp.n == 1 ? 1 : 0;
     uint32_t lgen = 0;
@@ -542,7 +546,8 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
               atom = nt;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              lds128_if(xstage + (uint32_t)atom * 1024 + xoff[J][c], col_ok[nt], xr[nt][4 * c + 0],
+              lds128_if(xstage + (uint32_t)atom * (GATEUP ? 8 * C::kXRowPitch : 1024) + xoff[J][c], col_ok[nt],
+                        xr[nt][4 * c + 0],
                         xr[nt][4 * c + 1], xr[nt][4 * c + 2], xr[nt][4 * c + 3]);
               dep ^= xr[nt][4 * c + 0];
             }
@@ -737,7 +742,7 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
   P.stages = K / (64 * P.subs);
   P.n_max = a.T < 16 ? a.T : 16;
   P.code_stage = (uint32_t)(C::kMats * dk::kRows * 32 * P.subs);
-  P.x_stage = (uint32_t)(P.subs * C::kAtoms * 1024);
+  P.x_stage = (uint32_t)(P.subs * C::kXSuper);
   P.scale_stage = (uint32_t)(C::kMats * dk::kRows * dk::kScaleSlot);
   P.partial = partial;
   P.counter = counter;
@@ -765,7 +770,7 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
   if (GATEUP) {
     ok = dk_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.gate_w, a.H / 2, (uint64_t)a.E * a.I, cbox, dk::kRows, csw) &&
          dk_map(&twb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.up_w, a.H / 2, (uint64_t)a.E * a.I, cbox, dk::kRows, csw);
-    tx = txl = twa;  // unused: activation rows come by cp.async
+    tx = txl = twa;  // unused: activation rows come by untiled bulk copies
   } else {
     ok = dk_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.down_w, a.I / 2, (uint64_t)a.E * a.H, cbox, dk::kRows,
                 csw) &&
