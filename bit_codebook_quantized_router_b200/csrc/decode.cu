@@ -76,10 +76,8 @@ struct DkCfg {
   static constexpr int kMats = GATEUP ? 2 : 1;
   // 1-KB activation atoms (8 rows x 128 B, 128-byte swizzle) per 64-K super-step
   static constexpr int kAtoms = GATEUP ? NT : (NT == 4 ? 4 : 2);
-  // gate/up activation rows: unswizzled 128-byte rows at a 144-byte pitch (the
-  // odd 16-byte multiple spreads rows over the banks); bytes per super-step
-  static constexpr int kXRowPitch = 144;
-  static constexpr int kXSuper = GATEUP ? 8 * NT * kXRowPitch : kAtoms * 1024;
+  // down: bytes of activation atoms per 64-K super-step
+  static constexpr int kXSuper = kAtoms * 1024;
   // 8-token groups of the result
   static constexpr int kTT = GATEUP ? NT : (NT == 4 ? 2 : 1);
   // independent accumulators per (matrix, token group): MMA mm of K half J adds
@@ -151,6 +149,7 @@ struct DkParams {
   DkLayout lay;     // shared-memory placement (offsets)
   int n_max;        // token columns kept in partial sums: min(16, T)
   uint32_t code_stage, x_stage, scale_stage;
+  uint32_t x_pitch;  // gate/up: bytes per activation row in a stage (subs * 128 + 16)
   float* partial;   // [2 * gridDim.x][mats][n_max][128]
   int32_t* counter; // [units][8 slabs], zero at launch
 };
@@ -334,6 +333,9 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   if (tp.n == 1 && warp >= 1) build_lut_slot(lut, tp.t[0], 0, threadIdx.x - 32);
   __syncthreads();
 
+  // down: the next kernel (the combine, small CTAs that fit beside this one)
+  // may be scheduled now; its own wait still covers all of this kernel's work
+  if (!GATEUP) pdl_trigger();
   pdl_wait();
   const int n_dec = a.hdr[kNumDecode];
   const int rows_total = GATEUP ? a.I : a.H;
@@ -357,18 +359,14 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       const int t = unit % P.tiles_per_e;
       const int wrow = e * rows_total + t * dk::kRows;
       const int row0 = a.offsets[e];
-      // gate/up: activation rows by untiled bulk copies (128 B of x[token] per
-      // 64 K; a tiled TMA would need a 128-byte-aligned destination),
-      // n_e rows x subs super-steps per stage spread over the lanes: lane l
-      // copies items l and l + 32 (row item % n_e, super-step item / n_e).
+      // gate/up: activation rows by untiled bulk copies, one per row and stage
+      // (the stage's 32 * subs * 4 bytes of x[token], contiguous in x), lane n
+      // copying row n; a tiled TMA would need a 128-byte-aligned destination.
       // Rows past n_e are not written: the compute lanes never read them.
-      int n_e = 0, tok_a = 0, tok_b = 0;
+      int n_e = 0, my_tok = 0;
       if (GATEUP) {
         n_e = a.counts[e];
-        const int my_tok = lane < n_e ? a.row_token[row0 + lane] : 0;  // n_e <= 16
-        const int ne = n_e > 0 ? n_e : 1;
-        tok_a = __shfl_sync(0xffffffffu, my_tok, lane % ne);
-        tok_b = __shfl_sync(0xffffffffu, my_tok, (lane + 32) % ne);
+        my_tok = lane < n_e ? a.row_token[row0 + lane] : 0;  // n_e <= 16
       }
       for (int st = st0; st < st0 + (int)(seg_end - g); ++st) {
         if (!mbar_wait_warp(&stage_empty[s], ph ^ 1, abort_flag, dk::kWaitNs)) {
@@ -377,7 +375,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes +
-                                              (GATEUP ? n_e * subs * 128 : subs * C::kAtoms * 1024));
+                                              (GATEUP ? n_e * subs * 128 : subs * C::kXSuper));
           uint8_t* cdst = smem_raw + (code_base(s) - raw_s);
           tma_load_2d(cdst, &tm_wa, &full[s], st * row_bytes, wrow);
           if (GATEUP) tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
@@ -400,18 +398,11 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           }
         }
         const uint32_t xdst = Ls.x + (uint32_t)s * P.x_stage;
-        if (GATEUP) {
-          // row n of super-step j lands at j * kXSuper + n * kXRowPitch (16-byte
-          // aligned: x-ring and stage sizes are multiples of 16, the pitch is 144)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int item = lane + 32 * h;
-            if (item < n_e * subs) {
-              const int n = item % n_e, j = item / n_e;
-              uint8_t* d = smem_raw + (xdst - raw_s) + j * C::kXSuper + n * C::kXRowPitch;
-              bulk_load(d, a.x + (size_t)(h ? tok_b : tok_a) * a.H + (st * subs + j) * 64, 128u, &full[s]);
-            }
-          }
+        if (GATEUP && lane < n_e) {
+          // row n lands at n * x_pitch (x_pitch = stage bytes + 16: 16-byte
+          // aligned, and an odd number of 16-byte chunks spreads rows over banks)
+          uint8_t* d = smem_raw + (xdst - raw_s) + lane * P.x_pitch;
+          bulk_load(d, a.x + (size_t)my_tok * a.H + st * subs * 64, (uint32_t)(subs * 128), &full[s]);
         }
         cp_async_arrive_noinc(&full[s]);
         if (!GATEUP && lane == 0) {
@@ -419,7 +410,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           // lie outside the array: they only feed columns nobody writes
           for (int j = 0; j < subs; ++j) {
             const int kx = (st * subs + j) * 64;
-            uint8_t* d = smem_raw + (xdst - raw_s) + j * C::kXSuper;
+            uint8_t* d = smem_raw + (xdst - raw_s) + j * C::kXSuper;  // down only
             if (NT == 1) {
               tma_load_2d(d, &tm_x, &full[s], kx, row0);             // h rows 0..3 at atom rows 0..3
               tma_load_2d(d + 1024, &tm_xl, &full[s], kx, row0 - 4);  // h_lo rows 0..3 at atom rows 4..7
@@ -455,7 +446,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       coff[J][1] = (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4));
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        xoff[J][c] = GATEUP ? (uint32_t)((2 * J + (tq >> 1)) * C::kXSuper + gq * C::kXRowPitch + ((tq & 1) * 4 + c) * 16)
+        xoff[J][c] = GATEUP ? (uint32_t)(gq * P.x_pitch + (2 * J + (tq >> 1)) * 128 + ((tq & 1) * 4 + c) * 16)
                             : (uint32_t)((2 * J + (tq >> 1)) * C::kXSuper + gq * 128 + ((((tq & 1) * 4 + c) ^ gq) << 4));
     }
     int slot_tab0 = tp.n == 1 ? 0 : -1, slot_tab1 = -1, victim = tp.n == 1 ? 1 : 0;
@@ -546,7 +537,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
               atom = nt;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              lds128_if(xstage + (uint32_t)atom * (GATEUP ? 8 * C::kXRowPitch : 1024) + xoff[J][c], col_ok[nt],
+              lds128_if(xstage + (uint32_t)atom * (GATEUP ? 8 * P.x_pitch : 1024) + xoff[J][c], col_ok[nt],
                         xr[nt][4 * c + 0],
                         xr[nt][4 * c + 1], xr[nt][4 * c + 2], xr[nt][4 * c + 3]);
               dep ^= xr[nt][4 * c + 0];
@@ -696,7 +687,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         }
   }
   __syncthreads();
-  pdl_trigger();
+  if (GATEUP) pdl_trigger();
 }
 
 // ---------------------------------------------------------------------------
@@ -742,7 +733,8 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
   P.stages = K / (64 * P.subs);
   P.n_max = a.T < 16 ? a.T : 16;
   P.code_stage = (uint32_t)(C::kMats * dk::kRows * 32 * P.subs);
-  P.x_stage = (uint32_t)(P.subs * C::kXSuper);
+  P.x_pitch = (uint32_t)(P.subs * 128 + 16);
+  P.x_stage = GATEUP ? (uint32_t)(8 * NT) * P.x_pitch : (uint32_t)(P.subs * C::kXSuper);
   P.scale_stage = (uint32_t)(C::kMats * dk::kRows * dk::kScaleSlot);
   P.partial = partial;
   P.counter = counter;

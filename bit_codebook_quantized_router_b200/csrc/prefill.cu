@@ -343,6 +343,9 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
+  // triggered at the end: the next kernel's CTAs (shared memory near the SM's
+  // limit) could not share an SM with this one anyway, and launching them while
+  // this persistent grid still runs measured slower
   pdl_trigger();
 }
 

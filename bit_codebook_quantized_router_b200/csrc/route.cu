@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_fused_kernel(const __grid
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int e = tid; e < E; e += kRouteThreads) counts[e] = 0;
   for (int i = tid; i < E * W; i += kRouteThreads) tokmask[i] = 0u;
+  pdl_trigger();  // scheduling only: the next kernel's wait covers this one
   pdl_wait();
   if (tid == 0) a.hdr[kStatus] = MOE_Q4_OK;
   // per-tile arrival counters of the small-M kernels start at zero every call
@@ -311,12 +312,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_fused_kernel(const __grid
     a.row_token[pos] = t;
     a.inv[r] = pos;
   }
-  pdl_trigger();
 }
 
 // Large T: top-k on many CTAs (one warp per token; the host clears the
 // status word before this launch) ...
 __global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__ FwdArgs a) {
+  pdl_trigger();  // scheduling only: the next kernel's wait covers this one
   pdl_wait();
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -326,21 +327,21 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__
     topk_warp(a.logits + (size_t)t * a.E, a.E, a.k, lane, a.hdr + kStatus, id, w);
     store_route(a, t, lane, id, w);
   }
-  pdl_trigger();
 }
 
 // ... then one CTA groups.
 __global__ void __launch_bounds__(kRouteThreads) route_group_kernel(const __grid_constant__ FwdArgs a) {
   extern __shared__ int sm[];
+  pdl_trigger();  // scheduling only: the next kernel's wait covers this one
   pdl_wait();
   group_rows(a, sm);
-  pdl_trigger();
 }
 
 // Gather the activation rows in expert-grouped order for the tensor-core
 // GEMMs (both paths read activations by TMA from contiguous rows):
 // xg[row] = x[row_token[row]] for all T*k rows.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant__ FwdArgs a) {
+  pdl_trigger();  // scheduling only: the next kernel's wait covers this one
   pdl_wait();
   const int vec_per_row = a.H / 8;  // 16-byte vectors
   const int64_t n = (int64_t)a.T * a.k * vec_per_row;
@@ -350,7 +351,6 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant_
     const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)a.row_token[r] * a.H) + q;
     reinterpret_cast<uint4*>(a.xg + (size_t)r * a.H)[q] = *src;
   }
-  pdl_trigger();
 }
 
 }  // namespace q4
