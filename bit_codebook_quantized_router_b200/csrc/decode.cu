@@ -278,7 +278,9 @@ __device__ __forceinline__ void decode_chunk(const uint4 c, const Planes& PL, ui
   for (int i = 0; i < 16; ++i) p[i] = bf16x2_mul(p[i], scale2);
 }
 
-template <bool GATEUP, int NT>
+// SUBS (64-K super-steps per stage, 4 or 2) is a template argument so that a
+// stage's two 128-K halves form one unrolled block the compiler can interleave.
+template <bool GATEUP, int NT, int SUBS>
 __global__ void __launch_bounds__(dk::kThreads, 1)
     dk_kernel(const __grid_constant__ DkParams P, const __grid_constant__ TableParams tp,
               const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
@@ -340,8 +342,8 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   const int n_dec = a.hdr[kNumDecode];
   const int rows_total = GATEUP ? a.I : a.H;
   const int K = GATEUP ? a.H : a.I;
-  const int subs = P.subs;
-  const int row_bytes = 32 * subs;  // code bytes per row per stage
+  constexpr int subs = SUBS;
+  constexpr int row_bytes = 32 * subs;  // code bytes per row per stage
   const long long total = (long long)n_dec * P.tiles_per_e * P.stages;
   const int G = gridDim.x, b = blockIdx.x;
   const long long k0 = dk_range(b, total, G), k1 = dk_range(b + 1, total, G);
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
             const int r = lane + 32 * j;
             const uint32_t dst =
                 Ls.scales + (uint32_t)s * P.scale_stage + (uint32_t)(m * dk::kRows + r) * dk::kScaleSlot;
-            if (subs == 4)
+            if constexpr (subs == 4)
               cp_async_small<8>(dst, sbase + (size_t)r * (K / 32));
             else
               cp_async_small<4>(dst, sbase + (size_t)r * (K / 32));
@@ -431,7 +433,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     const int gq = lane >> 2;      // MMA group: rows gq, gq + 8; token column gq
     const int tq = lane & 3;       // code chunk of a half; token columns 2tq, 2tq + 1
     const int ctid = threadIdx.x - 32;
-    const int n_halves = subs / 2; // 128-K halves per stage
+    constexpr int n_halves = subs / 2; // 128-K halves per stage
     const int r0 = 16 * slab + gq, r1 = r0 + 8;
     const int swz0 = subs == 4 ? (r0 & 7) : ((r0 >> 1) & 3);
     const int swz1 = subs == 4 ? (r1 & 7) : ((r1 >> 1) & 3);
@@ -721,15 +723,15 @@ static bool dk_map(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, con
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GATEUP, int NT>
-static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, int32_t* counter, int grid,
+template <bool GATEUP, int NT, int SUBS>
+static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partial, int32_t* counter, int grid,
                      cudaStream_t s) {
   using C = DkCfg<GATEUP, NT>;
   DkParams P;
   P.a = a;
   const int K = GATEUP ? a.H : a.I;
   P.tiles_per_e = (GATEUP ? a.I : a.H) / dk::kRows;
-  P.subs = (K % 256 == 0) ? 4 : 2;  // K % 128 == 0 always
+  P.subs = SUBS;
   P.stages = K / (64 * P.subs);
   P.n_max = a.T < 16 ? a.T : 16;
   P.code_stage = (uint32_t)(C::kMats * dk::kRows * 32 * P.subs);
@@ -771,7 +773,7 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
     twb = twa;
   }
   if (!ok) return MOE_Q4_ECUDA;
-  if (cudaFuncSetAttribute(dk_kernel<GATEUP, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+  if (cudaFuncSetAttribute(dk_kernel<GATEUP, NT, SUBS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return MOE_Q4_ECUDA;
   cudaLaunchAttribute attr[1];
@@ -784,8 +786,17 @@ static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, in
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, dk_kernel<GATEUP, NT>, P, tp, twa, twb, tx, txl) == cudaSuccess ? MOE_Q4_OK
+  return cudaLaunchKernelEx(&cfg, dk_kernel<GATEUP, NT, SUBS>, P, tp, twa, twb, tx, txl) == cudaSuccess ? MOE_Q4_OK
                                                                                                  : MOE_Q4_ECUDA;
+}
+
+// stages of 256 K when K allows, else 128 (K % 128 == 0 always)
+template <bool GATEUP, int NT>
+static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, int32_t* counter, int grid,
+                     cudaStream_t s) {
+  const int K = GATEUP ? a.H : a.I;
+  return K % 256 == 0 ? launch_dk_subs<GATEUP, NT, 4>(a, tp, partial, counter, grid, s)
+                      : launch_dk_subs<GATEUP, NT, 2>(a, tp, partial, counter, grid, s);
 }
 
 }  // namespace q4
