@@ -154,11 +154,12 @@ struct DkParams {
   int32_t* counter; // [units][8 slabs], zero at launch
 };
 
-__device__ __forceinline__ long long dk_range(int b, long long total, int G) { return (long long)b * total / G; }
+// Start of CTA b's range of stages (the host keeps total below 2^31).
+__device__ __forceinline__ int dk_range(int b, int total, int G) { return (int)((long long)b * total / G); }
 
 // CTA whose range holds stage g.
-__device__ __forceinline__ int dk_owner(long long g, long long total, int G) {
-  int b = (int)((g * G) / total);
+__device__ __forceinline__ int dk_owner(int g, int total, int G) {
+  int b = (int)(((long long)g * G) / total);
   while (b + 1 < G && dk_range(b + 1, total, G) <= g) ++b;
   while (b > 0 && dk_range(b, total, G) > g) --b;
   return b;
@@ -166,13 +167,26 @@ __device__ __forceinline__ int dk_owner(long long g, long long total, int G) {
 
 // CTAs holding part of [us, ue): the owners of its ends and every non-empty
 // range between them (with fewer stages than CTAs some ranges are empty).
-__device__ __forceinline__ int dk_contributors(long long us, long long ue, long long total, int G, int& c_first,
-                                               int& c_last) {
+__device__ __forceinline__ int dk_contributors(int us, int ue, int total, int G, int& c_first, int& c_last) {
   c_first = dk_owner(us, total, G);
   c_last = dk_owner(ue - 1, total, G);
   int n = 0;
   for (int c = c_first; c <= c_last; ++c) n += dk_range(c + 1, total, G) > dk_range(c, total, G);
   return n;
+}
+
+// A unit shared by several CTAs: its contributors, and the partial-sum slot
+// of the first (2c + 1 when the unit is not where that CTA's range starts).
+struct DkSplit {
+  int c_first, c_last, n_contrib, first_slot;
+};
+
+__device__ __forceinline__ DkSplit dk_split(int unit, int stages, int total, int G) {
+  DkSplit d;
+  const int us = unit * stages;
+  d.n_contrib = dk_contributors(us, us + stages, total, G, d.c_first, d.c_last);
+  d.first_slot = dk_range(d.c_first, total, G) != us ? 2 * d.c_first + 1 : 2 * d.c_first;
+  return d;
 }
 
 __device__ __forceinline__ int atom_add_acq_rel(int32_t* p, int v) {
@@ -344,19 +358,19 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   const int K = GATEUP ? a.H : a.I;
   constexpr int subs = SUBS;
   constexpr int row_bytes = 32 * subs;  // code bytes per row per stage
-  const long long total = (long long)n_dec * P.tiles_per_e * P.stages;
+  const int total = n_dec * P.tiles_per_e * P.stages;
   const int G = gridDim.x, b = blockIdx.x;
-  const long long k0 = dk_range(b, total, G), k1 = dk_range(b + 1, total, G);
+  const int k0 = dk_range(b, total, G), k1 = dk_range(b + 1, total, G);
 
   if (warp == 0) {
     // ------------------------------ producer ------------------------------
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (long long g = k0; g < k1 && ok;) {
-      const int unit = (int)(g / P.stages);
-      const int st0 = (int)(g - (long long)unit * P.stages);
-      const long long seg_end = min(k1, (long long)(unit + 1) * P.stages);
+    for (int g = k0; g < k1 && ok;) {
+      const int unit = g / P.stages;
+      const int st0 = g - unit * P.stages;
+      const int seg_end = min(k1, (unit + 1) * P.stages);
       const int e = a.dec_list[unit / P.tiles_per_e];
       const int t = unit % P.tiles_per_e;
       const int wrow = e * rows_total + t * dk::kRows;
@@ -454,13 +468,20 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     int slot_tab0 = tp.n == 1 ? 0 : -1, slot_tab1 = -1, victim = tp.n == 1 ? 1 : 0;
     uint32_t lgen = 0;
     const uint32_t lane_k = (Ls.lut & 0xffff0000u) | ((uint32_t)lane << 2);
+    // only the first and the last unit of the range can be shared with other
+    // CTAs: their contributors are found now, while the first stage is in flight
+    DkSplit sp_first = {0, 0, 1, 0}, sp_last = {0, 0, 1, 0};
+    if (k0 < k1) {
+      sp_first = dk_split(k0 / P.stages, P.stages, total, G);
+      sp_last = (k1 - 1) / P.stages == k0 / P.stages ? sp_first : dk_split((k1 - 1) / P.stages, P.stages, total, G);
+    }
     int s = 0;
     uint32_t ph = 0;
     bool ok = true;
-    for (long long g = k0; g < k1 && ok;) {
-      const int unit = (int)(g / P.stages);
-      const long long ustart = (long long)unit * P.stages, uend = ustart + P.stages;
-      const long long seg_end = min(k1, uend);
+    for (int g = k0; g < k1 && ok;) {
+      const int unit = g / P.stages;
+      const int ustart = unit * P.stages, uend = ustart + P.stages;
+      const int seg_end = min(k1, uend);
       const int nst = (int)(seg_end - g);
       const int e = a.dec_list[unit / P.tiles_per_e];
       const int tile = unit % P.tiles_per_e;
@@ -617,12 +638,10 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         // stores, ordered before lane 0's atomic by the warp barrier); the last
         // warp of a slab to sign in (acquire) finishes those rows
         __syncwarp();
+        // a shared segment is the first or the last of this CTA's range
+        const DkSplit sp = g == k0 ? sp_first : sp_last;
         int last = 0;
-        if (lane == 0) {
-          int c_first, c_last;
-          const int n_contrib = dk_contributors(ustart, uend, total, G, c_first, c_last);
-          last = atom_add_acq_rel(&P.counter[(size_t)unit * 8 + slab], 1) == n_contrib - 1;
-        }
+        if (lane == 0) last = atom_add_acq_rel(&P.counter[(size_t)unit * 8 + slab], 1) == sp.n_contrib - 1;
         last = __shfl_sync(0xffffffffu, last, 0);
         if (!last) {
           g = seg_end;
@@ -630,17 +649,16 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         }
         __syncwarp();
         // last arrival: add the partials of every CTA on this tile in K order
-        int c_first, c_last;
-        dk_contributors(ustart, uend, total, G, c_first, c_last);
 #pragma unroll
         for (int m = 0; m < kMats; ++m)
 #pragma unroll
           for (int tt = 0; tt < C::kTT; ++tt)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[m][tt][i] = 0.0f;
-        for (int c = c_first; c <= c_last; ++c) {
-          if (dk_range(c + 1, total, G) == dk_range(c, total, G)) continue;  // empty range
-          const int sl = (c == c_first && dk_range(c, total, G) != ustart) ? 2 * c + 1 : 2 * c;
+        for (int c = sp.c_first; c <= sp.c_last; ++c) {
+          // with fewer stages than CTAs some ranges are empty
+          if (total < G && dk_range(c + 1, total, G) == dk_range(c, total, G)) continue;
+          const int sl = c == sp.c_first ? sp.first_slot : 2 * c;
           const float* qp = P.partial + (size_t)sl * kMats * P.n_max * dk::kRows;
 #pragma unroll
           for (int m = 0; m < kMats; ++m)
@@ -733,6 +751,8 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   P.tiles_per_e = (GATEUP ? a.I : a.H) / dk::kRows;
   P.subs = SUBS;
   P.stages = K / (64 * P.subs);
+  // stage indices are 32-bit on the device
+  if ((uint64_t)a.E * (uint64_t)P.tiles_per_e * (uint64_t)P.stages >= (1ull << 31)) return MOE_Q4_EINVAL;
   P.n_max = a.T < 16 ? a.T : 16;
   P.code_stage = (uint32_t)(C::kMats * dk::kRows * 32 * P.subs);
   P.x_pitch = (uint32_t)(P.subs * 128 + 16);
