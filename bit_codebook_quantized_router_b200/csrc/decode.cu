@@ -74,10 +74,12 @@ constexpr uint32_t kBarBytes = 1024;   // barriers and flags
 template <bool GATEUP, int NT>
 struct DkCfg {
   static constexpr int kMats = GATEUP ? 2 : 1;
-  // 1-KB activation atoms (8 rows x 128 B, 128-byte swizzle) per 64-K super-step
-  static constexpr int kAtoms = GATEUP ? NT : (NT == 4 ? 4 : 2);
-  // down: bytes of activation atoms per 64-K super-step
-  static constexpr int kXSuper = kAtoms * 1024;
+  // activation row slots of a stage: 8 per n-tile; slot 8 nt + c feeds column
+  // c of n-tile nt.  Gate/up: x of the expert's row n at slot n.  Down: h of
+  // row n at slot n and h_lo of row n at slot kLoSlot + n (NT = 1: h in
+  // columns 0..3, h_lo in 4..7 of one tile; else separate tiles)
+  static constexpr int kXSlots = 8 * NT;
+  static constexpr int kLoSlot = 4 * NT;
   // 8-token groups of the result
   static constexpr int kTT = GATEUP ? NT : (NT == 4 ? 2 : 1);
   // independent accumulators per (matrix, token group): MMA mm of K half J adds
@@ -220,7 +222,8 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
 }
 
 // 16-byte shared load by the lanes with `pred` set; the others get zeros and
-// touch no shared memory.
+// touch no shared memory (a 16-byte load is served a quarter-warp at a time,
+// so a quarter-warp with no active lane costs nothing).
 __device__ __forceinline__ void lds128_if(uint32_t addr, uint32_t pred, uint32_t& x, uint32_t& y, uint32_t& z,
                                           uint32_t& w) {
   asm("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %5, 0;\n\t"
@@ -297,8 +300,7 @@ __device__ __forceinline__ void decode_chunk(const uint4 c, const Planes& PL, ui
 template <bool GATEUP, int NT, int SUBS>
 __global__ void __launch_bounds__(dk::kThreads, 1)
     dk_kernel(const __grid_constant__ DkParams P, const __grid_constant__ TableParams tp,
-              const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb,
-              const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xl) {
+              const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb) {
   using C = DkCfg<GATEUP, NT>;
   constexpr int kMats = C::kMats;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -339,10 +341,6 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     fence_mbar_init();
     prefetch_tmap(&tm_wa);
     if (GATEUP) prefetch_tmap(&tm_wb);
-    if (!GATEUP) {
-      prefetch_tmap(&tm_x);
-      prefetch_tmap(&tm_xl);
-    }
   }
   // with a single table every expert uses table 0: its table slot is built
   // before waiting for the previous kernel
@@ -375,14 +373,25 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       const int t = unit % P.tiles_per_e;
       const int wrow = e * rows_total + t * dk::kRows;
       const int row0 = a.offsets[e];
-      // gate/up: activation rows by untiled bulk copies, one per row and stage
-      // (the stage's 32 * subs * 4 bytes of x[token], contiguous in x), lane n
-      // copying row n; a tiled TMA would need a 128-byte-aligned destination.
-      // Rows past n_e are not written: the compute lanes never read them.
-      int n_e = 0, my_tok = 0;
+      // Activation rows by untiled bulk copies (a tiled TMA would need a
+      // 128-byte-aligned destination), one per row and stage: the stage's
+      // 32 * subs * 4 bytes of x[token] (gate/up, lane n: row n) or of h / h_lo
+      // (down, lane n: h of row n; lane 16 + n: h_lo of row n).  Slots past
+      // n_e are not written: they only feed columns nobody writes.
+      const int n_e = a.counts[e];  // <= 16
+      int my_slot = -1;
+      const __nv_bfloat16* my_src = nullptr;
       if (GATEUP) {
-        n_e = a.counts[e];
-        my_tok = lane < n_e ? a.row_token[row0 + lane] : 0;  // n_e <= 16
+        if (lane < n_e) {
+          my_slot = lane;
+          my_src = a.x + (size_t)a.row_token[row0 + lane] * a.H;
+        }
+      } else {
+        const int n = lane & 15;
+        if (n < n_e) {
+          my_slot = lane < 16 ? n : C::kLoSlot + n;
+          my_src = (lane < 16 ? a.h : a.h_lo) + (size_t)(row0 + n) * a.I;
+        }
       }
       for (int st = st0; st < st0 + (int)(seg_end - g); ++st) {
         if (!mbar_wait_warp(&stage_empty[s], ph ^ 1, abort_flag, dk::kWaitNs)) {
@@ -390,8 +399,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           break;
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes +
-                                              (GATEUP ? n_e * subs * 128 : subs * C::kXSuper));
+          mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes + (GATEUP ? 1 : 2) * n_e * subs * 128);
           uint8_t* cdst = smem_raw + (code_base(s) - raw_s);
           tma_load_2d(cdst, &tm_wa, &full[s], st * row_bytes, wrow);
           if (GATEUP) tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
@@ -413,29 +421,13 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
               cp_async_small<4>(dst, sbase + (size_t)r * (K / 32));
           }
         }
-        const uint32_t xdst = Ls.x + (uint32_t)s * P.x_stage;
-        if (GATEUP && lane < n_e) {
-          // row n lands at n * x_pitch (x_pitch = stage bytes + 16: 16-byte
-          // aligned, and an odd number of 16-byte chunks spreads rows over banks)
-          uint8_t* d = smem_raw + (xdst - raw_s) + lane * P.x_pitch;
-          bulk_load(d, a.x + (size_t)my_tok * a.H + st * subs * 64, (uint32_t)(subs * 128), &full[s]);
+        if (my_slot >= 0) {
+          // slot n at n * x_pitch (x_pitch = stage bytes + 16: 16-byte aligned,
+          // and an odd number of 16-byte chunks spreads the slots over the banks)
+          uint8_t* d = smem_raw + (Ls.x - raw_s) + (uint32_t)s * P.x_stage + (uint32_t)my_slot * P.x_pitch;
+          bulk_load(d, my_src + st * subs * 64, (uint32_t)(subs * 128), &full[s]);
         }
         cp_async_arrive_noinc(&full[s]);
-        if (!GATEUP && lane == 0) {
-          // the expert's h rows, grouped; rows past n_e belong to the next expert or
-          // lie outside the array: they only feed columns nobody writes
-          for (int j = 0; j < subs; ++j) {
-            const int kx = (st * subs + j) * 64;
-            uint8_t* d = smem_raw + (xdst - raw_s) + j * C::kXSuper;  // down only
-            if (NT == 1) {
-              tma_load_2d(d, &tm_x, &full[s], kx, row0);             // h rows 0..3 at atom rows 0..3
-              tma_load_2d(d + 1024, &tm_xl, &full[s], kx, row0 - 4);  // h_lo rows 0..3 at atom rows 4..7
-            } else {
-              tma_load_2d(d, &tm_x, &full[s], kx, row0);                     // h: NT / 2 atoms
-              tma_load_2d(d + (NT / 2) * 1024, &tm_xl, &full[s], kx, row0);  // h_lo
-            }
-          }
-        }
         __syncwarp();
         ring_next(s, ph, ring);
       }
@@ -451,19 +443,14 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     const int r0 = 16 * slab + gq, r1 = r0 + 8;
     const int swz0 = subs == 4 ? (r0 & 7) : ((r0 >> 1) & 3);
     const int swz1 = subs == 4 ? (r1 & 7) : ((r1 >> 1) & 3);
-    // per-lane offsets inside a stage: code chunk 4J + tq of rows r0 / r1, and
-    // this lane's activation run (super-step 2J + (tq >> 1), row gq, chunks
-    // 4 (tq & 1) .. +3 in the 128-byte swizzle)
-    uint32_t coff[2][2], xoff[2][4];
+    // per-lane offsets inside a stage: code chunk 4J + tq of rows r0 / r1; the
+    // activation run of K half J is bytes 256 J + 64 tq .. + 63 of a slot
+    uint32_t coff[2][2];
 #pragma unroll
     for (int J = 0; J < 2; ++J) {
       const int chunk = 4 * J + tq;
       coff[J][0] = (uint32_t)(r0 * row_bytes + ((chunk ^ swz0) << 4));
       coff[J][1] = (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4));
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        xoff[J][c] = GATEUP ? (uint32_t)(gq * P.x_pitch + (2 * J + (tq >> 1)) * 128 + ((tq & 1) * 4 + c) * 16)
-                            : (uint32_t)((2 * J + (tq >> 1)) * C::kXSuper + gq * 128 + ((((tq & 1) * 4 + c) ^ gq) << 4));
     }
     int slot_tab0 = tp.n == 1 ? 0 : -1, slot_tab1 = -1, victim = tp.n == 1 ? 1 : 0;
     uint32_t lgen = 0;
@@ -508,10 +495,11 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       }
       const uint32_t kreg = lane_k | ((uint32_t)slot << 7);
       const Planes PL = make_planes(tp.t[tid]);
-      // activation rows of absent tokens are not read (their operands are zero;
-      // their MMA columns are never written)
+      // activation slot of this lane's column gq in each n-tile; columns of
+      // absent tokens are not read (zero operands; their MMA columns are never
+      // written)
       const int n_e_seg = a.counts[e];
-      uint32_t col_ok[NT];
+      uint32_t xrow[NT], col_ok[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         int tok;
@@ -524,6 +512,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         else
           tok = 8 * (nt & 1) + gq;
         col_ok[nt] = tok < n_e_seg ? 1u : 0u;
+        xrow[nt] = (uint32_t)(8 * nt + gq) * P.x_pitch + (uint32_t)(64 * tq);
       }
       float accc[kMats][C::kTT][C::kChains][4];
 #pragma unroll
@@ -551,17 +540,9 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           uint32_t xr[NT][16];
 #pragma unroll
           for (int nt = 0; nt < NT; ++nt) {
-            int atom;
-            if (GATEUP)
-              atom = nt;
-            else if (NT == 1)
-              atom = gq >> 2;  // h at rows 0..3 of atom 0, h_lo at rows 4..7 of atom 1
-            else
-              atom = nt;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-              lds128_if(xstage + (uint32_t)atom * (GATEUP ? 8 * P.x_pitch : 1024) + xoff[J][c], col_ok[nt],
-                        xr[nt][4 * c + 0],
+              lds128_if(xstage + xrow[nt] + (uint32_t)(256 * J + 16 * c), col_ok[nt], xr[nt][4 * c + 0],
                         xr[nt][4 * c + 1], xr[nt][4 * c + 2], xr[nt][4 * c + 3]);
               dep ^= xr[nt][4 * c + 0];
             }
@@ -756,7 +737,7 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   P.n_max = a.T < 16 ? a.T : 16;
   P.code_stage = (uint32_t)(C::kMats * dk::kRows * 32 * P.subs);
   P.x_pitch = (uint32_t)(P.subs * 128 + 16);
-  P.x_stage = GATEUP ? (uint32_t)(8 * NT) * P.x_pitch : (uint32_t)(P.subs * C::kXSuper);
+  P.x_stage = (uint32_t)C::kXSlots * P.x_pitch;
   P.scale_stage = (uint32_t)(C::kMats * dk::kRows * dk::kScaleSlot);
   P.partial = partial;
   P.counter = counter;
@@ -775,21 +756,17 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   if (!P.ring) return MOE_Q4_ECUDA;
   const uint32_t smem = P.lay.end;
 
-  const int R = a.T * a.k;
   const CUtensorMapSwizzle csw = P.subs == 4 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   const uint32_t cbox = 32u * P.subs;
-  const uint32_t xrows = GATEUP ? 8u * NT : (NT == 4 ? 16u : 8u);
-  CUtensorMap twa, twb, tx, txl;
+  // activation rows come by untiled bulk copies: only the weight codes have maps
+  CUtensorMap twa, twb;
   bool ok;
   if (GATEUP) {
     ok = dk_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.gate_w, a.H / 2, (uint64_t)a.E * a.I, cbox, dk::kRows, csw) &&
          dk_map(&twb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.up_w, a.H / 2, (uint64_t)a.E * a.I, cbox, dk::kRows, csw);
-    tx = txl = twa;  // unused: activation rows come by untiled bulk copies
   } else {
     ok = dk_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.down_w, a.I / 2, (uint64_t)a.E * a.H, cbox, dk::kRows,
-                csw) &&
-         dk_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.h, a.I, R, 64, xrows, CU_TENSOR_MAP_SWIZZLE_128B) &&
-         dk_map(&txl, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.h_lo, a.I, R, 64, xrows, CU_TENSOR_MAP_SWIZZLE_128B);
+                csw);
     twb = twa;
   }
   if (!ok) return MOE_Q4_ECUDA;
@@ -806,7 +783,7 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, dk_kernel<GATEUP, NT, SUBS>, P, tp, twa, twb, tx, txl) == cudaSuccess ? MOE_Q4_OK
+  return cudaLaunchKernelEx(&cfg, dk_kernel<GATEUP, NT, SUBS>, P, tp, twa, twb) == cudaSuccess ? MOE_Q4_OK
                                                                                                  : MOE_Q4_ECUDA;
 }
 
