@@ -63,11 +63,10 @@ namespace dk {
 constexpr int kComputeWarps = 8;                     // one 16-row slab each
 constexpr int kThreads = 32 * (1 + kComputeWarps);   // + the producer warp
 constexpr int kRows = 128;                           // weight rows per tile
-constexpr int kMaxRing = 6;                          // shared-memory stages, at most
+constexpr int kMaxRing = 10;                         // shared-memory stages, at most
 constexpr int kPrmtWords = 1;                        // of the 4 words of a chunk, decoded in registers
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr uint32_t kLutBytes = 65536;  // 256 entries x (2 table slots x 32 lanes x 4 B)
-constexpr uint32_t kScaleSlot = 8;     // scale bytes per row per stage (4 used for 128-K stages)
 constexpr uint32_t kBarBytes = 1024;   // barriers and flags
 }  // namespace dk
 
@@ -82,6 +81,16 @@ struct DkCfg {
   static constexpr int kLoSlot = 4 * NT;
   // 8-token groups of the result
   static constexpr int kTT = GATEUP ? NT : (NT == 4 ? 2 : 1);
+  // bytes of one ring stage of 64 * SUBS K: codes, activation slots, scales
+  template <int SUBS>
+  struct Geom {
+    static constexpr uint32_t kRowBytes = 32 * SUBS;  // code bytes per weight row
+    static constexpr uint32_t kCodeStage = kMats * dk::kRows * kRowBytes;
+    static constexpr uint32_t kXPitch = SUBS * 128 + 16;  // stage bytes of a row + 16
+    static constexpr uint32_t kXStage = kXSlots * kXPitch;
+    static constexpr uint32_t kScaleSlot = 2 * SUBS;  // E8M0 bytes per weight row
+    static constexpr uint32_t kScaleStage = kMats * dk::kRows * kScaleSlot;
+  };
   // independent accumulators per (matrix, token group): MMA mm of K half J adds
   // into chain 2J + (mm & 1) (or J), so no MMA waits on the one before it for
   // long; the chains are added in a fixed order at the end
@@ -150,8 +159,6 @@ struct DkParams {
   int ring;         // shared-memory stages
   DkLayout lay;     // shared-memory placement (offsets)
   int n_max;        // token columns kept in partial sums: min(16, T)
-  uint32_t code_stage, x_stage, scale_stage;
-  uint32_t x_pitch;  // gate/up: bytes per activation row in a stage (subs * 128 + 16)
   float* partial;   // [2 * gridDim.x][mats][n_max][128]
   int32_t* counter; // [units][8 slabs], zero at launch
 };
@@ -233,6 +240,17 @@ __device__ __forceinline__ void lds128_if(uint32_t addr, uint32_t pred, uint32_t
       : "r"(addr), "r"(pred));
 }
 
+// bf16 of 2^(s - 127) for the E8M0 byte of row r0 (low half) and of row r1
+// (high half), `p` = s0 | s1 << 16; s = 0 gives the bf16 subnormal 0x0040 and
+// s = 255 the NaN 0x7FC0, as in the format's definition.
+__device__ __forceinline__ uint32_t e8m0_pair_bf16(uint32_t p) {
+  const uint32_t a = p << 7;                                  // s << 7 per half
+  const uint32_t nan = ((a + 0x00800080u) >> 9) & 0x00400040u;  // bit 6 where s == 255
+  uint32_t m;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(m) : "r"(a), "r"(0x00400040u));  // s == 0 -> 0x0040
+  return m | nan;
+}
+
 __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   uint2 v;
   asm("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
@@ -303,6 +321,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
               const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb) {
   using C = DkCfg<GATEUP, NT>;
   constexpr int kMats = C::kMats;
+  constexpr int kComputeW = dk::kComputeWarps;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   // absolute shared addresses of the placement
@@ -319,8 +338,10 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     if (threadIdx.x == 0) record_error(a.hdr + kStatus, MOE_Q4_ECUDA);
     return;
   }
+  using Geo = typename C::template Geom<SUBS>;
   const auto code_base = [&](int s) -> uint32_t {
-    return s < Ls.n_hi ? Ls.code_hi + (uint32_t)s * P.code_stage : Ls.code_lo + (uint32_t)(s - Ls.n_hi) * P.code_stage;
+    return s < Ls.n_hi ? Ls.code_hi + (uint32_t)s * Geo::kCodeStage
+                       : Ls.code_lo + (uint32_t)(s - Ls.n_hi) * Geo::kCodeStage;
   };
   uint8_t* lut = smem_raw + (Ls.lut - raw_s);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem_raw + (Ls.bars - raw_s));
@@ -334,9 +355,9 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < ring; ++s) {
       mbar_init(&full[s], 1 + 32);  // producer lane 0 (with the TMA bytes) + 32 cp.async arrivals
-      mbar_init(&stage_empty[s], dk::kComputeWarps);
+      mbar_init(&stage_empty[s], kComputeW);
     }
-    mbar_init(lut_bar, 32 * dk::kComputeWarps);
+    mbar_init(lut_bar, 32 * kComputeW);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_wa);
@@ -414,7 +435,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           for (int j = 0; j < 4; ++j) {
             const int r = lane + 32 * j;
             const uint32_t dst =
-                Ls.scales + (uint32_t)s * P.scale_stage + (uint32_t)(m * dk::kRows + r) * dk::kScaleSlot;
+                Ls.scales + (uint32_t)s * Geo::kScaleStage + (uint32_t)(m * dk::kRows + r) * Geo::kScaleSlot;
             if constexpr (subs == 4)
               cp_async_small<8>(dst, sbase + (size_t)r * (K / 32));
             else
@@ -424,7 +445,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         if (my_slot >= 0) {
           // slot n at n * x_pitch (x_pitch = stage bytes + 16: 16-byte aligned,
           // and an odd number of 16-byte chunks spreads the slots over the banks)
-          uint8_t* d = smem_raw + (Ls.x - raw_s) + (uint32_t)s * P.x_stage + (uint32_t)my_slot * P.x_pitch;
+          uint8_t* d = smem_raw + (Ls.x - raw_s) + (uint32_t)s * Geo::kXStage + (uint32_t)my_slot * Geo::kXPitch;
           bulk_load(d, my_src + st * subs * 64, (uint32_t)(subs * 128), &full[s]);
         }
         cp_async_arrive_noinc(&full[s]);
@@ -435,23 +456,34 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     }
   } else {
     // ------------------------------ compute ------------------------------
-    const int slab = warp - 1;     // rows 16 slab .. + 15 of the tile
+    const int cw = warp - 1;
+    const int slab = cw;           // rows 16 slab .. + 15 of the tile
     const int gq = lane >> 2;      // MMA group: rows gq, gq + 8; token column gq
     const int tq = lane & 3;       // code chunk of a half; token columns 2tq, 2tq + 1
     const int ctid = threadIdx.x - 32;
-    constexpr int n_halves = subs / 2; // 128-K halves per stage
-    const int r0 = 16 * slab + gq, r1 = r0 + 8;
+    constexpr int kJ = subs / 2;   // 128-K halves per stage
+    constexpr int kCh = C::kChains;
+    // MMA rows gq and gq + 8 of the slab are tile rows r0 and r1.  With the
+    // 128-byte swizzle the rows of one quarter-warp (gq = 2q, 2q + 1) are
+    // taken 4 apart (r0 & 7 = q and q + 4), so their code chunks, XOR-ed with
+    // r & 7, fall in disjoint halves of the 8 bank groups: no conflict.  (The
+    // 64-byte swizzle of 128-K stages puts consecutive rows in disjoint bank
+    // groups already.)
+    const int r0 = 16 * slab + (subs == 4 ? (((gq & 1) << 2) | (gq >> 1)) : gq), r1 = r0 + 8;
     const int swz0 = subs == 4 ? (r0 & 7) : ((r0 >> 1) & 3);
     const int swz1 = subs == 4 ? (r1 & 7) : ((r1 >> 1) & 3);
-    // per-lane offsets inside a stage: code chunk 4J + tq of rows r0 / r1; the
-    // activation run of K half J is bytes 256 J + 64 tq .. + 63 of a slot
-    uint32_t coff[2][2];
+    // per-lane offsets inside a stage: code chunk 4J + tq of rows r0 / r1 for
+    // each 128-K half J; the activation run of half J is bytes 256 J + 64 tq ..
+    // + 63 of a slot, its scale byte tq of word J of the row
+    uint32_t coff[kJ][2];
 #pragma unroll
-    for (int J = 0; J < 2; ++J) {
+    for (int J = 0; J < kJ; ++J) {
       const int chunk = 4 * J + tq;
       coff[J][0] = (uint32_t)(r0 * row_bytes + ((chunk ^ swz0) << 4));
       coff[J][1] = (uint32_t)(r1 * row_bytes + ((chunk ^ swz1) << 4));
     }
+    // PRMT selector: byte tq of the row-r0 word to byte 0, of the row-r1 word to byte 2
+    const uint32_t psel = (uint32_t)tq | ((uint32_t)(4 + tq) << 8);
     int slot_tab0 = tp.n == 1 ? 0 : -1, slot_tab1 = -1, victim = tp.n == 1 ? 1 : 0;
     uint32_t lgen = 0;
     const uint32_t lane_k = (Ls.lut & 0xffff0000u) | ((uint32_t)lane << 2);
@@ -464,6 +496,22 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     }
     int s = 0;
     uint32_t ph = 0;
+    // shared addresses of ring slot s, advanced with it (no per-stage multiplies)
+    const uint32_t c_first = Ls.n_hi > 0 ? Ls.code_hi : Ls.code_lo;
+    uint32_t cur_c = c_first, cur_s = Ls.scales, cur_x = Ls.x;
+    const auto advance = [&]() {
+      if (++s == ring) {
+        s = 0;
+        ph ^= 1u;
+        cur_c = c_first;
+        cur_s = Ls.scales;
+        cur_x = Ls.x;
+      } else {
+        cur_c = s == Ls.n_hi ? Ls.code_lo : cur_c + Geo::kCodeStage;
+        cur_s += Geo::kScaleStage;
+        cur_x += Geo::kXStage;
+      }
+    };
     bool ok = true;
     for (int g = k0; g < k1 && ok;) {
       const int unit = g / P.stages;
@@ -488,7 +536,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           slot_tab0 = tid;
         else
           slot_tab1 = tid;
-        build_lut_slot(lut, tp.t[tid], slot, ctid);
+        if (ctid < 256) build_lut_slot(lut, tp.t[tid], slot, ctid);  // one table entry per thread
         mbar_arrive(lut_bar);
         if (!mbar_wait_warp(lut_bar, lgen & 1, abort_flag, dk::kWaitNs)) break;
         ++lgen;
@@ -512,15 +560,15 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         else
           tok = 8 * (nt & 1) + gq;
         col_ok[nt] = tok < n_e_seg ? 1u : 0u;
-        xrow[nt] = (uint32_t)(8 * nt + gq) * P.x_pitch + (uint32_t)(64 * tq);
+        xrow[nt] = (uint32_t)(8 * nt + gq) * Geo::kXPitch + (uint32_t)(64 * tq);
       }
-      float accc[kMats][C::kTT][C::kChains][4];
+      float accc[kMats][C::kTT][kCh][4];
 #pragma unroll
       for (int m = 0; m < kMats; ++m)
 #pragma unroll
         for (int tt = 0; tt < C::kTT; ++tt)
 #pragma unroll
-          for (int c = 0; c < C::kChains; ++c)
+          for (int c = 0; c < kCh; ++c)
 #pragma unroll
             for (int i = 0; i < 4; ++i) accc[m][tt][c][i] = 0.0f;
 
@@ -529,13 +577,12 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           ok = false;
           break;
         }
-        const uint32_t cbase = after_wait(code_base(s));
-        const uint32_t sbase = after_wait(Ls.scales + (uint32_t)s * P.scale_stage);
-        const uint32_t xstage = after_wait(Ls.x + (uint32_t)s * P.x_stage);
+        const uint32_t cbase = after_wait(cur_c);
+        const uint32_t sbase = after_wait(cur_s);
+        const uint32_t xstage = after_wait(cur_x);
         uint32_t dep = 0;  // every word read from the stage, folded
 #pragma unroll
-        for (int J = 0; J < 2; ++J) {
-          if (J >= n_halves) break;
+        for (int J = 0; J < kJ; ++J) {
           // activation operands: 16 pairs per n-tile, pair p at K offset 32 tq + 2p
           uint32_t xr[NT][16];
 #pragma unroll
@@ -552,15 +599,23 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
             const uint32_t mb = cbase + (uint32_t)(m * dk::kRows * row_bytes);
             const uint4 c0 = lds128(mb + coff[J][0]);
             const uint4 c1 = lds128(mb + coff[J][1]);
-            const uint2 s0 = lds64(sbase + (uint32_t)((m * dk::kRows + r0) * dk::kScaleSlot));
-            const uint2 s1 = lds64(sbase + (uint32_t)((m * dk::kRows + r1) * dk::kScaleSlot));
-            dep ^= c0.x ^ c1.x ^ s0.x ^ s1.x;
-            // E8M0 byte of block 4J + tq
-            const uint32_t e0 = ((J ? s0.y : s0.x) >> (8 * tq)) & 0xffu;
-            const uint32_t e1 = ((J ? s1.y : s1.x) >> (8 * tq)) & 0xffu;
+            // scale word of this half (4 E8M0 bytes, block 4J + tq in byte tq)
+            uint32_t w0, w1;
+            if constexpr (SUBS == 4) {
+              const uint2 s0 = lds64(sbase + (uint32_t)((m * dk::kRows + r0) * Geo::kScaleSlot));
+              const uint2 s1 = lds64(sbase + (uint32_t)((m * dk::kRows + r1) * Geo::kScaleSlot));
+              w0 = J ? s0.y : s0.x;
+              w1 = J ? s1.y : s1.x;
+            } else {
+              w0 = lds32_nv(sbase + (uint32_t)((m * dk::kRows + r0) * Geo::kScaleSlot));
+              w1 = lds32_nv(sbase + (uint32_t)((m * dk::kRows + r1) * Geo::kScaleSlot));
+            }
+            dep ^= c0.x ^ c1.x ^ w0 ^ w1;
+            // byte tq of each row's word (block 4J + tq), as bf16 scales for both rows
+            const uint32_t sc = e8m0_pair_bf16(prmt(w0, w1, psel) & 0x00ff00ffu);
             uint32_t pa[16], pb[16];
-            decode_chunk(c0, PL, kreg, scale_bf16x2(e0), pa);
-            decode_chunk(c1, PL, kreg, scale_bf16x2(e1), pb);
+            decode_chunk(c0, PL, kreg, prmt(sc, 0u, 0x1010u), pa);
+            decode_chunk(c1, PL, kreg, prmt(sc, 0u, 0x3232u), pb);
 #pragma unroll
             for (int mm = 0; mm < 8; ++mm) {
 #pragma unroll
@@ -577,7 +632,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         // once the loads above have returned (their values feed `dep`)
         dep = __reduce_xor_sync(0xffffffffu, dep);
         if (lane == 0) arrive_after(&stage_empty[s], dep);
-        ring_next(s, ph, ring);
+        advance();
       }
       if (!ok) break;
 
@@ -590,7 +645,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           for (int i = 0; i < 4; ++i) {
             float v = accc[m][tt][0][i];
 #pragma unroll
-            for (int c = 1; c < C::kChains; ++c) v += accc[m][tt][c][i];
+            for (int c = 1; c < kCh; ++c) v += accc[m][tt][c][i];
             acc[m][tt][i] = v;
           }
       if (!GATEUP && NT == 1) {
@@ -735,10 +790,7 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   // stage indices are 32-bit on the device
   if ((uint64_t)a.E * (uint64_t)P.tiles_per_e * (uint64_t)P.stages >= (1ull << 31)) return MOE_Q4_EINVAL;
   P.n_max = a.T < 16 ? a.T : 16;
-  P.code_stage = (uint32_t)(C::kMats * dk::kRows * 32 * P.subs);
-  P.x_pitch = (uint32_t)(P.subs * 128 + 16);
-  P.x_stage = (uint32_t)C::kXSlots * P.x_pitch;
-  P.scale_stage = (uint32_t)(C::kMats * dk::kRows * dk::kScaleSlot);
+  using Geo = typename C::template Geom<SUBS>;
   P.partial = partial;
   P.counter = counter;
 
@@ -750,7 +802,8 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
   P.ring = 0;
   for (int rs = dk::kMaxRing; rs >= 2 && !P.ring; --rs)
-    if (dk_layout((uint32_t)reserved, (uint32_t)reserved + (uint32_t)optin, P.code_stage, P.x_stage, P.scale_stage,
+    if (dk_layout((uint32_t)reserved, (uint32_t)reserved + (uint32_t)optin, Geo::kCodeStage, Geo::kXStage,
+                  Geo::kScaleStage,
                   rs, P.lay))
       P.ring = rs;
   if (!P.ring) return MOE_Q4_ECUDA;
