@@ -296,25 +296,37 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
       const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * (C::kMats * kBN);
       const int wrow = m * kBM + row;
       const int n_hi = n_e - nt * kBN < kBN ? n_e - nt * kBN : kBN;  // tokens of this tile
-#pragma unroll 1
-      for (int c0 = 0; c0 < n_hi; c0 += 16) {
-        float g[16];
-        tmem_ld16(tb + c0, g);
-        if (GATEUP) {
-          float u[16];
-          tmem_ld16(tb + kBN + c0, u);
+      // 8 token columns of every matrix per chunk; the next chunk's TMEM loads
+      // are in flight while this chunk is finished (one wait per chunk)
+      constexpr int kCw = 8;
+      uint32_t va[C::kMats][kCw], vb[C::kMats][kCw];
+      const auto issue = [&](uint32_t (*v)[kCw], int c0) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = nt * kBN + c0 + j;
-            if (n < n_e) a.h[(size_t)(row0 + n) * a.I + wrow] = __float2bfloat16_rn(silu_mul(g[j], u[j]));
-          }
-        } else {
+        for (int mt = 0; mt < C::kMats; ++mt) tmem_ld8_nowait(tb + mt * kBN + c0, v[mt]);
+      };
+      const auto finish = [&](uint32_t (*v)[kCw], int c0) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = nt * kBN + c0 + j;
-            if (n < n_e) a.y[(size_t)(row0 + n) * a.H + wrow] = g[j];
-          }
+        for (int j = 0; j < kCw; ++j) {
+          const int n = nt * kBN + c0 + j;
+          if (n >= n_e) break;
+          if (GATEUP)
+            a.h[(size_t)(row0 + n) * a.I + wrow] =
+                __float2bfloat16_rn(silu_mul_fast(__uint_as_float(v[0][j]), __uint_as_float(v[C::kMats - 1][j])));
+          else
+            a.y[(size_t)(row0 + n) * a.H + wrow] = __uint_as_float(v[0][j]);
         }
+      };
+      issue(va, 0);
+      tmem_wait_ld();
+#pragma unroll 1
+      for (int c0 = 0; c0 < n_hi; c0 += 2 * kCw) {
+        if (c0 + kCw < n_hi) issue(vb, c0 + kCw);
+        finish(va, c0);
+        tmem_wait_ld();
+        if (c0 + kCw >= n_hi) break;
+        if (c0 + 2 * kCw < n_hi) issue(va, c0 + 2 * kCw);
+        finish(vb, c0 + kCw);
+        tmem_wait_ld();
       }
       tc_fence_before();
       __syncwarp();
