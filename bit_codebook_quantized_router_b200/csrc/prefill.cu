@@ -55,7 +55,9 @@ struct TcCfg {
   // gate/up 2 matrices x 128 rows x 2 chunks, down 128 rows x 2 chunks
   static constexpr int kDequantThreads = kMats * 256;
   static constexpr int kEpiWarp0 = 2 + kDequantThreads / 32;
-  static constexpr int kThreads = 32 * (kEpiWarp0 + 4);
+  // epilogue: two warps per 32-lane TMEM quarter, each finishing half the tokens
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
   static constexpr int kStages = GATEUP ? 3 : 4;
   static constexpr int kATile = kBM * kBK * 2;        // 16 KB bf16 per matrix
   static constexpr int kBTile = kBN * kBK * 2;        // 16 KB
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], C::kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -281,6 +283,7 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
   } else {
     // ---------------- epilogue ----------------
     const int quad = warp & 3;          // TMEM lanes 32*quad .. +31
+    const int ehalf = (warp - C::kEpiWarp0) >> 2;  // tokens 128 ehalf .. + 127 of the tile
     const int row = quad * 32 + lane;   // weight row in the tile
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < total && !warp_aborted(abort_flag); tile += gridDim.x, ++tcount) {
@@ -304,29 +307,38 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
 #pragma unroll
         for (int mt = 0; mt < C::kMats; ++mt) tmem_ld8_nowait(tb + mt * kBN + c0, v[mt]);
       };
+      // this thread's row in the output rows of the tile's tokens: token c of the
+      // tile at out_row + c * stride
+      const size_t stride = GATEUP ? (size_t)a.I : (size_t)a.H;
+      const size_t out_off = (size_t)(row0 + nt * kBN) * stride + (size_t)wrow;
       const auto finish = [&](uint32_t (*v)[kCw], int c0) {
+        const int valid = n_hi - c0;  // tokens of this chunk that exist (>= 1)
+        size_t o = out_off + (size_t)c0 * stride;
 #pragma unroll
-        for (int j = 0; j < kCw; ++j) {
-          const int n = nt * kBN + c0 + j;
-          if (n >= n_e) break;
+        for (int j = 0; j < kCw; ++j, o += stride) {
+          if (valid < kCw && j >= valid) break;
           if (GATEUP)
-            a.h[(size_t)(row0 + n) * a.I + wrow] =
-                __float2bfloat16_rn(silu_mul_fast(__uint_as_float(v[0][j]), __uint_as_float(v[C::kMats - 1][j])));
+            a.h[o] = __float2bfloat16_rn(silu_mul_fast(__uint_as_float(v[0][j]), __uint_as_float(v[C::kMats - 1][j])));
           else
-            a.y[(size_t)(row0 + n) * a.H + wrow] = __uint_as_float(v[0][j]);
+            a.y[o] = __uint_as_float(v[0][j]);
         }
       };
-      issue(va, 0);
-      tmem_wait_ld();
+      // this warp's tokens: [c_lo, c_hi) of the tile
+      const int c_lo = (kBN / 2) * ehalf;
+      const int c_hi = n_hi < c_lo + kBN / 2 ? n_hi : c_lo + kBN / 2;
+      if (c_lo < c_hi) {
+        issue(va, c_lo);
+        tmem_wait_ld();
 #pragma unroll 1
-      for (int c0 = 0; c0 < n_hi; c0 += 2 * kCw) {
-        if (c0 + kCw < n_hi) issue(vb, c0 + kCw);
-        finish(va, c0);
-        tmem_wait_ld();
-        if (c0 + kCw >= n_hi) break;
-        if (c0 + 2 * kCw < n_hi) issue(va, c0 + 2 * kCw);
-        finish(vb, c0 + kCw);
-        tmem_wait_ld();
+        for (int c0 = c_lo; c0 < c_hi; c0 += 2 * kCw) {
+          if (c0 + kCw < c_hi) issue(vb, c0 + kCw);
+          finish(va, c0);
+          tmem_wait_ld();
+          if (c0 + kCw >= c_hi) break;
+          if (c0 + 2 * kCw < c_hi) issue(va, c0 + 2 * kCw);
+          finish(vb, c0 + kCw);
+          tmem_wait_ld();
+        }
       }
       tc_fence_before();
       __syncwarp();
