@@ -148,10 +148,11 @@ MOE_Q4_API size_t moe_q4_forward_workspace(const moe_q4_layer* layer, int T, int
  * logits in fp32.  Rows are grouped by expert (ascending id), tokens
  * ascending within an expert.  Each expert's rows go through the small-M
  * streaming path or the tensor-core path, chosen on the device from the
- * per-expert row count.  The intermediate h = silu(g)*u is kept as a pair of
- * bf16 values (its rounding and the rounding of the remainder), so the down
- * GEMM sees it to ~16 significant bits; y is fp32; the combine sums
- * the top_k slots in slot order in fp32 (deterministic, no atomics).
+ * per-expert row count.  The intermediate h = silu(g)*u is computed in fp32
+ * and stored as bf16; on the small-M path also the bf16 rounding of its
+ * remainder, so that path's down GEMM sees h to ~16 significant bits.  y is
+ * fp32; the combine sums the top_k slots in slot order in fp32
+ * (deterministic, no atomics).
  * Arguments:
  *   layer      see moe_q4_layer;
  *   x          device, bf16 [T][H];
