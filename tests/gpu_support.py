@@ -22,6 +22,29 @@ from bit_codebook_quantized_router_b200 import inputs
 REL_FRO = 5e-3
 MAX_ABS_RMS = 2e-2
 
+# Canary bands: every buffer the library writes in the forward tests sits
+# inside a larger allocation whose bytes before and after it hold a fixed
+# pattern, checked after the call (catches writes past an output's end).
+GUARD_BYTES = 4096  # keeps the view 512-byte aligned, as the workspace needs
+GUARD_BYTE = 0xA5
+
+
+class Guarded:
+    """A tensor `view` of `shape` and `dtype` with canary bands around it."""
+
+    def __init__(self, shape, dtype, device="cuda"):
+        esize = torch.tensor([], dtype=dtype).element_size()
+        self.n = int(np.prod(shape)) * esize
+        self.buf = torch.full((self.n + 2 * GUARD_BYTES,), GUARD_BYTE, dtype=torch.uint8, device=device)
+        self.view = self.buf[GUARD_BYTES:GUARD_BYTES + self.n].view(dtype).view(shape)
+
+    def check(self, what=""):
+        head = self.buf[:GUARD_BYTES]
+        tail = self.buf[GUARD_BYTES + self.n:]
+        assert bool((head == GUARD_BYTE).all()) and bool((tail == GUARD_BYTE).all()), \
+            f"{what}: bytes written outside the buffer"
+
+
 _POOL = None
 
 

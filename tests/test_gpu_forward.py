@@ -30,14 +30,20 @@ def _small_device_layer(w, identical_to=None):
 
 
 def _run(dev, x, lg, k):
+    """One forward with every output and the workspace inside canary bands."""
     T = x.shape[0]
-    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
-    wts = torch.empty((T, k), dtype=torch.float32, device="cuda")
-    counts = torch.empty(dev.E, dtype=torch.int32, device="cuda")
-    out_f32 = torch.empty((T, dev.H), dtype=torch.float32, device="cuda")
-    ws = q4.alloc_workspace(q4.forward_workspace(dev, T, k))
-    out = q4.forward(dev, x, lg, k, ws=ws, topk_ids=ids, topk_w=wts, counts=counts, out_f32=out_f32)
+    G = gpu_support.Guarded
+    bufs = {"ids": G((T, k), torch.int32), "wts": G((T, k), torch.float32), "counts": G((dev.E,), torch.int32),
+            "out_f32": G((T, dev.H), torch.float32), "out": G((T, dev.H), torch.bfloat16),
+            "ws": G((q4.forward_workspace(dev, T, k),), torch.uint8)}
+    ids, wts, counts = bufs["ids"].view, bufs["wts"].view, bufs["counts"].view
+    out_f32, ws = bufs["out_f32"].view, bufs["ws"].view
+    out = q4.forward(dev, x, lg, k, out=bufs["out"].view, ws=ws, topk_ids=ids, topk_w=wts, counts=counts,
+                     out_f32=out_f32)
+    torch.cuda.synchronize()
     assert q4.forward_status(ws) == 0
+    for name, b in bufs.items():
+        b.check(name)
     gpu_support.check_bf16_is_rounding(out, out_f32)
     return out_f32, ids, wts, counts
 
@@ -54,11 +60,13 @@ def test_tiny_workload_full():
     gpu_support.check_out(out, ref, "tiny")
 
 
-# Edge cases on a small layer (H=256, I=128, E=8): T=1; counts of exactly a
-# token tile (16) and a tile + 1 (17); experts with 0 rows; every token on one
-# expert; k = 1; k = E.
+# Edge cases on a small layer (H=256, I=128, E=8): T=1; an expert with
+# exactly the small-M path's limit (16 rows) and one more (17, the tensor-core
+# path); exactly one tensor-core token tile (256) and one more (257); experts
+# with 0 rows; every token on one expert; k = 1; k = E.
 @pytest.mark.parametrize("T,k,bias", [(1, 2, None), (16, 1, 3), (17, 1, 3), (33, 2, None),
-                                      (40, 2, 5), (64, 8, None), (200, 2, None), (300, 3, 0)])
+                                      (40, 2, 5), (64, 8, None), (200, 2, None), (256, 1, 3), (257, 1, 3),
+                                      (300, 3, 0)])
 def test_small_layer_edge_counts(T, k, bias):
     w = inputs.Workload("small", 7, T, inputs.TINY)
     L, dev = _small_device_layer(w)

@@ -68,7 +68,10 @@ def test_dequant_bit_exact_every_scale_byte(table_index):
     scales = np.empty((E, N, K // 32), np.uint8)
     scales.reshape(-1)[:] = np.arange(scales.size) % 256  # every scale byte, 0..255
     ref = oracle.dequant(codes, scales, tables, tid, E, N, K)
-    got = q4.dequant(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), tables, tid)
+    out = gpu_support.Guarded((E, N, K), torch.bfloat16)  # canary bands around the output
+    got = q4.dequant(torch.from_numpy(codes).cuda(), torch.from_numpy(scales).cuda(), tables, tid, out=out.view)
+    torch.cuda.synchronize()
+    out.check("dequant output")
     got_bits = inputs.bf16_bits(got)
     bad = np.nonzero(got_bits != ref)
     assert bad[0].size == 0, (bad[0][:5], got_bits[bad][:5], ref[bad][:5])
