@@ -411,6 +411,41 @@ def measure_dequant(q4, layer, hbm_peak, flush_l2, stream, reps=5):
             "gbs": gbs, "frac": gbs / hbm_peak, "frac_of_datasheet": gbs / DATASHEET_HBM_GBS}
 
 
+def measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream, reps=20):
+    """The router gate ahead of the layer (moe_q4_router): bf16 x [T, H] times
+    the bf16 gate [E, H] -> fp32 logits.  Algorithmic work: the gate and x read
+    and the logits written (bytes), 2 T E H flop; reported against the HBM
+    roofline at decode sizes and the tensor roofline at prefill sizes."""
+    sh = w.shape
+    gate = inputs.router_weight(w, device="cuda")
+    T = xs[0].shape[0]
+    out = torch.empty((T, sh.E), dtype=torch.float32, device="cuda")
+    need = q4.router_workspace(T, sh.H, sh.E)
+    ws = q4.alloc_workspace(need) if need else None
+    for i in range(3):
+        q4.router(xs[i % len(xs)], gate, out=out, ws=ws)
+    torch.cuda.synchronize()
+    st = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    en = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    for i in range(reps):
+        flush_l2(i)
+        st[i].record(stream)
+        q4.router(xs[i % len(xs)], gate, out=out, ws=ws)
+        en[i].record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in zip(st, en)) / reps
+    nbytes = sh.E * sh.H * 2 + T * sh.H * 2 + T * sh.E * 4
+    flop = 2.0 * T * sh.E * sh.H
+    gbs = nbytes / (ms / 1e3) / 1e9
+    tfs = flop / (ms / 1e3) / 1e12
+    hbm_bound = T <= 256
+    return {"kernel": "router_kernel (+ router_reduce_kernel when K is split)", "ms": ms, "bytes": nbytes,
+            "flop": flop, "gbs": gbs, "tflops": tfs, "bound": "hbm" if hbm_bound else "tensor",
+            "frac": gbs / hbm_peak if hbm_bound else tfs / tf_peak,
+            "frac_of_datasheet": gbs / DATASHEET_HBM_GBS if hbm_bound else tfs / DATASHEET_BF16_TFLOPS,
+            "note": "mma.sync bf16 GEMM; not part of the step (the layer's input is the logits)"}
+
+
 def run_ours(args, w):
     import torch.distributed as dist
 
@@ -514,6 +549,7 @@ def run_ours(args, w):
     hbm_peak, tf_peak, peak_src = load_peaks()
     graph_ms, graph_why = measure_graph(q4, layer, xs, lgs, k, out, ws, flush_l2, min(args.steps, 200), stream)
     dq = measure_dequant(q4, layer, hbm_peak, flush_l2, stream) if not args.no_dequant else None
+    rt = measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream)
     work = [kernel_work(sh, T, c) for c in counts]
     roof, kernels = roofline(work, kern_ms, n_prof, hbm_peak, tf_peak, peak_src)
     gu, dn = expert_bytes(sh)
@@ -538,6 +574,7 @@ def run_ours(args, w):
                    "note": "same forward replayed from CUDA graphs, L2 flushed outside the events"}
                   if graph_ms else {"value": None, "unavailable": graph_why}),
         "dequant": dq,
+        "router": rt,
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk.summary(),
     }

@@ -7,8 +7,9 @@ raises if the library was not built (there is no CPU fallback).
 """
 from ._lib import (Layer, MoeQ4Error, alloc_workspace, dequant, forward, forward_host,
                    forward_host_workspace, forward_stages, forward_status, forward_workspace, lib, pack, route,
+                   router, router_workspace,
                    status_string)
 
 __all__ = ["Layer", "MoeQ4Error", "alloc_workspace", "dequant", "forward", "forward_host",
            "forward_host_workspace", "forward_stages", "forward_status", "forward_workspace", "lib", "pack",
-           "route", "status_string"]
+           "route", "router", "router_workspace", "status_string"]

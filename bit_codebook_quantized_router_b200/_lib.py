@@ -62,9 +62,12 @@ def lib():
         L.moe_q4_route.argtypes = [vp, ci, ci, ci, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_q4_forward_stages.argtypes = [ctypes.POINTER(_LayerStruct), vp, vp, ci, ci, vp, vp, sz, vp,
                                             ctypes.POINTER(ctypes.c_void_p), ci]
+        L.moe_q4_router_workspace.argtypes = [ci, ci, ci]
+        L.moe_q4_router_workspace.restype = sz
+        L.moe_q4_router.argtypes = [vp, vp, ci, ci, ci, vp, vp, sz, vp]
         for f in (L.moe_q4_pack, L.moe_q4_dequant, L.moe_q4_forward, L.moe_q4_forward_host,
                   L.moe_q4_forward_status, L.moe_q4_read_status, L.moe_q4_route,
-                  L.moe_q4_forward_stages):
+                  L.moe_q4_forward_stages, L.moe_q4_router):
             f.restype = ci
         if L.moe_q4_abi_version() != 1:
             raise ImportError("libmoe_q4 ABI version mismatch")
@@ -222,6 +225,28 @@ def route(logits: torch.Tensor, k: int, stream=None):
                               _stream(stream)), "moe_q4_route")
     st = forward_status(ws, stream)
     return ids, w, counts, offsets, row_token, inv, st
+
+
+def router_workspace(T: int, H: int, E: int) -> int:
+    return int(lib().moe_q4_router_workspace(T, H, E))
+
+
+def router(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+           stream=None) -> torch.Tensor:
+    """Router logits: bf16 hidden states x [T, H] and bf16 gate w [E, H] ->
+    fp32 logits [T, E] (into `out` if given)."""
+    if x.dtype != torch.bfloat16 or w.dtype != torch.bfloat16 or x.dim() != 2 or w.dim() != 2:
+        raise ValueError("x [T, H] and w [E, H] must be bf16 matrices")
+    T, H = x.shape
+    E = w.shape[0]
+    if out is None:
+        out = torch.empty((T, E), dtype=torch.float32, device=x.device)
+    need = router_workspace(T, H, E)
+    if ws is None and need > 0:
+        ws = alloc_workspace(need, x.device)
+    _check(lib().moe_q4_router(_ptr(x.contiguous()), _ptr(w.contiguous()), T, H, E, _ptr(out), _ptr(ws),
+                               0 if ws is None else ws.numel(), _stream(stream)), "moe_q4_router")
+    return out
 
 
 def forward_stages(layer: Layer, x, logits, k: int, out, ws, events, stream=None) -> None:

@@ -179,6 +179,14 @@ def router_logits(w: Workload, device="cpu", T: int | None = None, variant: int 
     return lg.contiguous()
 
 
+def router_weight(w: Workload, device="cpu") -> torch.Tensor:
+    """bf16 [E, H] router gate (the "mlp.gate" linear the pages hold in
+    BF16): N(0, 0.02), seeded from the workload's weight seed."""
+    g = _gen(w.seed_weights * 7919 + 5, device)
+    return (torch.randn((w.shape.E, w.shape.H), generator=g, device=device, dtype=torch.float32) * 0.02).to(
+        torch.bfloat16).contiguous()
+
+
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """Host uint16 view of a bf16 tensor's bit patterns."""
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)

@@ -119,6 +119,27 @@ MOE_Q4_API int moe_q4_dequant(const uint8_t* weight, const uint8_t* weight_scale
                    int n_tables, const uint8_t* table_id, int E, int N, int K, void* out,
                    void* stream);
 
+/* ---------------------------------------------------------------------------
+ * moe_q4_router -- router logits of T tokens: the router gate ("mlp.gate",
+ * held in BF16 per "GLM-5.2-EXL3-DENSE6-MTP78", "Quant recipe") applied to
+ * the hidden states ahead of routing:
+ *   logits[t][e] = sum over h of x[t][h] * w[e][h]   (fp32 accumulate)
+ * Deterministic: the same inputs give the same bits (fixed summation order).
+ *   x         device, bf16 [T][H], 16-byte aligned;
+ *   w         device, bf16 [E][H], 16-byte aligned;
+ *   T >= 0; H > 0, H % 32 == 0; E > 0;
+ *   logits    device, fp32 [T][E] (out): the input of moe_q4_forward;
+ *   ws        device workspace of at least moe_q4_router_workspace(T, H, E)
+ *             bytes (16-byte aligned; may be NULL when that is 0), owned by
+ *             the call until the enqueued work completes;
+ *   ws_bytes  size of ws.
+ * Returns MOE_Q4_EINVAL for bad sizes or pointers, MOE_Q4_EWORKSPACE for a
+ * missing or short workspace; no host synchronisation, no allocation.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API size_t moe_q4_router_workspace(int T, int H, int E);
+MOE_Q4_API int moe_q4_router(const void* x, const void* w, int T, int H, int E, float* logits, void* ws,
+                             size_t ws_bytes, void* stream);
+
 /* A packed MoE layer.  Device pointers are borrowed for the duration of
  * each call; tables and table_id are host memory read during each call. */
 typedef struct moe_q4_layer {

@@ -61,11 +61,12 @@ def lib():
         L.oq_decode_matrix_f64.argtypes = [vp, vp, vp, ci, ci, vp]
         L.oq_pack.argtypes = [vp, ci, ci, ci, vp, ci, vp, vp, vp]
         L.oq_route.argtypes = [vp, ci, ci, ci, vp, vp]
+        L.oq_router_logits.argtypes = [vp, vp, ci, ci, ci, vp, vp]
         L.oq_group.argtypes = [vp, ci, ci, ci, vp, vp, vp, vp]
         L.oq_moe_tokens.argtypes = [ctypes.POINTER(_Layer), vp, vp, ci, ci, vp, vp, vp]
         L.oq_expert_partial.argtypes = [ctypes.POINTER(_Layer), ci, vp, ci, ci, vp]
         for f in (L.oq_dequant, L.oq_decode_matrix_f64, L.oq_pack, L.oq_route, L.oq_group, L.oq_moe_tokens,
-                  L.oq_expert_partial):
+                  L.oq_expert_partial, L.oq_router_logits):
             f.restype = ci
         _lib = L
     return _lib
@@ -126,6 +127,22 @@ def pack(src_bf16_bits, tables, table_id, E, N, K):
     s = np.empty((E, N, K // 32), np.uint8)
     _check(lib().oq_pack(_p(src), E, N, K, _p(t), nt, _p(tid), _p(w), _p(s)))
     return w, s
+
+
+def router_logits(x_bf16_bits, w_bf16_bits):
+    """Router logits of the bf16 hidden states x [T, H] under the bf16 router
+    gate w [E, H], in fp64: (logits [T, E], absdot [T, E]) with absdot the sum
+    of |x[t][h] w[e][h]| (the scale of a finite-precision evaluation's error)."""
+    x = _c(x_bf16_bits, np.uint16)
+    w = _c(w_bf16_bits, np.uint16)
+    T, H = x.shape
+    E = w.shape[0]
+    if w.shape[1] != H:
+        raise OracleError("x and w disagree on H")
+    logits = np.zeros((T, E), np.float64)
+    absdot = np.zeros((T, E), np.float64)
+    _check(lib().oq_router_logits(_p(x), _p(w), T, H, E, _p(logits), _p(absdot)))
+    return logits, absdot
 
 
 def route(logits, k):

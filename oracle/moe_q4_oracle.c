@@ -16,6 +16,8 @@
  *   [TR3v4]      "GLM-5.2 EXL3 TR3 v4 -- 3.5 bpw mixed experts" README,
  *                "Shared residual rotations, private intermediate rotations"
  *                (routing-weighted sum of expert outputs).
+ *   [DENSE6]     "GLM-5.2-EXL3-DENSE6-MTP78", section "Quant recipe" (the
+ *                router mlp.gate is held in BF16).
  *
  * Precision: every floating-point value of the MoE is carried in fp64.  The
  * dequantisation entry point produces bf16 bit patterns under the rule
@@ -231,6 +233,34 @@ int oq_pack(const uint16_t* src, int E, int N, int K, const float* tables, int n
       }
     }
   }
+  return OQ_OK;
+}
+
+/* ---- router logits ----------------------------------------------------- */
+
+/* Router logits of T tokens: logits[t][e] = sum over h of x[t][h] * w[e][h],
+ * the router gate ("mlp.gate", held in BF16 per [DENSE6, "Quant recipe"])
+ * applied to the hidden states, with the geometry of [ROUND7, "Ground truth
+ * and corrections"] (hidden 6144, 256 routed experts).  x and w are bf16 bit
+ * patterns; each product is exact in fp64 and the sum runs over h in order.
+ * absdot[t][e] (optional) = sum of |x[t][h] * w[e][h]|, the scale of the
+ * rounding error a finite-precision evaluation may make.
+ * x: [T][H]; w: [E][H]; logits, absdot: [T][E]. */
+int oq_router_logits(const uint16_t* x, const uint16_t* w, int T, int H, int E, double* logits, double* absdot) {
+  if (T < 0 || H < 0 || E < 1) return OQ_EINVAL;
+  if (T == 0) return OQ_OK;
+  if (!x || !w || !logits) return OQ_EINVAL;
+  for (int t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0, mag = 0.0;
+      for (int h = 0; h < H; ++h) {
+        const double p = (double)bf16_bits_to_f32(x[(size_t)t * H + h]) * (double)bf16_bits_to_f32(w[(size_t)e * H + h]);
+        acc += p;
+        mag += fabs(p);
+      }
+      logits[(size_t)t * E + e] = acc;
+      if (absdot) absdot[(size_t)t * E + e] = mag;
+    }
   return OQ_OK;
 }
 
