@@ -32,11 +32,23 @@ struct RouterPlan {
   int e_tiles, t_tiles, chunks, steps;
 };
 
+// With one token tile (decode sizes) each warp unit takes exactly kFewSteps
+// steps of K, a compile-time count, so that all its loads are issued before
+// its first MMA waits; the K range is then cut into H / (32 kFewSteps) chunks.
+constexpr int kFewSteps = 4;
+
+static bool router_few(int T, int H) { return T <= rt::kTokens && H % (rt::kKStep * kFewSteps) == 0; }
+
 static RouterPlan router_plan(int T, int H, int E) {
   RouterPlan p;
   p.e_tiles = (E + rt::kRows - 1) / rt::kRows;
   p.t_tiles = (T + rt::kTokens - 1) / rt::kTokens;
   const int ksteps = H / rt::kKStep;
+  if (router_few(T, H)) {
+    p.steps = kFewSteps;
+    p.chunks = ksteps / kFewSteps;
+    return p;
+  }
   const long long base = (long long)p.e_tiles * p.t_tiles;
   long long want = base > 0 ? rt::kTargetWarps / base : 1;
   if (want < 1) want = 1;
@@ -46,6 +58,8 @@ static RouterPlan router_plan(int T, int H, int E) {
   return p;
 }
 
+// FEW: every unit takes exactly kFewSteps steps (plan.steps == kFewSteps).
+template <bool FEW>
 __global__ void __launch_bounds__(rt::kThreads) router_kernel(const uint16_t* __restrict__ x,
                                                               const uint16_t* __restrict__ w, int T, int H, int E,
                                                               RouterPlan plan, float* __restrict__ out) {
@@ -75,14 +89,35 @@ __global__ void __launch_bounds__(rt::kThreads) router_kernel(const uint16_t* __
     for (int nt = 0; nt < rt::kNT; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
-#pragma unroll 4
-    for (int k = k_begin; k < k_end; k += rt::kKStep) {
-      const uint4 a = ldg_nc(wa + k), b = ldg_nc(wb + k);
+    if constexpr (FEW) {
+      // all loads of the unit first, then the MMAs (one token tile: the x rows
+      // of the four column tiles repeat, so only distinct rows are loaded)
+      uint4 a[kFewSteps], b[kFewSteps], v[kFewSteps][rt::kNT];
 #pragma unroll
-      for (int nt = 0; nt < rt::kNT; ++nt) {
-        const uint4 v = ldg_nc(xr[nt] + k);
-        mma_16816(acc[nt], a.x, b.x, a.y, b.y, v.x, v.y);
-        mma_16816(acc[nt], a.z, b.z, a.w, b.w, v.z, v.w);
+      for (int j = 0; j < kFewSteps; ++j) {
+        const int k = k_begin + j * rt::kKStep;
+        a[j] = ldg_nc(wa + k);
+        b[j] = ldg_nc(wb + k);
+#pragma unroll
+        for (int nt = 0; nt < rt::kNT; ++nt) v[j][nt] = ldg_nc(xr[nt] + k);
+      }
+#pragma unroll
+      for (int j = 0; j < kFewSteps; ++j)
+#pragma unroll
+        for (int nt = 0; nt < rt::kNT; ++nt) {
+          mma_16816(acc[nt], a[j].x, b[j].x, a[j].y, b[j].y, v[j][nt].x, v[j][nt].y);
+          mma_16816(acc[nt], a[j].z, b[j].z, a[j].w, b[j].w, v[j][nt].z, v[j][nt].w);
+        }
+    } else {
+#pragma unroll 4
+      for (int k = k_begin; k < k_end; k += rt::kKStep) {
+        const uint4 a = ldg_nc(wa + k), b = ldg_nc(wb + k);
+#pragma unroll
+        for (int nt = 0; nt < rt::kNT; ++nt) {
+          const uint4 v = ldg_nc(xr[nt] + k);
+          mma_16816(acc[nt], a.x, b.x, a.y, b.y, v.x, v.y);
+          mma_16816(acc[nt], a.z, b.z, a.w, b.w, v.z, v.w);
+        }
       }
     }
     // D fragment: rows g / g + 8 (gate rows e_a / e_b), columns 2 tq, 2 tq + 1
@@ -150,8 +185,12 @@ extern "C" int moe_q4_router(const void* x, const void* w, int T, int H, int E, 
   const long long want = (units + rt::kWarps - 1) / rt::kWarps;
   const int grid = (int)(want < 148 * 8 ? want : 148 * 8);
   float* dst = p.chunks > 1 ? reinterpret_cast<float*>(ws) : logits;
-  router_kernel<<<grid, rt::kThreads, 0, s>>>(static_cast<const uint16_t*>(x), static_cast<const uint16_t*>(w), T,
-                                               H, E, p, dst);
+  if (router_few(T, H))
+    router_kernel<true><<<grid, rt::kThreads, 0, s>>>(static_cast<const uint16_t*>(x),
+                                                       static_cast<const uint16_t*>(w), T, H, E, p, dst);
+  else
+    router_kernel<false><<<grid, rt::kThreads, 0, s>>>(static_cast<const uint16_t*>(x),
+                                                        static_cast<const uint16_t*>(w), T, H, E, p, dst);
   if (cudaGetLastError() != cudaSuccess) return MOE_Q4_ECUDA;
   if (p.chunks > 1) {
     const size_t n = (size_t)T * E;
