@@ -420,7 +420,9 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           break;
         }
         if (lane == 0) {
-          mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes + (GATEUP ? 1 : 2) * n_e * subs * 128);
+          // the codes' bytes; each activation copy adds its own below (the TMA
+          // needs only the expert, not its rows)
+          mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes);
           uint8_t* cdst = smem_raw + (code_base(s) - raw_s);
           tma_load_2d(cdst, &tm_wa, &full[s], st * row_bytes, wrow);
           if (GATEUP) tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
@@ -446,6 +448,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           // slot n at n * x_pitch (x_pitch = stage bytes + 16: 16-byte aligned,
           // and an odd number of 16-byte chunks spreads the slots over the banks)
           uint8_t* d = smem_raw + (Ls.x - raw_s) + (uint32_t)s * Geo::kXStage + (uint32_t)my_slot * Geo::kXPitch;
+          mbar_expect_tx(&full[s], (uint32_t)(subs * 128));
           bulk_load(d, my_src + st * subs * 64, (uint32_t)(subs * 128), &full[s]);
         }
         cp_async_arrive_noinc(&full[s]);
