@@ -12,8 +12,12 @@
 // over warps so that every SM streams part of the gate; the partial sums are
 // added afterwards in a fixed order, so the result does not depend on
 // scheduling.
+#include <cooperative_groups.h>
+
 #include "q4_api_internal.h"
 #include "q4_common.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace q4 {
 
@@ -58,8 +62,47 @@ static RouterPlan router_plan(int T, int H, int E) {
   return p;
 }
 
-// FEW: every unit takes exactly kFewSteps steps (plan.steps == kFewSteps).
-template <bool FEW>
+// One warp unit's loads and MMAs over `steps` 32-K steps from k_begin:
+// acc[nt] (16 gate rows x 8 tokens each) += w[rows] . x[tokens]^T.
+// FEW_STEPS > 0: exactly that many steps, all loads issued before the first
+// MMA, and only the first NT 8-token column tiles (the tokens present).
+template <int FEW_STEPS, int NT = rt::kNT>
+__device__ __forceinline__ void router_unit(const uint16_t* wa, const uint16_t* wb, const uint16_t* const xr[rt::kNT],
+                                            int k_begin, int k_end, float acc[rt::kNT][4]) {
+  if constexpr (FEW_STEPS > 0) {
+    uint4 a[FEW_STEPS], b[FEW_STEPS], v[FEW_STEPS][NT];
+#pragma unroll
+    for (int j = 0; j < FEW_STEPS; ++j) {
+      const int k = k_begin + j * rt::kKStep;
+      a[j] = ldg_nc(wa + k);
+      b[j] = ldg_nc(wb + k);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) v[j][nt] = ldg_nc(xr[nt] + k);
+    }
+#pragma unroll
+    for (int j = 0; j < FEW_STEPS; ++j)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma_16816(acc[nt], a[j].x, b[j].x, a[j].y, b[j].y, v[j][nt].x, v[j][nt].y);
+        mma_16816(acc[nt], a[j].z, b[j].z, a[j].w, b[j].w, v[j][nt].z, v[j][nt].w);
+      }
+  } else {
+#pragma unroll 4
+    for (int k = k_begin; k < k_end; k += rt::kKStep) {
+      const uint4 a = ldg_nc(wa + k), b = ldg_nc(wb + k);
+#pragma unroll
+      for (int nt = 0; nt < rt::kNT; ++nt) {
+        const uint4 v = ldg_nc(xr[nt] + k);
+        mma_16816(acc[nt], a.x, b.x, a.y, b.y, v.x, v.y);
+        mma_16816(acc[nt], a.z, b.z, a.w, b.w, v.z, v.w);
+      }
+    }
+  }
+}
+
+// General sizes: one warp per (gate tile, token tile, K chunk) unit; with
+// more than one chunk the partial sums go to the workspace for
+// router_reduce_kernel.
 __global__ void __launch_bounds__(rt::kThreads) router_kernel(const uint16_t* __restrict__ x,
                                                               const uint16_t* __restrict__ w, int T, int H, int E,
                                                               RouterPlan plan, float* __restrict__ out) {
@@ -89,37 +132,7 @@ __global__ void __launch_bounds__(rt::kThreads) router_kernel(const uint16_t* __
     for (int nt = 0; nt < rt::kNT; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
-    if constexpr (FEW) {
-      // all loads of the unit first, then the MMAs (one token tile: the x rows
-      // of the four column tiles repeat, so only distinct rows are loaded)
-      uint4 a[kFewSteps], b[kFewSteps], v[kFewSteps][rt::kNT];
-#pragma unroll
-      for (int j = 0; j < kFewSteps; ++j) {
-        const int k = k_begin + j * rt::kKStep;
-        a[j] = ldg_nc(wa + k);
-        b[j] = ldg_nc(wb + k);
-#pragma unroll
-        for (int nt = 0; nt < rt::kNT; ++nt) v[j][nt] = ldg_nc(xr[nt] + k);
-      }
-#pragma unroll
-      for (int j = 0; j < kFewSteps; ++j)
-#pragma unroll
-        for (int nt = 0; nt < rt::kNT; ++nt) {
-          mma_16816(acc[nt], a[j].x, b[j].x, a[j].y, b[j].y, v[j][nt].x, v[j][nt].y);
-          mma_16816(acc[nt], a[j].z, b[j].z, a[j].w, b[j].w, v[j][nt].z, v[j][nt].w);
-        }
-    } else {
-#pragma unroll 4
-      for (int k = k_begin; k < k_end; k += rt::kKStep) {
-        const uint4 a = ldg_nc(wa + k), b = ldg_nc(wb + k);
-#pragma unroll
-        for (int nt = 0; nt < rt::kNT; ++nt) {
-          const uint4 v = ldg_nc(xr[nt] + k);
-          mma_16816(acc[nt], a.x, b.x, a.y, b.y, v.x, v.y);
-          mma_16816(acc[nt], a.z, b.z, a.w, b.w, v.z, v.w);
-        }
-      }
-    }
+    router_unit<0>(wa, wb, xr, k_begin, k_end, acc);
     // D fragment: rows g / g + 8 (gate rows e_a / e_b), columns 2 tq, 2 tq + 1
     float* dst = out + (plan.chunks > 1 ? (size_t)c * TE : 0);
 #pragma unroll
@@ -131,6 +144,71 @@ __global__ void __launch_bounds__(rt::kThreads) router_kernel(const uint16_t* __
         if (t < T && e < E) dst[(size_t)t * E + e] = acc[nt][i];
       }
   }
+}
+
+// Decode sizes (one token tile, H a multiple of 32 kFewSteps): one kernel,
+// NT = ceil(T / 8) column tiles computed (the others stay zero).
+// A cluster of C CTAs owns one 16-row gate tile; warp w of cluster rank r
+// takes the K chunks w C + r, w C + r + 8 C, ...  Each CTA adds its warps'
+// partial tiles in warp order in shared memory; after a cluster barrier each
+// rank finishes 16 x 32 / C of the tile's logits, adding the C CTA sums in
+// rank order through distributed shared memory.  The order of every sum is
+// fixed by (H, C), so the result does not depend on scheduling.
+template <int NT>
+__global__ void __launch_bounds__(rt::kThreads, 1) router_few_kernel(const uint16_t* __restrict__ x,
+                                                                  const uint16_t* __restrict__ w, int T, int H, int E,
+                                                                  int chunks, float* __restrict__ logits) {
+  constexpr int kTile = rt::kRows * rt::kTokens;  // 512 logits: [gate row][token]
+  __shared__ float part[rt::kWarps][kTile];
+  __shared__ float cta_sum[kTile];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int C = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, tq = lane & 3;
+  const int et = blockIdx.x / C;
+  const int e_a = et * rt::kRows + g, e_b = e_a + 8;
+  const uint16_t* wa = w + (size_t)(e_a < E ? e_a : 0) * H + 8 * tq;
+  const uint16_t* wb = w + (size_t)(e_b < E ? e_b : 0) * H + 8 * tq;
+  const uint16_t* xr[rt::kNT];
+#pragma unroll
+  for (int nt = 0; nt < rt::kNT; ++nt) {
+    const int t = 8 * nt + g;
+    xr[nt] = x + (size_t)(t < T ? t : 0) * H + 8 * tq;
+  }
+  float acc[rt::kNT][4];
+#pragma unroll
+  for (int nt = 0; nt < rt::kNT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.0f;
+  for (int c = warp * C + rank; c < chunks; c += rt::kWarps * C) {
+    const int k0 = c * kFewSteps * rt::kKStep;
+    router_unit<kFewSteps, NT>(wa, wb, xr, k0, k0 + kFewSteps * rt::kKStep, acc);
+  }
+#pragma unroll
+  for (int nt = 0; nt < rt::kNT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int row = g + 8 * (i >> 1), t = 8 * nt + 2 * tq + (i & 1);
+      part[warp][row * rt::kTokens + t] = acc[nt][i];
+    }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kTile; i += rt::kThreads) {
+    float s = 0.0f;
+#pragma unroll
+    for (int q = 0; q < rt::kWarps; ++q) s += part[q][i];
+    cta_sum[i] = s;
+  }
+  cluster.sync();  // every CTA's sums are complete and visible cluster-wide
+  const int per_rank = kTile / C;
+  for (int i = rank * per_rank + threadIdx.x; i < (rank + 1) * per_rank; i += rt::kThreads) {
+    const int row = i / rt::kTokens, t = i % rt::kTokens;
+    const int e = et * rt::kRows + row;
+    float s = 0.0f;
+    for (int q = 0; q < C; ++q) s += *cluster.map_shared_rank(&cta_sum[i], q);
+    if (t < T && e < E) logits[(size_t)t * E + e] = s;
+  }
+  cluster.sync();  // no CTA leaves while another still reads its shared memory
 }
 
 // logits = the chunks' partial sums, added in a fixed order: one thread per
@@ -165,8 +243,16 @@ static bool router_args_ok(int T, int H, int E) {
          (long long)T * E < (1ll << 31);
 }
 
+// Cluster size of the decode-size kernel: the smallest of 1, 2, 4, 8 whose
+// 8 C warps cover the K chunks (8 at most; beyond that warps loop).
+static int router_few_cluster(int chunks) {
+  int c = 1;
+  while (c < 8 && rt::kWarps * c < chunks) c *= 2;
+  return c;
+}
+
 extern "C" size_t moe_q4_router_workspace(int T, int H, int E) {
-  if (!router_args_ok(T, H, E) || T == 0) return 0;
+  if (!router_args_ok(T, H, E) || T == 0 || router_few(T, H)) return 0;
   const RouterPlan p = router_plan(T, H, E);
   return p.chunks > 1 ? sizeof(float) * (size_t)p.chunks * T * E : 0;
 }
@@ -178,19 +264,41 @@ extern "C" int moe_q4_router(const void* x, const void* w, int T, int H, int E, 
   if (!x || !w || !logits) return MOE_Q4_EINVAL;
   if (((uintptr_t)x & 15) || ((uintptr_t)w & 15)) return MOE_Q4_EINVAL;
   const RouterPlan p = router_plan(T, H, E);
+  cudaStream_t s = (cudaStream_t)stream;
+  const uint16_t* xb = static_cast<const uint16_t*>(x);
+  const uint16_t* wb = static_cast<const uint16_t*>(w);
+  if (router_few(T, H)) {
+    const int C = router_few_cluster(p.chunks);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.e_tiles * C);
+    cfg.blockDim = dim3(rt::kThreads);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int nt = (T + 7) / 8;
+    cudaError_t e;
+    if (nt == 1)
+      e = cudaLaunchKernelEx(&cfg, router_few_kernel<1>, xb, wb, T, H, E, p.chunks, logits);
+    else if (nt == 2)
+      e = cudaLaunchKernelEx(&cfg, router_few_kernel<2>, xb, wb, T, H, E, p.chunks, logits);
+    else if (nt == 3)
+      e = cudaLaunchKernelEx(&cfg, router_few_kernel<3>, xb, wb, T, H, E, p.chunks, logits);
+    else
+      e = cudaLaunchKernelEx(&cfg, router_few_kernel<4>, xb, wb, T, H, E, p.chunks, logits);
+    return e == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
+  }
   const size_t need = moe_q4_router_workspace(T, H, E);
   if (need > 0 && (!ws || ws_bytes < need || ((uintptr_t)ws & 15))) return MOE_Q4_EWORKSPACE;
-  cudaStream_t s = (cudaStream_t)stream;
   const long long units = (long long)p.e_tiles * p.t_tiles * p.chunks;
   const long long want = (units + rt::kWarps - 1) / rt::kWarps;
   const int grid = (int)(want < 148 * 8 ? want : 148 * 8);
   float* dst = p.chunks > 1 ? reinterpret_cast<float*>(ws) : logits;
-  if (router_few(T, H))
-    router_kernel<true><<<grid, rt::kThreads, 0, s>>>(static_cast<const uint16_t*>(x),
-                                                       static_cast<const uint16_t*>(w), T, H, E, p, dst);
-  else
-    router_kernel<false><<<grid, rt::kThreads, 0, s>>>(static_cast<const uint16_t*>(x),
-                                                        static_cast<const uint16_t*>(w), T, H, E, p, dst);
+  router_kernel<<<grid, rt::kThreads, 0, s>>>(xb, wb, T, H, E, p, dst);
   if (cudaGetLastError() != cudaSuccess) return MOE_Q4_ECUDA;
   if (p.chunks > 1) {
     const size_t n = (size_t)T * E;

@@ -130,8 +130,9 @@ MOE_Q4_API int moe_q4_dequant(const uint8_t* weight, const uint8_t* weight_scale
  *   T >= 0; H > 0, H % 32 == 0; E > 0;
  *   logits    device, fp32 [T][E] (out): the input of moe_q4_forward;
  *   ws        device workspace of at least moe_q4_router_workspace(T, H, E)
- *             bytes (16-byte aligned; may be NULL when that is 0), owned by
- *             the call until the enqueued work completes;
+ *             bytes (16-byte aligned; may be NULL when that is 0, as it is
+ *             for T <= 32 with H % 128 == 0), owned by the call until the
+ *             enqueued work completes;
  *   ws_bytes  size of ws.
  * Returns MOE_Q4_EINVAL for bad sizes or pointers, MOE_Q4_EWORKSPACE for a
  * missing or short workspace; no host synchronisation, no allocation.

@@ -37,10 +37,12 @@ def _run_guarded(x, w):
     return out.view.cpu().numpy().astype(np.float64)
 
 
-# decode sizes (K split over warps), a ragged token count, prefill-like sizes,
-# E not a multiple of 16 and tiny H
-@pytest.mark.parametrize("T,H,E", [(1, 6144, 256), (5, 256, 8), (8, 6144, 256), (33, 512, 40),
-                                   (64, 6144, 256), (300, 256, 24), (1, 32, 1)])
+# decode sizes (K split over warps and, up to 32 tokens, over clusters of 1, 2,
+# 4 and 8 CTAs; H = 16384 has warps looping over chunks), a ragged token
+# count, prefill-like sizes, E not a multiple of 16 and tiny H
+@pytest.mark.parametrize("T,H,E", [(1, 6144, 256), (5, 256, 8), (8, 6144, 256), (32, 6144, 256), (33, 512, 40),
+                                   (64, 6144, 256), (300, 256, 24), (1, 32, 1), (2, 128, 17), (3, 1024, 33),
+                                   (7, 16384, 64), (4, 1536, 48), (6, 4096, 100)])
 def test_router_logits_within_summation_bound(T, H, E):
     x, w = _case(T, H, E, seed=T * 1000 + H + E)
     got = _run_guarded(x, w)
@@ -70,8 +72,9 @@ def test_router_rejects_bad_arguments():
     x, w = _case(2, 48, 8, seed=1)  # H % 32 != 0
     with pytest.raises(q4.MoeQ4Error):
         q4.router(x.cuda(), w.cuda())
-    x, w = _case(1, 6144, 256, seed=2)
-    assert q4.router_workspace(1, 6144, 256) > 0
+    assert q4.router_workspace(1, 6144, 256) == 0  # decode sizes: one kernel, no workspace
+    x, w = _case(64, 6144, 256, seed=2)
+    assert q4.router_workspace(64, 6144, 256) > 0
     with pytest.raises(q4.MoeQ4Error):
         q4.router(x.cuda(), w.cuda(), ws=torch.empty(16, dtype=torch.uint8, device="cuda"))
 
