@@ -106,12 +106,12 @@ Layout layout(const moe_q4_layer* L, int T, int k) {
   }
   const int max_exp = (int)(R < (size_t)L->E ? R : (size_t)L->E);
   o.dk_units_gu = max_exp * (L->I / 128);
-  o.dk_units_dn = max_exp * (L->H / 128);
+  o.dk_units_dn = max_exp * ((L->H + 255) / 256);  // down units: two 128-row tiles
   o.n_max = T < 16 ? T : 16;
   o.dk_counter = p;
   p = align_up(p + sizeof(int32_t) * (size_t)(o.dk_units_gu + o.dk_units_dn) * kDkSlabs);
   o.dk_partial = p;
-  p = align_up(p + sizeof(float) * (size_t)2 * kDkMaxGrid * 3 * o.n_max * 128);
+  p = align_up(p + sizeof(float) * (size_t)2 * kDkMaxGrid * 4 * o.n_max * 128);  // 2 tiles per unit, both kernels
   o.end = p;
   return o;
 }

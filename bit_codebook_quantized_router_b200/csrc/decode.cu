@@ -7,8 +7,10 @@
 // ("Round 7 -- Rewrite the GLM-5.2 routed-expert encoder", "Owner-locked
 // decisions" 4 and 6.)
 //
-// * Work split.  A unit is (expert on this path, tile of 128 weight rows);
-//   the units' stages (256 weights of K each, 128 if K % 256 != 0) form one
+// * Work split.  A unit is (expert on this path, 128 weight rows of gate and
+//   of up, or 256 rows of down as two 128-row tiles), so a stage carries 256
+//   rows of codes in both kernels and the fixed cost of a stage (barriers,
+//   activation and scale reads) is spread over the same bytes; the units' stages (256 weights of K each, 128 if K % 256 != 0) form one
 //   sequence that the persistent CTAs (one per SM) cut into equal contiguous
 //   ranges, so every SM streams the same number of bytes.  A tile whose K
 //   range spans several CTAs is finished by the last of them to arrive (a
@@ -72,7 +74,11 @@ constexpr uint32_t kBarBytes = 1024;   // barriers and flags
 
 template <bool GATEUP, int NT>
 struct DkCfg {
-  static constexpr int kMats = GATEUP ? 2 : 1;
+  // two 128-row weight tiles per unit and stage: gate and up of the same rows
+  // (gate/up), or two consecutive row tiles of the down matrix (down), so a
+  // stage carries 256 rows of codes either way
+  static constexpr int kMats = 2;
+  static constexpr int kUnitRows = GATEUP ? dk::kRows : 2 * dk::kRows;  // output rows per unit
   // activation row slots of a stage: 8 per n-tile; slot 8 nt + c feeds column
   // c of n-tile nt.  Gate/up: x of the expert's row n at slot n.  Down: h of
   // row n at slot n and h_lo of row n at slot kLoSlot + n (NT = 1: h in
@@ -153,7 +159,7 @@ static bool dk_layout(uint32_t raw, uint32_t limit, uint32_t code_stage, uint32_
 
 struct DkParams {
   FwdArgs a;
-  int tiles_per_e;  // weight rows / 128
+  int tiles_per_e;  // units per expert: I / 128 (gate/up), ceil(H / 256) (down)
   int subs;         // 64-K super-steps per stage: 4 (K % 256 == 0) or 2
   int stages;       // stages per tile: K / (64 * subs)
   int ring;         // shared-memory stages
@@ -392,7 +398,9 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       const int seg_end = min(k1, (unit + 1) * P.stages);
       const int e = a.dec_list[unit / P.tiles_per_e];
       const int t = unit % P.tiles_per_e;
-      const int wrow = e * rows_total + t * dk::kRows;
+      const int wrow = e * rows_total + t * C::kUnitRows;
+      // down: the unit's second row tile exists unless H is an odd number of 128s
+      const bool two = GATEUP || t * C::kUnitRows + dk::kRows < rows_total;
       const int row0 = a.offsets[e];
       // Activation rows by untiled bulk copies (a tiled TMA would need a
       // 128-byte-aligned destination), one per row and stage: the stage's
@@ -422,17 +430,22 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
         if (lane == 0) {
           // the codes' bytes; each activation copy adds its own below (the TMA
           // needs only the expert, not its rows)
-          mbar_arrive_expect_tx(&full[s], kMats * dk::kRows * row_bytes);
+          mbar_arrive_expect_tx(&full[s], (two ? 2 : 1) * dk::kRows * row_bytes);
           uint8_t* cdst = smem_raw + (code_base(s) - raw_s);
           tma_load_2d(cdst, &tm_wa, &full[s], st * row_bytes, wrow);
-          if (GATEUP) tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
+          if (GATEUP)
+            tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
+          else if (two)
+            tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wa, &full[s], st * row_bytes, wrow + dk::kRows);
         }
         __syncwarp();  // the expected bytes are registered before any row copy can land
         // scale bytes of the stage (2 per 64-K super-step) for 4 rows per lane
 #pragma unroll
         for (int m = 0; m < kMats; ++m) {
-          const uint8_t* sbase = (GATEUP ? (m ? a.up_s : a.gate_s) : a.down_s) + (size_t)wrow * (K / 32) +
-                                 (size_t)st * 2 * subs;
+          if (!two && m == 1) break;  // (a missing tile's rows are computed on stale bytes, never written)
+          const uint8_t* sbase = GATEUP ? (m ? a.up_s : a.gate_s) + (size_t)wrow * (K / 32) + (size_t)st * 2 * subs
+                                        : a.down_s + (size_t)(wrow + m * dk::kRows) * (K / 32) +
+                                              (size_t)st * 2 * subs;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int r = lane + 32 * j;
@@ -654,7 +667,9 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       if (!GATEUP && NT == 1) {
         // columns 4..7 hold W h_lo for tokens 0..3: add them to columns 0..3
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[0][0][i] += __shfl_xor_sync(0xffffffffu, acc[0][0][i], 2);
+        for (int m = 0; m < kMats; ++m)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[m][0][i] += __shfl_xor_sync(0xffffffffu, acc[m][0][i], 2);
       }
 
       // ---- the warp finishes its rows: token n = 8 tt + 2 tq + (i & 1), row r0 / r1 ----
@@ -718,14 +733,15 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           const int n = 8 * tt + 2 * tq + (i & 1);
           if (n >= n_e) continue;
           const size_t row = (size_t)row0 + n;
-          const int wr = tile * dk::kRows + ((i >> 1) ? r1 : r0);
+          const int wr = tile * C::kUnitRows + ((i >> 1) ? r1 : r0);
           if (GATEUP) {
-            const float hv = silu_mul(acc[0][tt][i], acc[kMats - 1][tt][i]);
+            const float hv = silu_mul(acc[0][tt][i], acc[1][tt][i]);
             const __nv_bfloat16 hb = __float2bfloat16_rn(hv);
             a.h[row * a.I + wr] = hb;
             a.h_lo[row * a.I + wr] = __float2bfloat16_rn(hv - __bfloat162float(hb));
           } else {
             a.y[row * a.H + wr] = acc[0][tt][i];
+            if (wr + dk::kRows < a.H) a.y[row * a.H + wr + dk::kRows] = acc[1][tt][i];
           }
         }
       g = seg_end;
@@ -787,7 +803,7 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   DkParams P;
   P.a = a;
   const int K = GATEUP ? a.H : a.I;
-  P.tiles_per_e = (GATEUP ? a.I : a.H) / dk::kRows;
+  P.tiles_per_e = GATEUP ? a.I / dk::kRows : (a.H + C::kUnitRows - 1) / C::kUnitRows;
   P.subs = SUBS;
   P.stages = K / (64 * P.subs);
   // stage indices are 32-bit on the device
