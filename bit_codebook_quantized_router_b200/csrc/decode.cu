@@ -167,6 +167,7 @@ struct DkParams {
   int n_max;        // token columns kept in partial sums: min(16, T)
   float* partial;   // [2 * gridDim.x][mats][n_max][128]
   int32_t* counter; // [units][8 slabs], zero at launch
+  int self_k;       // gate/up at T = 1: top-k (the producer routes the token itself), else 0
 };
 
 // Start of CTA b's range of stages (the host keeps total below 2^31).
@@ -374,17 +375,97 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   if (tp.n == 1 && warp >= 1) build_lut_slot(lut, tp.t[0], 0, threadIdx.x - 32);
   __syncthreads();
 
-  // down: the next kernel (the combine, small CTAs that fit beside this one)
-  // may be scheduled now; its own wait still covers all of this kernel's work
-  if (!GATEUP) pdl_trigger();
-  pdl_wait();
-  const int n_dec = a.hdr[kNumDecode];
   const int rows_total = GATEUP ? a.I : a.H;
   const int K = GATEUP ? a.H : a.I;
   constexpr int subs = SUBS;
   constexpr int row_bytes = 32 * subs;  // code bytes per row per stage
-  const int total = n_dec * P.tiles_per_e * P.stages;
   const int G = gridDim.x, b = blockIdx.x;
+
+  // producer: one ring stage s of stage index st of a unit whose weight rows
+  // start at wrow: the codes (one TMA per 128-row tile, lane 0 registering
+  // their bytes), every row's scale bytes (cp.async, 4 rows per lane), this
+  // lane's activation row (untiled bulk copy, adding its own bytes) and the
+  // lanes' cp.async arrivals
+  const auto issue_stage = [&](int s, int st, int wrow, bool two, int my_slot, const __nv_bfloat16* my_src) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&full[s], (two ? 2 : 1) * dk::kRows * row_bytes);
+      uint8_t* cdst = smem_raw + (code_base(s) - raw_s);
+      tma_load_2d(cdst, &tm_wa, &full[s], st * row_bytes, wrow);
+      if (GATEUP)
+        tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
+      else if (two)
+        tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wa, &full[s], st * row_bytes, wrow + dk::kRows);
+    }
+    __syncwarp();  // the expected bytes are registered before any row copy can land
+    // scale bytes of the stage (2 per 64-K super-step) for 4 rows per lane
+#pragma unroll
+    for (int m = 0; m < kMats; ++m) {
+      if (!two && m == 1) break;  // (a missing tile's rows are computed on stale bytes, never written)
+      const uint8_t* sbase = GATEUP ? (m ? a.up_s : a.gate_s) + (size_t)wrow * (K / 32) + (size_t)st * 2 * subs
+                                    : a.down_s + (size_t)(wrow + m * dk::kRows) * (K / 32) + (size_t)st * 2 * subs;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int r = lane + 32 * j;
+        const uint32_t dst =
+            Ls.scales + (uint32_t)s * Geo::kScaleStage + (uint32_t)(m * dk::kRows + r) * Geo::kScaleSlot;
+        if constexpr (subs == 4)
+          cp_async_small<8>(dst, sbase + (size_t)r * (K / 32));
+        else
+          cp_async_small<4>(dst, sbase + (size_t)r * (K / 32));
+      }
+    }
+    if (my_slot >= 0) {
+      // slot n at n * x_pitch (x_pitch = stage bytes + 16: 16-byte aligned,
+      // and an odd number of 16-byte chunks spreads the slots over the banks)
+      uint8_t* d = smem_raw + (Ls.x - raw_s) + (uint32_t)s * Geo::kXStage + (uint32_t)my_slot * Geo::kXPitch;
+      mbar_expect_tx(&full[s], (uint32_t)(subs * 128));
+      bulk_load(d, my_src + st * subs * 64, (uint32_t)(subs * 128), &full[s]);
+    }
+    cp_async_arrive_noinc(&full[s]);
+    __syncwarp();
+  };
+
+  // Gate/up with one token (self_k > 0): its k experts are distinct and hold
+  // one row each, so the routing tables follow from the token's top-k alone
+  // (the expert list is the k ids in ascending order; expert j of it has row
+  // j, of token 0).  Warp 0 computes that top-k with the routing kernel's own
+  // warp routine on the same logits (hence the same ids) and the CTA runs on
+  // it without waiting for the routing kernel.  That kernel lets this one
+  // launch only after its own wait, so x and the logits are complete.  What
+  // this kernel does need of it, the split-tile counters it zeroes, is used
+  // only after a wait at the end of each unit; every thread waits again
+  // before it exits, so the kernels after this one still find the routing
+  // kernel complete.
+  const bool self = GATEUP && P.self_k > 0;
+  int* self_e = reinterpret_cast<int*>(bars) + 64;  // [k] expert list (bytes 256.. of the barrier block)
+  if (self) {
+    if (warp == 0) {
+      const int k = P.self_k;
+      int id;
+      float wt;
+      topk_warp(a.logits, a.E, k, lane, nullptr, id, wt);
+      int rank = 0;  // lane j < k: number of smaller ids among the k
+      for (int j = 0; j < k; ++j) {
+        const int o = __shfl_sync(0xffffffffu, id, j);
+        rank += (lane < k && o < id) ? 1 : 0;
+      }
+      if (lane < k) self_e[rank] = id;
+    }
+    __syncthreads();
+  }
+  // routing tables of a unit: expert, its first row, its rows
+  const auto unit_expert = [&](int unit) -> int {
+    return self ? self_e[unit / P.tiles_per_e] : a.dec_list[unit / P.tiles_per_e];
+  };
+  const auto expert_row0 = [&](int unit, int e) -> int { return self ? unit / P.tiles_per_e : a.offsets[e]; };
+  const auto expert_rows = [&](int e) -> int { return self ? 1 : a.counts[e]; };
+
+  // down: the next kernel (the combine, small CTAs that fit beside this one)
+  // may be scheduled now; its own wait still covers all of this kernel's work
+  if (!GATEUP) pdl_trigger();
+  if (!self) pdl_wait();
+  const int n_dec = self ? P.self_k : a.hdr[kNumDecode];
+  const int total = n_dec * P.tiles_per_e * P.stages;
   const int k0 = dk_range(b, total, G), k1 = dk_range(b + 1, total, G);
 
   if (warp == 0) {
@@ -396,24 +477,24 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       const int unit = g / P.stages;
       const int st0 = g - unit * P.stages;
       const int seg_end = min(k1, (unit + 1) * P.stages);
-      const int e = a.dec_list[unit / P.tiles_per_e];
+      const int e = unit_expert(unit);
       const int t = unit % P.tiles_per_e;
       const int wrow = e * rows_total + t * C::kUnitRows;
       // down: the unit's second row tile exists unless H is an odd number of 128s
       const bool two = GATEUP || t * C::kUnitRows + dk::kRows < rows_total;
-      const int row0 = a.offsets[e];
+      const int row0 = expert_row0(unit, e);
       // Activation rows by untiled bulk copies (a tiled TMA would need a
       // 128-byte-aligned destination), one per row and stage: the stage's
       // 32 * subs * 4 bytes of x[token] (gate/up, lane n: row n) or of h / h_lo
       // (down, lane n: h of row n; lane 16 + n: h_lo of row n).  Slots past
       // n_e are not written: they only feed columns nobody writes.
-      const int n_e = a.counts[e];  // <= 16
+      const int n_e = expert_rows(e);  // <= 16
       int my_slot = -1;
       const __nv_bfloat16* my_src = nullptr;
       if (GATEUP) {
         if (lane < n_e) {
           my_slot = lane;
-          my_src = a.x + (size_t)a.row_token[row0 + lane] * a.H;
+          my_src = a.x + (self ? (size_t)0 : (size_t)a.row_token[row0 + lane] * a.H);
         }
       } else {
         const int n = lane & 15;
@@ -427,45 +508,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           ok = false;
           break;
         }
-        if (lane == 0) {
-          // the codes' bytes; each activation copy adds its own below (the TMA
-          // needs only the expert, not its rows)
-          mbar_arrive_expect_tx(&full[s], (two ? 2 : 1) * dk::kRows * row_bytes);
-          uint8_t* cdst = smem_raw + (code_base(s) - raw_s);
-          tma_load_2d(cdst, &tm_wa, &full[s], st * row_bytes, wrow);
-          if (GATEUP)
-            tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wb, &full[s], st * row_bytes, wrow);
-          else if (two)
-            tma_load_2d(cdst + dk::kRows * row_bytes, &tm_wa, &full[s], st * row_bytes, wrow + dk::kRows);
-        }
-        __syncwarp();  // the expected bytes are registered before any row copy can land
-        // scale bytes of the stage (2 per 64-K super-step) for 4 rows per lane
-#pragma unroll
-        for (int m = 0; m < kMats; ++m) {
-          if (!two && m == 1) break;  // (a missing tile's rows are computed on stale bytes, never written)
-          const uint8_t* sbase = GATEUP ? (m ? a.up_s : a.gate_s) + (size_t)wrow * (K / 32) + (size_t)st * 2 * subs
-                                        : a.down_s + (size_t)(wrow + m * dk::kRows) * (K / 32) +
-                                              (size_t)st * 2 * subs;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int r = lane + 32 * j;
-            const uint32_t dst =
-                Ls.scales + (uint32_t)s * Geo::kScaleStage + (uint32_t)(m * dk::kRows + r) * Geo::kScaleSlot;
-            if constexpr (subs == 4)
-              cp_async_small<8>(dst, sbase + (size_t)r * (K / 32));
-            else
-              cp_async_small<4>(dst, sbase + (size_t)r * (K / 32));
-          }
-        }
-        if (my_slot >= 0) {
-          // slot n at n * x_pitch (x_pitch = stage bytes + 16: 16-byte aligned,
-          // and an odd number of 16-byte chunks spreads the slots over the banks)
-          uint8_t* d = smem_raw + (Ls.x - raw_s) + (uint32_t)s * Geo::kXStage + (uint32_t)my_slot * Geo::kXPitch;
-          mbar_expect_tx(&full[s], (uint32_t)(subs * 128));
-          bulk_load(d, my_src + st * subs * 64, (uint32_t)(subs * 128), &full[s]);
-        }
-        cp_async_arrive_noinc(&full[s]);
-        __syncwarp();
+        issue_stage(s, st, wrow, two, my_slot, my_src);
         ring_next(s, ph, ring);
       }
       g = seg_end;
@@ -534,7 +577,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       const int ustart = unit * P.stages, uend = ustart + P.stages;
       const int seg_end = min(k1, uend);
       const int nst = (int)(seg_end - g);
-      const int e = a.dec_list[unit / P.tiles_per_e];
+      const int e = unit_expert(unit);
       const int tile = unit % P.tiles_per_e;
       const int tid = tp.id[e];
       int slot = tid == slot_tab0 ? 0 : (tid == slot_tab1 ? 1 : -1);
@@ -562,7 +605,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       // activation slot of this lane's column gq in each n-tile; columns of
       // absent tokens are not read (zero operands; their MMA columns are never
       // written)
-      const int n_e_seg = a.counts[e];
+      const int n_e_seg = expert_rows(e);
       uint32_t xrow[NT], col_ok[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -673,7 +716,8 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       }
 
       // ---- the warp finishes its rows: token n = 8 tt + 2 tq + (i & 1), row r0 / r1 ----
-      const int row0 = a.offsets[e], n_e = a.counts[e];
+      if (self) pdl_wait();  // (the routing kernel zeroed the split-tile counters; returns at once after the first)
+      const int row0 = expert_row0(unit, e), n_e = expert_rows(e);
       const bool final_here = (g == ustart && seg_end == uend);
       if (!final_here) {
         // partial: slot 2b (segment starts this CTA's range) or 2b+1 (its last)
@@ -749,6 +793,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   }
 
   // ------------------------------ teardown ------------------------------
+  if (self) pdl_wait();  // the routing kernel is complete before this CTA is (and its status reset precedes ours)
   __syncthreads();
   if (threadIdx.x == 0 && *abort_flag) record_error(a.hdr + kStatus, MOE_Q4_ETIMEOUT);
   if (warp == 0 && *abort_flag) {
@@ -812,6 +857,7 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   using Geo = typename C::template Geom<SUBS>;
   P.partial = partial;
   P.counter = counter;
+  P.self_k = GATEUP && a.T == 1 ? a.k : 0;
 
   // deepest ring that fits; the dynamic window starts after the reserved bytes
   // (the kernel has no static shared memory)
@@ -849,7 +895,9 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  // one token: the routing kernel (one CTA) still runs while this kernel
+  // starts, so this kernel leaves it its SM rather than have one CTA start late
+  cfg.gridDim = dim3(P.self_k > 0 && grid > 1 ? grid - 1 : grid);
   cfg.blockDim = dim3(dk::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;

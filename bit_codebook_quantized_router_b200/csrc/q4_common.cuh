@@ -8,6 +8,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
 #include "moe_q4.h"
@@ -148,6 +149,67 @@ __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f +
 // a few ulp of fp32, far below the bf16 rounding of h that follows.
 __device__ __forceinline__ float silu_mul_fast(float g, float u) {
   return g * u * __fdividef(1.0f, 1.0f + __expf(-g));
+}
+
+constexpr int kMaxLogitsPerLane = kMaxExperts / 32;
+
+// One warp routes one token: lane l holds logits of experts l, l+32, ...
+// Each of the k rounds takes the best remaining (value, then lower id) by a
+// warp argmax; lane j ends up holding slot j.  Non-finite logits are
+// treated as -inf and recorded as a device error (unless status is null).
+__device__ __forceinline__ void topk_warp(const float* __restrict__ row, int E, int k, int lane,
+                                          int32_t* status, int& my_id, float& my_w) {
+  float v[kMaxLogitsPerLane];
+  uint32_t avail = 0;
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < kMaxLogitsPerLane; ++i) {
+    const int id = lane + 32 * i;
+    v[i] = -INFINITY;
+    if (id < E) {
+      float x = row[id];
+      if (!isfinite(x)) {
+        bad = true;
+        x = -INFINITY;
+      }
+      v[i] = x;
+      avail |= 1u << i;
+    }
+  }
+  if (__any_sync(0xffffffffu, bad) && lane == 0 && status) record_error(status, MOE_Q4_EDEVICE);
+  float mine = -INFINITY;
+  my_id = -1;
+  for (int j = 0; j < k; ++j) {
+    float bv = -INFINITY;
+    int bi = -1;
+#pragma unroll
+    for (int i = 0; i < kMaxLogitsPerLane; ++i)
+      if (((avail >> i) & 1u) && (bi < 0 || v[i] > bv)) {
+        bv = v[i];
+        bi = i;
+      }
+    int bid = bi < 0 ? 0x7fffffff : lane + 32 * bi;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
+      if (ov > bv || (ov == bv && oid < bid)) {
+        bv = ov;
+        bid = oid;
+      }
+    }
+    if ((bid & 31) == lane) avail &= ~(1u << (bid >> 5));
+    if (lane == j) {
+      my_id = bid;
+      mine = bv;
+    }
+  }
+  const float m = __shfl_sync(0xffffffffu, mine, 0);
+  float ex = (lane < k) ? expf(mine - m) : 0.0f;
+  float sum = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+  my_w = ex / sum;
 }
 
 // Programmatic dependent launch: wait for the previous kernel's results /

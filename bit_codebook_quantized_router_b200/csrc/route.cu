@@ -17,66 +17,6 @@ namespace q4 {
 constexpr int kRouteThreads = 1024;
 constexpr int kRouteWarps = kRouteThreads / 32;
 constexpr int kFusedMaxT = 256;  // above this, top-k runs on many CTAs first
-constexpr int kMaxLogitsPerLane = kMaxExperts / 32;
-
-// One warp routes one token: lane l holds logits of experts l, l+32, ...
-// Each of the k rounds takes the best remaining (value, then lower id) by a
-// warp argmax; lane j ends up holding slot j.  Non-finite logits are
-// recorded as a device error and treated as -inf.
-__device__ __forceinline__ void topk_warp(const float* __restrict__ row, int E, int k, int lane,
-                                          int32_t* status, int& my_id, float& my_w) {
-  float v[kMaxLogitsPerLane];
-  uint32_t avail = 0;
-  bool bad = false;
-#pragma unroll
-  for (int i = 0; i < kMaxLogitsPerLane; ++i) {
-    const int id = lane + 32 * i;
-    v[i] = -INFINITY;
-    if (id < E) {
-      float x = row[id];
-      if (!isfinite(x)) {
-        bad = true;
-        x = -INFINITY;
-      }
-      v[i] = x;
-      avail |= 1u << i;
-    }
-  }
-  if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(status, MOE_Q4_EDEVICE);
-  float mine = -INFINITY;
-  my_id = -1;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = -1;
-#pragma unroll
-    for (int i = 0; i < kMaxLogitsPerLane; ++i)
-      if (((avail >> i) & 1u) && (bi < 0 || v[i] > bv)) {
-        bv = v[i];
-        bi = i;
-      }
-    int bid = bi < 0 ? 0x7fffffff : lane + 32 * bi;
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oid = __shfl_xor_sync(0xffffffffu, bid, off);
-      if (ov > bv || (ov == bv && oid < bid)) {
-        bv = ov;
-        bid = oid;
-      }
-    }
-    if ((bid & 31) == lane) avail &= ~(1u << (bid >> 5));
-    if (lane == j) {
-      my_id = bid;
-      mine = bv;
-    }
-  }
-  const float m = __shfl_sync(0xffffffffu, mine, 0);
-  float ex = (lane < k) ? expf(mine - m) : 0.0f;
-  float sum = ex;
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-  my_w = ex / sum;
-}
 
 __device__ __forceinline__ void store_route(const FwdArgs& a, int t, int lane, int id, float w) {
   if (lane < a.k) {
@@ -229,8 +169,11 @@ __global__ void __launch_bounds__(kRouteThreads) route_fused_kernel(const __grid
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int e = tid; e < E; e += kRouteThreads) counts[e] = 0;
   for (int i = tid; i < E * W; i += kRouteThreads) tokmask[i] = 0u;
-  pdl_trigger();  // scheduling only: the next kernel's wait covers this one
   pdl_wait();
+  // The next kernel may be scheduled now.  Its own wait still covers this
+  // kernel's results; what it reads before that wait (the layer's inputs x
+  // and logits, the weights) is complete once this kernel's wait returned.
+  pdl_trigger();
   if (tid == 0) a.hdr[kStatus] = MOE_Q4_OK;
   // per-tile arrival counters of the small-M kernels start at zero every call
   for (int i = tid; i < a.dk_counter_n; i += kRouteThreads) a.dk_counter[i] = 0;
