@@ -150,9 +150,9 @@ __global__ void __launch_bounds__(rt::kThreads) router_kernel(const uint16_t* __
 // NT = ceil(T / 8) column tiles computed (the others stay zero).
 // A cluster of C CTAs owns one 16-row gate tile; warp w of cluster rank r
 // takes the K chunks w C + r, w C + r + 8 C, ...  Each CTA adds its warps'
-// partial tiles in warp order in shared memory; after a cluster barrier each
-// rank finishes 16 x 32 / C of the tile's logits, adding the C CTA sums in
-// rank order through distributed shared memory.  The order of every sum is
+// partial tiles in warp order in shared memory; after a cluster barrier rank
+// r finishes logits [r 512 / C, (r + 1) 512 / C) of the tile's 16 x 32,
+// adding the C CTA sums in rank order through distributed shared memory.  The order of every sum is
 // fixed by (H, C), so the result does not depend on scheduling.
 template <int NT>
 __global__ void __launch_bounds__(rt::kThreads, 1) router_few_kernel(const uint16_t* __restrict__ x,
@@ -200,8 +200,8 @@ __global__ void __launch_bounds__(rt::kThreads, 1) router_few_kernel(const uint1
     cta_sum[i] = s;
   }
   cluster.sync();  // every CTA's sums are complete and visible cluster-wide
-  const int per_rank = kTile / C;
-  for (int i = rank * per_rank + threadIdx.x; i < (rank + 1) * per_rank; i += rt::kThreads) {
+  const int lo = rank * kTile / C, hi = (rank + 1) * kTile / C;
+  for (int i = lo + threadIdx.x; i < hi; i += rt::kThreads) {
     const int row = i / rt::kTokens, t = i % rt::kTokens;
     const int e = et * rt::kRows + row;
     float s = 0.0f;
@@ -243,12 +243,14 @@ static bool router_args_ok(int T, int H, int E) {
          (long long)T * E < (1ll << 31);
 }
 
-// Cluster size of the decode-size kernel: the smallest of 1, 2, 4, 8 whose
-// 8 C warps cover the K chunks (8 at most; beyond that warps loop).
+// Cluster size of the decode-size kernel: just enough CTAs for one K chunk
+// per warp (8 at most, the portable limit; beyond that warps loop).  Sizes
+// that are not powers of two keep the cluster count of a 256-expert gate
+// (16 clusters) within what the GPU holds at once: clusters of 8 fit only 15
+// times on 148 SMs, and a 16th would run as a second wave.
 static int router_few_cluster(int chunks) {
-  int c = 1;
-  while (c < 8 && rt::kWarps * c < chunks) c *= 2;
-  return c;
+  const int c = (chunks + rt::kWarps - 1) / rt::kWarps;
+  return c < 1 ? 1 : (c > 8 ? 8 : c);
 }
 
 extern "C" size_t moe_q4_router_workspace(int T, int H, int E) {

@@ -97,6 +97,39 @@ def test_layer_k_not_multiple_of_256(T, k):
     gpu_support.check_out(out, ref, f"H=I=384 T={T} k={k}")
 
 
+# One token: the small-M gate/up kernel routes the token itself (the routing
+# kernel's warp top-k on the same logits) and starts before the routing kernel
+# ends.  Equal logits (lower id first), a tie at the k-th place and top-k ids
+# in descending id order must still select and order the oracle's experts.
+@pytest.mark.parametrize("case", ["ties", "tie_at_k", "descending_ids"])
+def test_one_token_self_routing(case):
+    w = inputs.Workload("one", 12, 1, inputs.TINY)
+    L, dev = _small_device_layer(w)
+    x = inputs.activations(w)
+    lg = inputs.router_logits(w)
+    k = 3
+    if case == "ties":
+        lg[0, :] = torch.tensor([2.0, 3.0, 3.0, 1.0, 3.0, 0.5, 3.0, -1.0])
+    elif case == "tie_at_k":
+        lg[0, :] = torch.tensor([1.0, 4.0, 2.0, 2.0, 0.0, 5.0, 2.0, 2.0])
+    else:
+        lg[0, :] = torch.arange(8, dtype=torch.float32)
+    out, ids, _, _ = _run(dev, x.cuda(), lg.cuda(), k)
+    ref, rids, _ = oracle.moe_tokens(L, inputs.bf16_bits(x), lg.numpy(), k, return_routing=True)
+    assert np.array_equal(ids.cpu().numpy(), rids)
+    gpu_support.check_out(out, ref, f"one token, {case}")
+
+
+def test_one_token_non_finite_logit_reports_device_status():
+    w = inputs.Workload("one_nan", 13, 1, inputs.TINY)
+    _, dev = _small_device_layer(w)
+    lg = inputs.router_logits(w).cuda()
+    lg[0, 3] = float("nan")
+    ws = q4.alloc_workspace(q4.forward_workspace(dev, 1, 2))
+    q4.forward(dev, inputs.activations(w).cuda(), lg, 2, ws=ws)
+    assert q4.forward_status(ws) == q4._lib.EDEVICE
+
+
 def test_identical_experts_equal_dense_ffn():
     w = inputs.Workload("ident", 8, 24, inputs.TINY)
     L, dev = _small_device_layer(w, identical_to=2)

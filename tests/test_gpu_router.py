@@ -37,12 +37,13 @@ def _run_guarded(x, w):
     return out.view.cpu().numpy().astype(np.float64)
 
 
-# decode sizes (K split over warps and, up to 32 tokens, over clusters of 1, 2,
-# 4 and 8 CTAs; H = 16384 has warps looping over chunks), a ragged token
-# count, prefill-like sizes, E not a multiple of 16 and tiny H
+# decode sizes (K split over warps and, up to 32 tokens, over clusters of 1 to
+# 8 CTAs, 3, 5, 6 and 7 among them; H = 16384 has warps looping over chunks),
+# a ragged token count, prefill-like sizes, E not a multiple of 16 and tiny H
 @pytest.mark.parametrize("T,H,E", [(1, 6144, 256), (5, 256, 8), (8, 6144, 256), (32, 6144, 256), (33, 512, 40),
                                    (64, 6144, 256), (300, 256, 24), (1, 32, 1), (2, 128, 17), (3, 1024, 33),
-                                   (7, 16384, 64), (4, 1536, 48), (6, 4096, 100)])
+                                   (7, 16384, 64), (4, 1536, 48), (6, 4096, 100),
+                                   (2, 2560, 64), (3, 5120, 40), (1, 7168, 160)])
 def test_router_logits_within_summation_bound(T, H, E):
     x, w = _case(T, H, E, seed=T * 1000 + H + E)
     got = _run_guarded(x, w)
