@@ -81,10 +81,14 @@ def load_peaks():
 
 
 def source_digest(files) -> str:
+    """Digest of the kernel sources as compiled: line comments and blank lines
+    do not count, so a comment edit keeps a profile's figures valid."""
+    import re
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            text = re.sub(r"//[^\n]*", "", fh.read())
+        h.update("\n".join(ln.rstrip() for ln in text.splitlines() if ln.strip()).encode())
     return h.hexdigest()[:16]
 
 

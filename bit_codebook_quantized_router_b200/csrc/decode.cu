@@ -16,13 +16,13 @@
 //   range spans several CTAs is finished by the last of them to arrive (a
 //   per-tile counter): it adds the partial sums in K order (deterministic)
 //   and writes the result.
-// * Data movement (warp 0): per stage and matrix one TMA brings 128 weight
-//   rows x 128 bytes of codes (a full 128-byte line per row: narrower boxes
-//   stream at a fraction of HBM bandwidth) with the 128-byte swizzle; the
-//   warp's lanes copy each row's scale bytes for the stage and (gate/up) the
-//   expert's activation rows, straight from x through the row -> token map,
-//   with cp.async, completing on the stage barrier; the down projection's h
-//   rows come by TMA.
+// * Data movement (warp 0): per stage and 128-row tile one TMA brings 128
+//   weight rows x 128 bytes of codes (a full 128-byte line per row: narrower
+//   boxes stream at a fraction of HBM bandwidth) with the 128-byte swizzle;
+//   the warp's lanes copy each row's scale bytes for the stage with cp.async
+//   and the expert's activation rows (x through the row -> token map for
+//   gate/up, h and h_lo for down) by untiled bulk copies, all completing on
+//   the stage barrier.
 // * Decode + MMA (warps 1..8): warp s owns weight rows 16s..16s+15 of the
 //   tile.  In each 128-K half of a stage, lane (g, t) reads the 16-byte code
 //   chunk t of rows g and g+8 (32 weights, one E8M0 block), decodes it to bf16 pairs ("aidendle94/GLM-5.2-NF4-Lloyd-
