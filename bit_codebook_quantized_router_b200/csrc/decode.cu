@@ -370,6 +370,31 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     prefetch_tmap(&tm_wa);
     if (GATEUP) prefetch_tmap(&tm_wb);
   }
+  // Gate/up with one token (self_k > 0): its k experts are distinct and hold
+  // one row each, so the routing tables follow from the token's top-k alone
+  // (the expert list is the k ids in ascending order; expert j of it has row
+  // j, of token 0).  Warp 0 computes that top-k with the routing kernel's own
+  // warp routine on the same logits (hence the same ids) and the CTA runs on
+  // it without waiting for the routing kernel.  That kernel lets this one
+  // launch only after its own wait, so x and the logits are complete.  What
+  // this kernel does need of it, the split-tile counters it zeroes, is used
+  // only after a wait at the end of each unit; every thread waits again
+  // before it exits, so the kernels after this one still find the routing
+  // kernel complete.
+  const bool self = GATEUP && P.self_k > 0;
+  int* self_e = reinterpret_cast<int*>(bars) + 64;  // [k] expert list (bytes 256.. of the barrier block)
+  if (self && warp == 0) {  // (while warps 1..8 build the table below)
+    const int k = P.self_k;
+    int id;
+    float wt;
+    topk_warp(a.logits, a.E, k, lane, nullptr, id, wt);
+    int rank = 0;  // lane j < k: number of smaller ids among the k
+    for (int j = 0; j < k; ++j) {
+      const int o = __shfl_sync(0xffffffffu, id, j);
+      rank += (lane < k && o < id) ? 1 : 0;
+    }
+    if (lane < k) self_e[rank] = id;
+  }
   // with a single table every expert uses table 0: its table slot is built
   // before waiting for the previous kernel
   if (tp.n == 1 && warp >= 1) build_lut_slot(lut, tp.t[0], 0, threadIdx.x - 32);
@@ -425,34 +450,6 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
     __syncwarp();
   };
 
-  // Gate/up with one token (self_k > 0): its k experts are distinct and hold
-  // one row each, so the routing tables follow from the token's top-k alone
-  // (the expert list is the k ids in ascending order; expert j of it has row
-  // j, of token 0).  Warp 0 computes that top-k with the routing kernel's own
-  // warp routine on the same logits (hence the same ids) and the CTA runs on
-  // it without waiting for the routing kernel.  That kernel lets this one
-  // launch only after its own wait, so x and the logits are complete.  What
-  // this kernel does need of it, the split-tile counters it zeroes, is used
-  // only after a wait at the end of each unit; every thread waits again
-  // before it exits, so the kernels after this one still find the routing
-  // kernel complete.
-  const bool self = GATEUP && P.self_k > 0;
-  int* self_e = reinterpret_cast<int*>(bars) + 64;  // [k] expert list (bytes 256.. of the barrier block)
-  if (self) {
-    if (warp == 0) {
-      const int k = P.self_k;
-      int id;
-      float wt;
-      topk_warp(a.logits, a.E, k, lane, nullptr, id, wt);
-      int rank = 0;  // lane j < k: number of smaller ids among the k
-      for (int j = 0; j < k; ++j) {
-        const int o = __shfl_sync(0xffffffffu, id, j);
-        rank += (lane < k && o < id) ? 1 : 0;
-      }
-      if (lane < k) self_e[rank] = id;
-    }
-    __syncthreads();
-  }
   // routing tables of a unit: expert, its first row, its rows
   const auto unit_expert = [&](int unit) -> int {
     return self ? self_e[unit / P.tiles_per_e] : a.dec_list[unit / P.tiles_per_e];
