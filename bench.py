@@ -80,6 +80,22 @@ def load_peaks():
     return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def max_over_ranks(ms: float, device) -> float:
+    """The job's device time: the slowest rank's.  Every rank calls it at the
+    same point (an all-reduce with op MAX when more than one rank runs)."""
+    import torch.distributed as dist
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_step: int, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: the tokens every rank processed over the slowest
+    rank's time (replicas: each rank runs its own batches)."""
+    return tokens_per_step * steps * world / (max_ms / 1e3)
+
+
 def source_digest(files) -> str:
     """Digest of the kernel sources as compiled: line comments and blank lines
     do not count, so a comment edit keeps a profile's figures valid."""
@@ -520,12 +536,8 @@ def run_ours(args, w):
         t_end.record(stream)
         torch.cuda.synchronize()
     barrier()
-    total_ms = t_beg.elapsed_time(t_end)
-    tmax = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-    total_ms = float(tmax.item())
-    value = T * args.steps * world / (total_ms / 1e3)
+    total_ms = max_over_ranks(t_beg.elapsed_time(t_end), dev)
+    value = job_tokens_per_s(T, args.steps, world, total_ms)
     assert q4.forward_status(ws) == 0
 
     # the same steps one at a time, L2 flushed before each, outside its events
@@ -539,11 +551,7 @@ def run_ours(args, w):
         q4.forward(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)
         ends[i].record(stream)
     torch.cuda.synchronize()
-    flushed_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / n_fl
-    ft = torch.tensor([flushed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ft, op=dist.ReduceOp.MAX)
-    flushed_ms = float(ft.item())
+    flushed_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / n_fl, dev)
 
     # per-kernel times (separate pass, events between the kernels)
     n_prof = min(args.steps, 100)
@@ -577,11 +585,8 @@ def run_ours(args, w):
         e_e[i].record(stream)
         assert st == 0
     torch.cuda.synchronize()
-    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))
-    e2e_t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = T * n_e2e * world / (float(e2e_t.item()) / 1e3)
+    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), dev)
+    e2e_value = job_tokens_per_s(T, n_e2e, world, e2e_ms)
 
     hbm_peak, tf_peak, peak_src = load_peaks()
     graph_ms, graph_why = measure_graph(q4, layer, xs, lgs, k, out, ws, flush_l2, min(args.steps, 200), stream)
