@@ -268,14 +268,22 @@ def run_reference(args, w):
 
 
 def cpu_baseline(w, x_bits, lg):
-    """The oracle on this host: 2 tokens x all routed experts, full channels."""
+    """The oracle on this host's cores: 2 tokens (1 at T=1) x all their routed
+    experts, full channels, each (token, expert) split over intermediate
+    channel ranges so that every core has work."""
     import oracle
     oracle.build()
     sh = w.shape
     tokens = [0, 1] if w.T > 1 else [0]
     L, ids, _ = oracle_sample_layer(w, x_bits, lg, tokens, "cuda")
-    units = [(t, int(ids[i, j]), 0, sh.I) for i, t in enumerate(tokens) for j in range(sh.k)]
-    threads = min(len(units), os.cpu_count() or 1)
+    cores = max(1, os.cpu_count() or 1)
+    pairs = [(t, int(ids[i, j])) for i, t in enumerate(tokens) for j in range(sh.k)]
+    q = 1
+    while len(pairs) * q < cores and q < sh.I // 32:
+        q *= 2
+    chunk = sh.I // q
+    units = [(t, e, c * chunk, (c + 1) * chunk) for t, e in pairs for c in range(q)]
+    threads = min(len(units), cores)
     # repeated until about 10 s of wall time have been measured
     dt, reps = 0.0, 0
     while dt < 10.0 and reps < 200:
@@ -283,7 +291,8 @@ def cpu_baseline(w, x_bits, lg):
         reps += 1
     return {"value": reps * len(tokens) / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{len(tokens)} token(s) x {sh.k} routed experts, full layer arithmetic in fp64, "
-                      f"one (token, expert) per thread, repeated {reps} times ({dt:.1f} s)"}
+                      f"each (token, expert) in {q} channel ranges of {chunk} over {threads} threads, "
+                      f"repeated {reps} times ({dt:.1f} s)"}
 
 
 # ---------------------------------------------------------------------------
