@@ -61,7 +61,8 @@ bool shape_ok(const moe_q4_layer* L, int T, int top_k) {
 //   dec_list int32[E] | pre_list int32[E] | tiles int32[E+1] | h bf16[T*k][I] |
 //   h_lo bf16[T*k][I] | y f32[T*k][H] | xg bf16[T*k][H] (activation rows in
 //   expert order, T > 16 only) | split-tile counters int32[units] | partial sums of the
-//   small-M kernels f32[2*160][3][min(16,T)][128]
+//   small-M kernels f32[2*160][4][min(16,T)][128] (two 128-row tiles per unit,
+//   gate/up then down)
 struct Layout {
   size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, tiles, h, h_lo, y, xg, dk_counter,
       dk_partial, end;
