@@ -2,7 +2,8 @@
 
 ctypes wrapper around ``moe_q4_oracle.c``: a plain single-threaded fp64 CPU
 restatement of the routed-expert MoE over 4-bit codebook weights (decode,
-pack, top-k routing, expert grouping, the layer).  Only ``tests/``, the
+pack, top-k routing, expert grouping, the layer, the router gate and the
+weighted Lloyd-Max grid fit).  Only ``tests/``, the
 package's ``smoke()`` check and ``bench.py``'s CPU-baseline leg may import
 this module.  It shares no code with the CUDA library.
 
@@ -65,8 +66,9 @@ def lib():
         L.oq_group.argtypes = [vp, ci, ci, ci, vp, vp, vp, vp]
         L.oq_moe_tokens.argtypes = [ctypes.POINTER(_Layer), vp, vp, ci, ci, vp, vp, vp]
         L.oq_expert_partial.argtypes = [ctypes.POINTER(_Layer), ci, vp, ci, ci, vp]
+        L.oq_lloyd_fit.argtypes = [vp, ctypes.c_longlong, vp, ci, ctypes.c_double, vp, vp]
         for f in (L.oq_dequant, L.oq_decode_matrix_f64, L.oq_pack, L.oq_route, L.oq_group, L.oq_moe_tokens,
-                  L.oq_expert_partial, L.oq_router_logits):
+                  L.oq_expert_partial, L.oq_router_logits, L.oq_lloyd_fit):
             f.restype = ci
         _lib = L
     return _lib
@@ -127,6 +129,21 @@ def pack(src_bf16_bits, tables, table_id, E, N, K):
     s = np.empty((E, N, K // 32), np.uint8)
     _check(lib().oq_pack(_p(src), E, N, K, _p(t), nt, _p(tid), _p(w), _p(s)))
     return w, s
+
+
+def lloyd_fit(src_bf16_bits, grid0, max_iter: int, tol: float = 0.0):
+    """Weighted Lloyd-Max fit of the 8 grid magnitudes over the ratios
+    |w / 2^e| of bf16 weights (any shape, a whole number of 32-blocks along
+    the last axis), weighted by (2^e)^2, from the ascending grid0:
+    (grid fp32 [8], steps taken)."""
+    src = _c(src_bf16_bits, np.uint16).reshape(-1)
+    if src.size % 32:
+        raise OracleError("weights must be whole 32-blocks")
+    g0 = _c(grid0, np.float32)
+    out = np.empty(8, np.float32)
+    it = np.zeros(1, np.int32)
+    _check(lib().oq_lloyd_fit(_p(src), src.size // 32, _p(g0), max_iter, float(tol), _p(out), _p(it)))
+    return out, int(it[0])
 
 
 def router_logits(x_bf16_bits, w_bf16_bits):

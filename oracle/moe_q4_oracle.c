@@ -29,7 +29,9 @@
  * all 16 codes x edge scale bytes x both nibble positions; the E2M1 table
  * against the closed-form OCP E2M1 decode; brute-force signed-level search
  * for pack; library (numpy) sort for routing/grouping; dense-FFN reductions
- * and the intermediate-channel permutation invariant for the MoE.
+ * and the intermediate-channel permutation invariant for the MoE; for the
+ * grid fit, the uniform quantiser of U(0,1), a closed-form weighted step,
+ * decoded weights as a fixed point and power-of-two scale invariance.
  */
 #include <math.h>
 #include <stdint.h>
@@ -462,5 +464,91 @@ int oq_expert_partial(const oq_layer* L, int e, const uint16_t* x, int i0, int i
                          L->down_s[e][(size_t)n * (I / 32) + i / 32], tb) * hi;
   }
   free(xv);
+  return OQ_OK;
+}
+
+/* ---- weighted Lloyd-Max grid fit ---------------------------------------- */
+
+/* Index of the level closest (fp64 distance) to r; on a tie the lower index
+ * wins (the same rule as the pack's nearest_level). */
+static int nearest_level_f64(double r, const double* m) {
+  int best = 0;
+  double bd = fabs(r - m[0]);
+  for (int i = 1; i < 8; ++i) {
+    double d = fabs(r - m[i]);
+    if (d < bd) {
+      bd = d;
+      best = i;
+    }
+  }
+  return best;
+}
+
+/* The per-layer grid fit of [NF4-Lloyd, "What this is"]: 8 magnitudes fitted
+ * by weighted Lloyd-Max over the pooled ratios |W / 2^e| of all the layer's
+ * weights, each ratio weighted by (2^e)^2 so that it counts in proportion to
+ * its weight-space squared error.  Readings (the page names the objective,
+ * not the procedure around it):
+ *   - e is each 32-block's exponent under the pack rule ([NF4-Lloyd], "Codes
+ *     are indices...": gmax * 2^e >= amax) with gmax the largest level of the
+ *     starting grid, fixed for the whole fit;
+ *   - a Lloyd step assigns every ratio to its nearest level (tie -> lower
+ *     index) and moves each level to the weighted mean sum(w r) / sum(w) of
+ *     its ratios; a level with no ratio keeps its value;
+ *   - steps repeat until no level moves by more than tol, or max_iter steps;
+ *   - the result is each fp64 level rounded to fp32.
+ * src: n_blocks x 32 bf16 bit patterns (each run of 32 one block along K);
+ * grid0: 8 fp32 magnitudes, strictly ascending, finite, >= 0, max > 0;
+ * grid: [8] fp32 (out); *iters: steps taken (out). */
+int oq_lloyd_fit(const uint16_t* src, long long n_blocks, const float* grid0, int max_iter, double tol,
+                 float* grid, int* iters) {
+  if (n_blocks < 0 || !grid0 || !grid || !iters || max_iter < 0 || !(tol >= 0.0)) return OQ_EINVAL;
+  if (n_blocks > 0 && !src) return OQ_EINVAL;
+  if (!table_ok(grid0)) return OQ_EINVAL;
+  for (int i = 1; i < 8; ++i)
+    if (!(grid0[i] > grid0[i - 1])) return OQ_EINVAL;
+  const double gmax = (double)grid0[7];
+  int* ex = (int*)malloc(sizeof(int) * (size_t)(n_blocks > 0 ? n_blocks : 1));
+  if (!ex) return OQ_EINVAL;
+  for (long long b = 0; b < n_blocks; ++b) {
+    double amax = 0.0;
+    for (int i = 0; i < 32; ++i) {
+      double v = (double)bf16_bits_to_f32(src[b * 32 + i]);
+      if (!isfinite(v)) {
+        free(ex);
+        return OQ_EINVAL;
+      }
+      if (fabs(v) > amax) amax = fabs(v);
+    }
+    ex[b] = block_exponent(amax, gmax);
+  }
+  double m[8];
+  for (int i = 0; i < 8; ++i) m[i] = (double)grid0[i];
+  int it = 0;
+  while (it < max_iter) {
+    double sw[8] = {0}, swr[8] = {0};
+    for (long long b = 0; b < n_blocks; ++b) {
+      const double wgt = ldexp(1.0, 2 * ex[b]);
+      for (int i = 0; i < 32; ++i) {
+        const double r = ldexp(fabs((double)bf16_bits_to_f32(src[b * 32 + i])), -ex[b]);
+        const int j = nearest_level_f64(r, m);
+        sw[j] += wgt;
+        swr[j] += wgt * r;
+      }
+    }
+    double moved = 0.0;
+    for (int j = 0; j < 8; ++j) {
+      if (sw[j] > 0.0) {
+        const double nm = swr[j] / sw[j];
+        if (fabs(nm - m[j]) > moved) moved = fabs(nm - m[j]);
+        m[j] = nm;
+      }
+    }
+    ++it;
+    if (moved <= tol) break;
+  }
+  for (int j = 0; j < 8; ++j) grid[j] = (float)m[j];
+  *iters = it;
+  free(ex);
   return OQ_OK;
 }
