@@ -90,6 +90,19 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _hold(stream, *tensors):
+    """Memory this binding allocated for a call (contiguous copies, internal
+    workspaces) is read by work enqueued on `stream`, which may run after the
+    call returns: when that is not torch's current stream, tell the caching
+    allocator, so the blocks are not handed out again before the work ran.
+    (On the current stream, stream order already keeps reuse safe.)"""
+    if stream is None:
+        return
+    for t in tensors:
+        if t is not None and t.is_cuda:
+            t.record_stream(stream)
+
+
 def _check(rc, what):
     if rc != OK:
         raise MoeQ4Error(rc, what)
@@ -142,6 +155,7 @@ def pack(w: torch.Tensor, tables, table_id, status: torch.Tensor | None = None, 
         status = torch.zeros(1, dtype=torch.int32, device=w.device)
     _check(lib().moe_q4_pack(_ptr(w), E, N, K, t.ctypes.data, t.shape[0], tid.ctypes.data,
                              _ptr(codes), _ptr(scales), _ptr(status), _stream(stream)), "moe_q4_pack")
+    _hold(stream, w, status)
     if own:
         st = lib().moe_q4_read_status(_ptr(status), _stream(stream))
         _check(st, "moe_q4_pack (device)")
@@ -158,9 +172,11 @@ def dequant(codes: torch.Tensor, scales: torch.Tensor, tables, table_id, stream=
         out = torch.empty((E, N, K), dtype=torch.bfloat16, device=codes.device)
     elif out.shape != (E, N, K) or out.dtype != torch.bfloat16 or not out.is_contiguous():
         raise ValueError("out must be a contiguous bf16 tensor [E, N, K]")
-    _check(lib().moe_q4_dequant(_ptr(codes.contiguous()), _ptr(scales.contiguous()), t.ctypes.data,
+    codes, scales = codes.contiguous(), scales.contiguous()
+    _check(lib().moe_q4_dequant(_ptr(codes), _ptr(scales), t.ctypes.data,
                                 t.shape[0], tid.ctypes.data, E, N, K, _ptr(out), _stream(stream)),
            "moe_q4_dequant")
+    _hold(stream, codes, scales)
     return out
 
 
@@ -184,12 +200,15 @@ def forward(layer: Layer, x: torch.Tensor, logits: torch.Tensor, k: int, out=Non
     T = x.shape[0]
     if out is None:
         out = torch.empty((T, layer.H), dtype=torch.bfloat16, device=x.device)
-    if ws is None:
+    own_ws = ws is None
+    if own_ws:
         ws = alloc_workspace(forward_workspace(layer, T, k), x.device)
     st = layer.struct()
     _check(lib().moe_q4_forward(ctypes.byref(st), _ptr(x), _ptr(logits), T, k, _ptr(out),
                                 _ptr(out_f32), _ptr(topk_ids), _ptr(topk_w), _ptr(counts), _ptr(ws), ws.numel(),
                                 _stream(stream)), "moe_q4_forward")
+    if own_ws:
+        _hold(stream, ws)
     return out
 
 
@@ -220,9 +239,11 @@ def route(logits: torch.Tensor, k: int, stream=None):
     if need == 0:
         raise MoeQ4Error(EINVAL, "moe_q4_route_workspace")
     ws = alloc_workspace(need, dev)
-    _check(lib().moe_q4_route(_ptr(logits.contiguous()), T, E, k, _ptr(ids), _ptr(w), _ptr(counts),
+    logits = logits.contiguous()
+    _check(lib().moe_q4_route(_ptr(logits), T, E, k, _ptr(ids), _ptr(w), _ptr(counts),
                               _ptr(offsets), _ptr(row_token), _ptr(inv), _ptr(ws), ws.numel(),
                               _stream(stream)), "moe_q4_route")
+    _hold(stream, logits, ws)
     st = forward_status(ws, stream)
     return ids, w, counts, offsets, row_token, inv, st
 
@@ -242,10 +263,13 @@ def router(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None, ws
     if out is None:
         out = torch.empty((T, E), dtype=torch.float32, device=x.device)
     need = router_workspace(T, H, E)
-    if ws is None and need > 0:
+    own_ws = ws is None and need > 0
+    if own_ws:
         ws = alloc_workspace(need, x.device)
-    _check(lib().moe_q4_router(_ptr(x.contiguous()), _ptr(w.contiguous()), T, H, E, _ptr(out), _ptr(ws),
+    x, w = x.contiguous(), w.contiguous()
+    _check(lib().moe_q4_router(_ptr(x), _ptr(w), T, H, E, _ptr(out), _ptr(ws),
                                0 if ws is None else ws.numel(), _stream(stream)), "moe_q4_router")
+    _hold(stream, x, w, ws if own_ws else None)
     return out
 
 
