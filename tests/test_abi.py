@@ -94,3 +94,26 @@ def test_route_workspace_validation(L):
     assert L.moe_q4_route_workspace(256, 8, 8) > 0
     assert L.moe_q4_route_workspace(256, 8, 17) == 0
     assert L.moe_q4_route_workspace(600, 8, 8) == 0
+
+
+def test_router_workspace_and_argument_validation(L):
+    # decode sizes (T <= 32, H % 128 == 0) run as one kernel: no workspace
+    assert L.moe_q4_router_workspace(1, 6144, 256) == 0
+    assert L.moe_q4_router_workspace(32, 6144, 256) == 0
+    # more tokens, or H not a multiple of 128: K-split partials in the workspace
+    assert L.moe_q4_router_workspace(64, 6144, 256) > 0
+    assert L.moe_q4_router_workspace(1, 6144 + 32, 256) > 0
+    assert L.moe_q4_router_workspace(0, 6144, 256) == 0
+    # invalid sizes: no workspace, and the call refuses before any launch
+    assert L.moe_q4_router_workspace(1, 48, 8) == 0  # H % 32
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    out = ctypes.c_void_p(1 << 21)
+    assert L.moe_q4_router(fake, fake, 1, 48, 8, out, None, 0, None) == _lib.EINVAL
+    assert L.moe_q4_router(fake, fake, 1, 64, 0, out, None, 0, None) == _lib.EINVAL
+    assert L.moe_q4_router(fake, fake, -1, 64, 8, out, None, 0, None) == _lib.EINVAL
+    assert L.moe_q4_router(None, fake, 1, 64, 8, out, None, 0, None) == _lib.EINVAL
+    assert L.moe_q4_router(ctypes.c_void_p((1 << 20) + 8), fake, 1, 64, 8, out, None, 0, None) == _lib.EINVAL
+    # T = 0 is a valid empty call
+    assert L.moe_q4_router(None, None, 0, 64, 8, None, None, 0, None) == _lib.OK
+    # a split K needs its workspace
+    assert L.moe_q4_router(fake, fake, 64, 6144, 256, out, None, 0, None) == _lib.EWORKSPACE
