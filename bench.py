@@ -476,7 +476,9 @@ def measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream, reps=20):
     gbs = nbytes / (ms / 1e3) / 1e9
     tfs = flop / (ms / 1e3) / 1e12
     hbm_bound = T <= 256
-    return {"kernel": "router_kernel (+ router_reduce_kernel when K is split)", "ms": ms, "bytes": nbytes,
+    kernel = ("router_few_kernel (one clustered launch)" if T <= 32 and sh.H % 128 == 0
+              else "router_kernel + router_reduce_kernel (K split)")
+    return {"kernel": kernel, "ms": ms, "bytes": nbytes,
             "flop": flop, "gbs": gbs, "tflops": tfs, "bound": "hbm" if hbm_bound else "tensor",
             "frac": gbs / hbm_peak if hbm_bound else tfs / tf_peak,
             "frac_of_datasheet": gbs / DATASHEET_HBM_GBS if hbm_bound else tfs / DATASHEET_BF16_TFLOPS,
