@@ -477,7 +477,7 @@ def measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream, reps=20):
     tfs = flop / (ms / 1e3) / 1e12
     hbm_bound = T <= 256
     kernel = ("router_few_kernel (one clustered launch)" if T <= 32 and sh.H % 128 == 0
-              else "router_kernel + router_reduce_kernel (K split)")
+              else "router_kernel" + (" + router_reduce_kernel (K split)" if need else ""))
     return {"kernel": kernel, "ms": ms, "bytes": nbytes,
             "flop": flop, "gbs": gbs, "tflops": tfs, "bound": "hbm" if hbm_bound else "tensor",
             "frac": gbs / hbm_peak if hbm_bound else tfs / tf_peak,
