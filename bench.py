@@ -261,7 +261,8 @@ def run_reference(args, w):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": workload_desc(w),
+            "data": "synthetic",
+            "config": dict(workload_desc(w), parallelism=f"replicas x{args.gpus}" if args.gpus > 1 else "single GPU"),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -289,10 +290,19 @@ def cpu_baseline(w, x_bits, lg):
     while dt < 10.0 and reps < 200:
         dt += time_oracle_units(L, x_bits, units, threads)
         reps += 1
+    # the same per-token code on one thread: the first token's units, about 5 s
+    one = [u for u in units if u[0] == tokens[0]]
+    dt1, reps1 = 0.0, 0
+    while dt1 < 5.0 and reps1 < 100:
+        dt1 += time_oracle_units(L, x_bits, one, 1)
+        reps1 += 1
     return {"value": reps * len(tokens) / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{len(tokens)} token(s) x {sh.k} routed experts, full layer arithmetic in fp64, "
                       f"each (token, expert) in {q} channel ranges of {chunk} over {threads} threads, "
-                      f"repeated {reps} times ({dt:.1f} s)"}
+                      f"repeated {reps} times ({dt:.1f} s)",
+            "single_thread": {"value": reps1 / dt1, "unit": UNIT, "cores": 1, "kind": "oracle",
+                              "sample": f"1 token x {sh.k} routed experts, full layer arithmetic in fp64 on "
+                                        f"one thread, repeated {reps1} times ({dt1:.1f} s)"}}
 
 
 # ---------------------------------------------------------------------------
@@ -485,18 +495,12 @@ def measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream, reps=20):
             "note": "mma.sync bf16 GEMM; not part of the step (the layer's input is the logits)"}
 
 
-def run_ours(args, w):
-    import torch.distributed as dist
-
-    import bit_codebook_quantized_router_b200 as q4
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
-    dev = torch.device("cuda", local)
+def measure_workload(q4, w, args, steps, warmup, world, dev, local, stream, flush_l2, barrier, full):
+    """Build workload w's layer and time its forward: K steps back to back
+    (the value), per-kernel times, the host-buffer entry point (e2e) and SM
+    clocks; with `full`, also the flushed one-at-a-time steps, CUDA-graph
+    replay, the full-layer dequant and the router gate.  Returns the fields
+    of a bench line (without cpu_baseline)."""
     sh = w.shape
     T, k = w.T, sh.k
     layer = build_device_layer(w)
@@ -510,19 +514,8 @@ def run_ours(args, w):
         counts.append(torch.bincount(ids.reshape(-1), minlength=sh.E).cpu().numpy())
     ws = q4.alloc_workspace(q4.forward_workspace(layer, T, k))
     out = torch.empty((T, sh.H), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    scrub = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream()
 
-    def flush_l2(i):
-        flush.fill_(i & 0xFF)
-        scrub.sum()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    for i in range(args.warmup):
+    for i in range(warmup):
         q4.forward(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)
     torch.cuda.synchronize()
     assert q4.forward_status(ws) == 0
@@ -538,34 +531,36 @@ def run_ours(args, w):
     barrier()
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
-        torch.cuda._sleep(int(min(args.steps, 2000) * 400_000))  # about 0.2 ms per step at 2 GHz
+        torch.cuda._sleep(int(min(steps, 2000) * 400_000))  # about 0.2 ms per step at 2 GHz
         t_beg.record(stream)
         h0 = time.perf_counter()
-        for i in range(args.steps):
+        for i in range(steps):
             q4.forward(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)
         enqueue_ms = (time.perf_counter() - h0) * 1e3
         t_end.record(stream)
         torch.cuda.synchronize()
     barrier()
     total_ms = max_over_ranks(t_beg.elapsed_time(t_end), dev)
-    value = job_tokens_per_s(T, args.steps, world, total_ms)
+    value = job_tokens_per_s(T, steps, world, total_ms)
     assert q4.forward_status(ws) == 0
 
-    # the same steps one at a time, L2 flushed before each, outside its events
-    n_fl = min(args.steps, 200)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_fl)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_fl)]
-    torch.cuda.synchronize()
-    for i in range(n_fl):
-        flush_l2(i)
-        starts[i].record(stream)
-        q4.forward(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)
-        ends[i].record(stream)
-    torch.cuda.synchronize()
-    flushed_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / n_fl, dev)
+    flushed_ms = None
+    if full:
+        # the same steps one at a time, L2 flushed before each, outside its events
+        n_fl = min(steps, 200)
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_fl)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(n_fl)]
+        torch.cuda.synchronize()
+        for i in range(n_fl):
+            flush_l2(i)
+            starts[i].record(stream)
+            q4.forward(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        flushed_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / n_fl, dev)
 
     # per-kernel times (separate pass, events between the kernels)
-    n_prof = min(args.steps, 100)
+    n_prof = min(steps, 100)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(8)] for _ in range(n_prof)]
     for row in evs:  # torch creates the CUDA event on first record
         for ev in row:
@@ -579,7 +574,7 @@ def run_ours(args, w):
     assert q4.forward_status(ws) == 0
 
     # e2e through the host-buffer entry point (pinned host memory)
-    n_e2e = min(args.steps, 200)
+    n_e2e = min(steps, 200)
     xh = [x.cpu().pin_memory() for x in xs]
     lh = [l.cpu().pin_memory() for l in lgs]
     oh = torch.empty((T, sh.H), dtype=torch.bfloat16).pin_memory()
@@ -598,45 +593,103 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), dev)
     e2e_value = job_tokens_per_s(T, n_e2e, world, e2e_ms)
+    del wsh
 
     hbm_peak, tf_peak, peak_src = load_peaks()
-    graph_ms, graph_why = measure_graph(q4, layer, xs, lgs, k, out, ws, flush_l2, min(args.steps, 200), stream)
-    dq = measure_dequant(q4, layer, hbm_peak, flush_l2, stream) if not args.no_dequant else None
-    rt = measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream)
     work = [kernel_work(sh, T, c) for c in counts]
     roof, kernels = roofline(work, kern_ms, n_prof, hbm_peak, tf_peak, peak_src)
     gu, dn = expert_bytes(sh)
     layer_bytes = float(np.mean(touched)) * (gu + dn) + T * sh.H * 2 * 2
-    # our kernels per forward: route (1 fused for T <= 256, else 2), gather,
-    # small-M gate/up and down, combine, and the two tensor-core GEMMs for T > 16
-    kernels_per_step = (1 if T <= 256 else 2) + 4 + (2 if T > 16 else 0)
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+    # our kernels per forward: route (1 fused for T <= 256, else 2), small-M
+    # gate/up and down, combine, and for T > 16 the gather and the two
+    # tensor-core GEMMs
+    kernels_per_step = (1 if T <= 256 else 2) + 3 + (3 if T > 16 else 0)
+    res = {
+        "value": value, "ms_per_step": total_ms / steps, "steps": steps, "warmup": warmup,
         "config": dict(workload_desc(w), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
         "roofline": roof,
         "kernels": kernels,
         "layer_hbm": {"touched_experts": float(np.mean(touched)), "bytes_per_step": layer_bytes,
-                      "gbs": layer_bytes / (total_ms / args.steps / 1e3) / 1e9,
-                      "frac_of_peak": layer_bytes / (total_ms / args.steps / 1e3) / 1e9 / hbm_peak,
-                      "frac_of_datasheet": layer_bytes / (total_ms / args.steps / 1e3) / 1e9 / DATASHEET_HBM_GBS},
+                      "gbs": layer_bytes / (total_ms / steps / 1e3) / 1e9,
+                      "frac_of_peak": layer_bytes / (total_ms / steps / 1e3) / 1e9 / hbm_peak,
+                      "frac_of_datasheet": layer_bytes / (total_ms / steps / 1e3) / 1e9 / DATASHEET_HBM_GBS},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * sh.H * 2 + T * sh.E * 4,
                 "d2h_bytes_per_step": T * sh.H * 2},
-        "flushed": {"value": T * world / (flushed_ms / 1e3), "unit": UNIT, "ms_per_step": flushed_ms,
-                    "steps": n_fl,
-                    "note": "each step alone between its own events, L2 flushed before it (outside the events)"},
         "enqueue_ms": enqueue_ms,
-        "graph": ({"value": T * world / (graph_ms / 1e3), "unit": UNIT, "ms_per_step": graph_ms,
-                   "note": "same forward replayed from CUDA graphs, L2 flushed outside the events"}
-                  if graph_ms else {"value": None, "unavailable": graph_why}),
-        "dequant": dq,
-        "router": rt,
-        "gpu_launches": kernels_per_step * args.steps,
+        "gpu_launches": kernels_per_step * steps,
         "clocks": clk.summary(),
     }
+    if full:
+        res["flushed"] = {"value": T * world / (flushed_ms / 1e3), "unit": UNIT, "ms_per_step": flushed_ms,
+                          "steps": n_fl,
+                          "note": "each step alone between its own events, L2 flushed before it (outside the events)"}
+        graph_ms, graph_why = measure_graph(q4, layer, xs, lgs, k, out, ws, flush_l2, min(steps, 200), stream)
+        res["graph"] = ({"value": T * world / (graph_ms / 1e3), "unit": UNIT, "ms_per_step": graph_ms,
+                         "note": "same forward replayed from CUDA graphs, L2 flushed outside the events"}
+                        if graph_ms else {"value": None, "unavailable": graph_why})
+        res["dequant"] = measure_dequant(q4, layer, hbm_peak, flush_l2, stream) if not args.no_dequant else None
+        res["router"] = measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream)
+        res["_cpu_inputs"] = (inputs.bf16_bits(xs[0]), lgs[0].cpu().numpy())
+    del layer, xs, lgs, ws, out
+    torch.cuda.empty_cache()
+    return res
+
+
+# workloads timed in the same run beside the primary one (one GPU only): the
+# second decode size and the tensor-core prefill size of the performance bars
+EXTRA_WORKLOADS = ("decode_t8", "prefill_t2048")
+EXTRA_STEPS = 50
+
+
+def run_ours(args, w):
+    import torch.distributed as dist
+
+    import bit_codebook_quantized_router_b200 as q4
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    scrub = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def flush_l2(i):
+        flush.fill_(i & 0xFF)
+        scrub.sum()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    res = measure_workload(q4, w, args, args.steps, args.warmup, world, dev, local, stream, flush_l2, barrier,
+                           full=True)
+    x_bits, lg0 = res.pop("_cpu_inputs")
+    line = {"metric": METRIC, "value": res.pop("value"), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res.pop("ms_per_step"), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic"}
+    res.pop("steps")
+    res.pop("warmup")
+    line.update(res)
+    if world == 1 and not args.no_extra:
+        extra = {}
+        for name in EXTRA_WORKLOADS:
+            if name == w.name:
+                continue
+            we = inputs.WORKLOADS[name]
+            if args.experts:
+                import dataclasses
+                we = dataclasses.replace(we, shape=dataclasses.replace(we.shape, E=args.experts))
+            r = measure_workload(q4, we, args, min(args.steps, EXTRA_STEPS), args.warmup, world, dev, local,
+                                 stream, flush_l2, barrier, full=False)
+            r["metric"], r["unit"] = METRIC, UNIT
+            extra[name] = r
+        line["workloads"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, inputs.bf16_bits(xs[0]), lgs[0].cpu().numpy())
+        line["cpu_baseline"] = cpu_baseline(w, x_bits, lg0)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -653,6 +706,8 @@ def main():
     ap.add_argument("--workload", default="decode_t1", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dequant", action="store_true", help="skip the standalone full-layer dequant measurement")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only --workload (not also decode_t8 and prefill_t2048 in the same line)")
     ap.add_argument("--experts", type=int, default=0,
                     help="layer with this many experts (same H, I, top-k) instead of the workload's; "
                          "for small profiling captures")
