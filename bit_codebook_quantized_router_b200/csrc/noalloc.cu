@@ -13,7 +13,11 @@
 // cannot use the array's name as a device address (on the host it names a
 // host-side stand-in), so the first call on each device looks the address up
 // with cudaGetSymbolAddress while that device is current and caches it; make
-// that first call outside any stream capture.  All calls share the one
+// that first call outside any stream capture.  The cached address belongs to
+// the device's primary context: after cudaDeviceReset on that device the
+// library's module is loaded afresh at another address, so this entry point
+// must not be used on a device that has been reset since its first call.
+// All calls share the one
 // array and it keeps the previous call's contents: the forward rewrites every
 // word it reads (the status word is reset by the routing step itself), and
 // two calls whose work overlaps on the GPU (different streams, or different
@@ -58,7 +62,11 @@ extern "C" int moe_q4_forward_noalloc(const moe_q4_layer* layer, const void* x, 
   if (!ws) return MOE_Q4_ECUDA;
   const int rc = q4_forward_in_workspace(layer, x, logits, T, top_k, out, out_f32, ws, kNoAllocScratchBytes,
                                          (cudaStream_t)stream);
-  if (rc != MOE_Q4_OK || !status || T == 0) return rc;
+  if (rc != MOE_Q4_OK || !status) return rc;
+  // no tokens: nothing ran, so the status is OK (written, not left stale)
+  if (T == 0)
+    return cudaMemsetAsync(status, 0, sizeof(int32_t), (cudaStream_t)stream) == cudaSuccess ? MOE_Q4_OK
+                                                                                            : MOE_Q4_ECUDA;
   // the status word is the workspace's first int32
   return cudaMemcpyAsync(status, ws, sizeof(int32_t), cudaMemcpyDeviceToDevice, (cudaStream_t)stream) ==
                  cudaSuccess

@@ -267,12 +267,16 @@ MOE_Q4_API int moe_q4_forward_stages(const moe_q4_layer* layer, const void* x,
  * MOE_Q4_ENOTSUP before anything is launched; at the GLM-5.2 layer shape
  * (H 6144, I 2048, 256 experts, top-8) that admits T <= 10.  The first call on
  * a device looks up the array's device address (cudaGetSymbolAddress) and
- * caches it: make that first call before any stream capture.  All calls share
- * the array; calls that overlap on the GPU race on it, so serialise them.
+ * caches it: make that first call before any stream capture, and do not use
+ * this entry point on a device after cudaDeviceReset of that device (the
+ * cached address would be stale).  All calls share the array and it keeps
+ * the last call's contents; calls that overlap on the GPU race on it, so
+ * serialise them.
  * Arguments as for moe_q4_forward, plus:
  *   status   optional device int32 (out), NULL to skip: receives the
  *            forward's device status word (MOE_Q4_OK / MOE_Q4_EDEVICE /
- *            MOE_Q4_ETIMEOUT) by a stream-ordered device-to-device copy.
+ *            MOE_Q4_ETIMEOUT) by a stream-ordered device-to-device copy;
+ *            with T == 0 it receives MOE_Q4_OK.
  * No allocation of any kind (no cudaMalloc/cudaFree, no allocating library
  * routine); the call returns without waiting for the GPU.
  * ------------------------------------------------------------------------- */
