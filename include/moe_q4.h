@@ -265,7 +265,7 @@ MOE_Q4_API int moe_q4_forward_stages(const moe_q4_layer* layer, const void* x,
  * every GPU that loads the library until the process exits.  Sizes whose
  * workspace (moe_q4_forward_workspace) exceeds it are rejected with
  * MOE_Q4_ENOTSUP before anything is launched; at the GLM-5.2 layer shape
- * (H 6144, I 2048, 256 experts, top-8) that admits T <= 10.  The first call on
+ * (H 6144, I 2048, 256 experts, top-8) that admits T <= 9.  The first call on
  * a device looks up the array's device address (cudaGetSymbolAddress) and
  * caches it: make that first call before any stream capture, and do not use
  * this entry point on a device after cudaDeviceReset of that device (the

@@ -123,10 +123,11 @@ def test_noalloc_zero_tokens_writes_ok_status():
     assert int(status.item()) == _lib.OK
 
 
-def test_noalloc_refuses_sizes_beyond_its_scratch():
+@pytest.mark.parametrize("T", [10, 24])
+def test_noalloc_refuses_sizes_beyond_its_scratch(T):
     w = inputs.WORKLOADS["decode_t8"]
     layer = gpu_support.device_layer(w)
-    T, k, H = 24, w.shape.k, w.shape.H  # workspace 16.9 MB > 8 MiB (the GLM shape admits T <= 10)
+    k, H = w.shape.k, w.shape.H  # the GLM shape admits T <= 9 (T = 10 needs 8.86 MiB, T = 24 16.9 MB)
     x = torch.zeros((T, H), dtype=torch.bfloat16, device="cuda")
     lg = torch.zeros((T, w.shape.E), dtype=torch.float32, device="cuda")
     out = torch.full((T, H), 7.0, dtype=torch.bfloat16, device="cuda")
