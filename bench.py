@@ -25,6 +25,7 @@ device time is the max over ranks; value = tokens of all ranks / that time.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import hashlib
 import json
 import os
@@ -458,6 +459,57 @@ def measure_dequant(q4, layer, hbm_peak, flush_l2, stream, reps=5):
             "gbs": gbs, "frac": gbs / hbm_peak, "frac_of_datasheet": gbs / DATASHEET_HBM_GBS}
 
 
+def measure_lloyd(q4, w, hbm_peak, flush_l2, stream, reps=3, max_iter=100):
+    """The layer's weighted Lloyd-Max grid fit on the GPU: one pass over all
+    the layer's bf16 expert weights (gate, up, down of every expert) into the
+    ratio histogram, then the Lloyd steps on it.  Algorithmic bytes: the bf16
+    weights read once."""
+    sh = w.shape
+    grid0 = inputs.lloyd_max_grid()
+    projs = []
+    for proj in inputs.PROJECTIONS:
+        N, K = inputs.proj_shape(sh, proj)
+        big = torch.empty((sh.E, N, K), dtype=torch.bfloat16, device="cuda")
+        for e in range(sh.E):
+            big[e] = inputs.expert_weight(w, e, proj, device="cuda")
+        projs.append(big)
+    nbytes = sum(p.numel() * 2 for p in projs)
+    g, it, st = q4.lloyd_fit(projs, grid0, max_iter=max_iter)  # warm
+    torch.cuda.synchronize()
+    ok = st == 0
+    need = int(q4.lib().moe_q4_lloyd_workspace(np.ascontiguousarray(grid0, np.float32).ctypes.data))
+    ws = q4.alloc_workspace(need)
+    g0 = np.ascontiguousarray(grid0, np.float32)
+    grid = torch.empty(8, dtype=torch.float32, device="cuda")
+    iters = torch.empty(1, dtype=torch.int32, device="cuda")
+    L = q4.lib()
+    sid = ctypes.c_void_p(stream.cuda_stream)
+    hist_ms, solve_ms = [], []
+    for i in range(reps):
+        flush_l2(i)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record(stream)
+        for j, p in enumerate(projs):
+            L.moe_q4_lloyd_hist(ctypes.c_void_p(p.data_ptr()), p.numel() // 32, g0.ctypes.data, 1 if j == 0 else 0,
+                                ctypes.c_void_p(ws.data_ptr()), ws.numel(), sid)
+        e1.record(stream)
+        L.moe_q4_lloyd_solve(g0.ctypes.data, max_iter, ctypes.c_double(1e-12), ctypes.c_void_p(grid.data_ptr()),
+                             ctypes.c_void_p(iters.data_ptr()), ctypes.c_void_p(ws.data_ptr()), ws.numel(), sid)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        hist_ms.append(e0.elapsed_time(e1))
+        solve_ms.append(e1.elapsed_time(e2))
+    ok = ok and torch.equal(grid, g) and int(iters.item()) == int(it.item())
+    del projs
+    torch.cuda.empty_cache()
+    hm, sm = float(np.median(hist_ms)), float(np.median(solve_ms))
+    gbs = nbytes / (hm / 1e3) / 1e9
+    return {"kernel": "lloyd_hist_kernel (ratio histogram over all 256 x 3 projections) + lloyd_solve_kernel",
+            "bytes": nbytes, "hist_ms": hm, "solve_ms": sm, "iters": int(it.item()),
+            "grid": [float(v) for v in g.cpu().numpy()], "gbs": gbs, "frac": gbs / hbm_peak,
+            "frac_of_datasheet": gbs / DATASHEET_HBM_GBS, "status_ok": bool(ok)}
+
+
 def measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream, reps=20):
     """The router gate ahead of the layer (moe_q4_router): bf16 x [T, H] times
     the bf16 gate [E, H] -> fp32 logits.  Algorithmic work: the gate and x read
@@ -629,6 +681,8 @@ def measure_workload(q4, w, args, steps, warmup, world, dev, local, stream, flus
                         if graph_ms else {"value": None, "unavailable": graph_why})
         res["dequant"] = measure_dequant(q4, layer, hbm_peak, flush_l2, stream) if not args.no_dequant else None
         res["router"] = measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream)
+        if not args.no_lloyd:
+            res["lloyd"] = measure_lloyd(q4, w, hbm_peak, flush_l2, stream)
         res["_cpu_inputs"] = (inputs.bf16_bits(xs[0]), lgs[0].cpu().numpy())
     del layer, xs, lgs, ws, out
     torch.cuda.empty_cache()
@@ -706,6 +760,7 @@ def main():
     ap.add_argument("--workload", default="decode_t1", choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dequant", action="store_true", help="skip the standalone full-layer dequant measurement")
+    ap.add_argument("--no-lloyd", action="store_true", help="skip the GPU grid-fit measurement")
     ap.add_argument("--no-extra", action="store_true",
                     help="time only --workload (not also decode_t8 and prefill_t2048 in the same line)")
     ap.add_argument("--experts", type=int, default=0,

@@ -6,10 +6,9 @@ binding.  Importing it does not load the library; the first call does, and
 raises if the library was not built (there is no CPU fallback).
 """
 from ._lib import (Layer, MoeQ4Error, alloc_workspace, dequant, forward, forward_host,
-                   forward_host_workspace, forward_stages, forward_status, forward_workspace, lib, pack, route,
-                   router, router_workspace,
-                   status_string)
+                   forward_host_workspace, forward_stages, forward_status, forward_workspace, lib, lloyd_fit,
+                   pack, route, router, router_workspace, status_string)
 
 __all__ = ["Layer", "MoeQ4Error", "alloc_workspace", "dequant", "forward", "forward_host",
-           "forward_host_workspace", "forward_stages", "forward_status", "forward_workspace", "lib", "pack",
-           "route", "router", "router_workspace", "status_string"]
+           "forward_host_workspace", "forward_stages", "forward_status", "forward_workspace", "lib", "lloyd_fit",
+           "pack", "route", "router", "router_workspace", "status_string"]

@@ -65,9 +65,13 @@ def lib():
         L.moe_q4_router_workspace.argtypes = [ci, ci, ci]
         L.moe_q4_router_workspace.restype = sz
         L.moe_q4_router.argtypes = [vp, vp, ci, ci, ci, vp, vp, sz, vp]
+        L.moe_q4_lloyd_workspace.argtypes = [vp]
+        L.moe_q4_lloyd_workspace.restype = sz
+        L.moe_q4_lloyd_hist.argtypes = [vp, ctypes.c_longlong, vp, ci, vp, sz, vp]
+        L.moe_q4_lloyd_solve.argtypes = [vp, ci, ctypes.c_double, vp, vp, vp, sz, vp]
         for f in (L.moe_q4_pack, L.moe_q4_dequant, L.moe_q4_forward, L.moe_q4_forward_host,
                   L.moe_q4_forward_status, L.moe_q4_read_status, L.moe_q4_route,
-                  L.moe_q4_forward_stages, L.moe_q4_router):
+                  L.moe_q4_forward_stages, L.moe_q4_router, L.moe_q4_lloyd_hist, L.moe_q4_lloyd_solve):
             f.restype = ci
         if L.moe_q4_abi_version() != 1:
             raise ImportError("libmoe_q4 ABI version mismatch")
@@ -281,3 +285,32 @@ def forward_stages(layer: Layer, x, logits, k: int, out, ws, events, stream=None
     _check(lib().moe_q4_forward_stages(ctypes.byref(st), _ptr(x), _ptr(logits), x.shape[0], k, _ptr(out),
                                        _ptr(ws), ws.numel(), _stream(stream), arr, len(events)),
            "moe_q4_forward_stages")
+
+
+def lloyd_fit(weights, grid0, max_iter: int = 300, tol: float = 1e-12, stream=None):
+    """Weighted Lloyd-Max fit of an 8-level grid over the pooled ratios of one
+    or more bf16 CUDA tensors (each a whole number of 32-weight blocks along
+    its last dimension).  Returns (grid fp32 CUDA [8], iters int32 CUDA [1],
+    status)."""
+    if isinstance(weights, torch.Tensor):
+        weights = [weights]
+    g0 = np.ascontiguousarray(np.asarray(grid0, np.float32).reshape(8))
+    need = int(lib().moe_q4_lloyd_workspace(g0.ctypes.data))
+    if need == 0:
+        raise MoeQ4Error(EINVAL, "moe_q4_lloyd_workspace")
+    dev = weights[0].device
+    ws = alloc_workspace(need, dev)
+    for i, w in enumerate(weights):
+        if w.dtype != torch.bfloat16 or not w.is_cuda or w.numel() % 32:
+            raise ValueError("weights must be bf16 CUDA tensors holding whole 32-weight blocks")
+        w = w.contiguous()
+        _check(lib().moe_q4_lloyd_hist(_ptr(w), w.numel() // 32, g0.ctypes.data, 1 if i == 0 else 0, _ptr(ws),
+                                       ws.numel(), _stream(stream)), "moe_q4_lloyd_hist")
+        _hold(stream, w)
+    grid = torch.empty(8, dtype=torch.float32, device=dev)
+    iters = torch.empty(1, dtype=torch.int32, device=dev)
+    _check(lib().moe_q4_lloyd_solve(g0.ctypes.data, int(max_iter), float(tol), _ptr(grid), _ptr(iters), _ptr(ws),
+                                    ws.numel(), _stream(stream)), "moe_q4_lloyd_solve")
+    _hold(stream, ws)
+    status = int(lib().moe_q4_read_status(_ptr(ws), _stream(stream)))
+    return grid, iters, status

@@ -284,6 +284,46 @@ MOE_Q4_API int moe_q4_forward_noalloc(const moe_q4_layer* layer, const void* x,
                                       const float* logits, int T, int top_k, void* out,
                                       float* out_f32, int32_t* status, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * moe_q4_lloyd_hist / moe_q4_lloyd_solve -- fit a layer's 8-level magnitude
+ * grid by weighted Lloyd-Max ("aidendle94/GLM-5.2-NF4-Lloyd-Experts-GPTQ",
+ * "What this is": Lloyd-Max over the pooled ratios |W / 2^e| of all the
+ * layer's weights, each ratio weighted by (2^e)^2).
+ *
+ * Procedure (the page names the objective; the steps around it are this
+ * library's reading):
+ *   - e is each 32-weight block's exponent under the pack rule (the smallest
+ *     e with gmax * 2^e >= max |w|, clamped to [-127, 127]), with gmax the
+ *     largest level of grid0, fixed for the whole fit;
+ *   - a step assigns every ratio |w| / 2^e to its nearest level (fp64
+ *     distance, a tie to the lower index) and moves each level to the
+ *     (2^e)^2-weighted mean of its ratios; a level with no ratio keeps its
+ *     value;
+ *   - steps repeat until no level moves by more than tol, or max_iter steps;
+ *     the levels are then rounded to fp32.
+ * moe_q4_lloyd_hist adds the ratios of n_blocks blocks of 32 bf16 weights
+ * (device, 16-byte aligned, each run of 32 one block along K) into the
+ * workspace's histogram (reset != 0 clears it first); call it once per array
+ * to pool several arrays (a layer's projections).  moe_q4_lloyd_solve runs
+ * the steps on the histogram and writes grid (device fp32 [8]) and iters
+ * (device int32, the steps taken).
+ *   grid0   host fp32 [8]: finite, no sign bit, strictly ascending, gmax < 16
+ *           (MOE_Q4_EINVAL / MOE_Q4_ENOTSUP otherwise);
+ *   ws      device workspace of moe_q4_lloyd_workspace(grid0) bytes, 256-byte
+ *           aligned; its first int32 is a status word (read with
+ *           moe_q4_read_status): MOE_Q4_EDEVICE if a weight is NaN or Inf
+ *           (those weights are left out), MOE_Q4_ENOTSUP if a ratio exceeds
+ *           gmax (only for blocks whose exponent is clamped at 127).
+ * Deterministic: the histogram sums powers of four (exact while a bin's sum
+ * stays within 2^53 of its smallest term) and the steps add the per-level
+ * sums in a fixed order.  No allocation, no host synchronisation.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API size_t moe_q4_lloyd_workspace(const float* grid0);
+MOE_Q4_API int moe_q4_lloyd_hist(const void* w, long long n_blocks, const float* grid0, int reset, void* ws,
+                                 size_t ws_bytes, void* stream);
+MOE_Q4_API int moe_q4_lloyd_solve(const float* grid0, int max_iter, double tol, float* grid, int32_t* iters,
+                                  const void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronise `stream` and return the int32 at device address `status`
  * (as written by moe_q4_pack), or MOE_Q4_ECUDA. */
 MOE_Q4_API int moe_q4_read_status(const int32_t* status, void* stream);

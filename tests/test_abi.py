@@ -117,3 +117,25 @@ def test_router_workspace_and_argument_validation(L):
     assert L.moe_q4_router(None, None, 0, 64, 8, None, None, 0, None) == _lib.OK
     # a split K needs its workspace
     assert L.moe_q4_router(fake, fake, 64, 6144, 256, out, None, 0, None) == _lib.EWORKSPACE
+
+
+def test_lloyd_host_checks(L):
+    g = np.array([0.13, 0.39, 0.66, 0.94, 1.26, 1.62, 2.08, 2.75], np.float32)
+    assert L.moe_q4_lloyd_workspace(g.ctypes.data) > 0
+    for bad in (g[::-1].copy(), np.where(np.arange(8) == 2, g[1], g).astype(np.float32),
+                np.concatenate([[-0.0], g[1:]]).astype(np.float32), (g * 8).astype(np.float32)):
+        assert L.moe_q4_lloyd_workspace(np.ascontiguousarray(bad).ctypes.data) == 0
+    assert L.moe_q4_lloyd_workspace(None) == 0
+    ws_n = L.moe_q4_lloyd_workspace(g.ctypes.data)
+    fake = ctypes.c_void_p(1 << 20)
+    # a gmax of 16 or more is beyond the histogram of this build
+    big = (g * 8).astype(np.float32)
+    assert L.moe_q4_lloyd_hist(fake, 1, big.ctypes.data, 1, fake, ws_n, None) == _lib.ENOTSUP
+    assert L.moe_q4_lloyd_hist(fake, -1, g.ctypes.data, 1, fake, ws_n, None) == _lib.EINVAL
+    assert L.moe_q4_lloyd_hist(ctypes.c_void_p((1 << 20) + 2), 1, g.ctypes.data, 1, fake, ws_n, None) == _lib.EINVAL
+    assert L.moe_q4_lloyd_hist(fake, 1, g.ctypes.data, 1, fake, ws_n - 8, None) == _lib.EWORKSPACE
+    assert L.moe_q4_lloyd_hist(fake, 1, g.ctypes.data, 1, None, ws_n, None) == _lib.EWORKSPACE
+    out = ctypes.c_void_p(1 << 21)
+    assert L.moe_q4_lloyd_solve(g.ctypes.data, -1, 0.0, out, out, fake, ws_n, None) == _lib.EINVAL
+    assert L.moe_q4_lloyd_solve(g.ctypes.data, 5, -1.0, out, out, fake, ws_n, None) == _lib.EINVAL
+    assert L.moe_q4_lloyd_solve(g.ctypes.data, 5, 0.0, None, out, fake, ws_n, None) == _lib.EINVAL
