@@ -67,6 +67,7 @@ def lib():
         L.oq_moe_tokens.argtypes = [ctypes.POINTER(_Layer), vp, vp, ci, ci, vp, vp, vp]
         L.oq_expert_partial.argtypes = [ctypes.POINTER(_Layer), ci, vp, ci, ci, vp]
         L.oq_lloyd_fit.argtypes = [vp, ctypes.c_longlong, vp, ci, ctypes.c_double, vp, vp]
+        L.oq_shared_ffn.argtypes = [vp, ci, ci, vp, vp, ci, vp]
         for f in (L.oq_dequant, L.oq_decode_matrix_f64, L.oq_pack, L.oq_route, L.oq_group, L.oq_moe_tokens,
                   L.oq_expert_partial, L.oq_router_logits, L.oq_lloyd_fit):
             f.restype = ci
@@ -160,6 +161,22 @@ def router_logits(x_bf16_bits, w_bf16_bits):
     absdot = np.zeros((T, E), np.float64)
     _check(lib().oq_router_logits(_p(x), _p(w), T, H, E, _p(logits), _p(absdot)))
     return logits, absdot
+
+
+def shared_ffn(x_bf16_bits, wgu_bf16_bits, wd_bf16_bits):
+    """The shared expert's output for every token, fp64 [T][H]: x [T][H],
+    merged gate+up Wgu [2I][H] (gate rows first), down Wd [H][I], all bf16
+    bit patterns."""
+    x = _c(x_bf16_bits, np.uint16)
+    wgu = _c(wgu_bf16_bits, np.uint16)
+    wd = _c(wd_bf16_bits, np.uint16)
+    T, H = x.shape
+    I2, H2 = wgu.shape
+    if H2 != H or I2 % 2 or wd.shape != (H, I2 // 2):
+        raise OracleError("shared expert shapes disagree")
+    out = np.zeros((T, H), np.float64)
+    _check(lib().oq_shared_ffn(_p(x), T, H, _p(wgu), _p(wd), I2 // 2, _p(out)))
+    return out
 
 
 def route(logits, k):

@@ -266,6 +266,50 @@ int oq_router_logits(const uint16_t* x, const uint16_t* w, int T, int H, int E, 
   return OQ_OK;
 }
 
+/* ---- shared expert ----------------------------------------------------- */
+
+/* The shared expert ([TR3v4] README, "Checkpoint layout update": the
+ * shared-expert MLP is kept as its original BF16 weights, gate and up
+ * concatenated into one payload): for every token,
+ *   g = Wg x, u = Wu x, h = silu(g) * u, y = Wd h,
+ * with Wgu = [Wg; Wu] ([2 I][H], rows 0..I-1 the gate, I..2I-1 the up, the
+ * order in which the page concatenates them) and Wd [H][I], all in fp64 from
+ * the bf16 values.  Readings: the shared expert sees every token with weight
+ * 1 and its output is added to the routed experts' weighted sum (the pages
+ * describe the shared expert beside the routed ones, with no gate of its own).
+ * x: [T][H] bf16; out: [T][H] fp64 (the shared expert's output alone). */
+int oq_shared_ffn(const uint16_t* x, int T, int H, const uint16_t* wgu, const uint16_t* wd, int I, double* out) {
+  if (T < 0 || H <= 0 || I <= 0) return OQ_EINVAL;
+  if (T == 0) return OQ_OK;
+  if (!x || !wgu || !wd || !out) return OQ_EINVAL;
+  double* xv = (double*)malloc(sizeof(double) * H);
+  double* hv = (double*)malloc(sizeof(double) * I);
+  if (!xv || !hv) {
+    free(xv);
+    free(hv);
+    return OQ_EINVAL;
+  }
+  for (int t = 0; t < T; ++t) {
+    for (int c = 0; c < H; ++c) xv[c] = (double)bf16_bits_to_f32(x[(size_t)t * H + c]);
+    for (int i = 0; i < I; ++i) {
+      double g = 0.0, u = 0.0;
+      for (int c = 0; c < H; ++c) {
+        g += (double)bf16_bits_to_f32(wgu[(size_t)i * H + c]) * xv[c];
+        u += (double)bf16_bits_to_f32(wgu[(size_t)(I + i) * H + c]) * xv[c];
+      }
+      hv[i] = g / (1.0 + exp(-g)) * u;
+    }
+    for (int c = 0; c < H; ++c) {
+      double y = 0.0;
+      for (int i = 0; i < I; ++i) y += (double)bf16_bits_to_f32(wd[(size_t)c * I + i]) * hv[i];
+      out[(size_t)t * H + c] = y;
+    }
+  }
+  free(xv);
+  free(hv);
+  return OQ_OK;
+}
+
 /* ---- routing ----------------------------------------------------------- */
 
 /* Top-k of E logits per token, then softmax over the k kept.
