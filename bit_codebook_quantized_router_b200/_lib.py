@@ -22,6 +22,10 @@ class MoeQ4Error(RuntimeError):
         super().__init__(f"{what}: moe_q4 status {status} ({status_string(status)})")
 
 
+class _SharedStruct(ctypes.Structure):
+    _fields_ = [("I", ctypes.c_int), ("gate_up", ctypes.c_void_p), ("down", ctypes.c_void_p)]
+
+
 class _LayerStruct(ctypes.Structure):
     _fields_ = [
         ("E", ctypes.c_int), ("H", ctypes.c_int), ("I", ctypes.c_int),
@@ -65,6 +69,11 @@ def lib():
         L.moe_q4_router_workspace.argtypes = [ci, ci, ci]
         L.moe_q4_router_workspace.restype = sz
         L.moe_q4_router.argtypes = [vp, vp, ci, ci, ci, vp, vp, sz, vp]
+        L.moe_q4_forward_ex_workspace.argtypes = [ctypes.POINTER(_LayerStruct), ctypes.POINTER(_SharedStruct), ci, ci]
+        L.moe_q4_forward_ex_workspace.restype = sz
+        L.moe_q4_forward_ex.argtypes = [ctypes.POINTER(_LayerStruct), ctypes.POINTER(_SharedStruct), vp, vp, ci, ci,
+                                        vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_q4_forward_ex.restype = ci
         L.moe_q4_lloyd_workspace.argtypes = [vp]
         L.moe_q4_lloyd_workspace.restype = sz
         L.moe_q4_lloyd_hist.argtypes = [vp, ctypes.c_longlong, vp, ci, vp, sz, vp]
@@ -211,6 +220,47 @@ def forward(layer: Layer, x: torch.Tensor, logits: torch.Tensor, k: int, out=Non
     _check(lib().moe_q4_forward(ctypes.byref(st), _ptr(x), _ptr(logits), T, k, _ptr(out),
                                 _ptr(out_f32), _ptr(topk_ids), _ptr(topk_w), _ptr(counts), _ptr(ws), ws.numel(),
                                 _stream(stream)), "moe_q4_forward")
+    if own_ws:
+        _hold(stream, ws)
+    return out
+
+
+class Shared:
+    """A BF16 shared expert: gate_up bf16 [2I, H] (gate rows first), down
+    bf16 [H, I] (CUDA tensors)."""
+
+    def __init__(self, gate_up: torch.Tensor, down: torch.Tensor):
+        if gate_up.dtype != torch.bfloat16 or down.dtype != torch.bfloat16 or not (gate_up.is_cuda and down.is_cuda):
+            raise ValueError("shared expert weights must be bf16 CUDA tensors")
+        if gate_up.dim() != 2 or down.dim() != 2 or gate_up.shape[0] % 2 or down.shape != (gate_up.shape[1],
+                                                                                          gate_up.shape[0] // 2):
+            raise ValueError("shared expert shapes: gate_up [2I, H], down [H, I]")
+        self.gate_up, self.down = gate_up.contiguous(), down.contiguous()
+        self.I = gate_up.shape[0] // 2
+
+    def struct(self) -> _SharedStruct:
+        return _SharedStruct(self.I, self.gate_up.data_ptr(), self.down.data_ptr())
+
+
+def forward_ex_workspace(layer: Layer, shared, T: int, k: int) -> int:
+    sh = ctypes.byref(shared.struct()) if shared is not None else None
+    return int(lib().moe_q4_forward_ex_workspace(ctypes.byref(layer.struct()), sh, T, k))
+
+
+def forward_ex(layer: Layer, shared, x: torch.Tensor, logits: torch.Tensor, k: int, out=None, ws=None,
+               topk_ids=None, topk_w=None, counts=None, out_f32=None, stream=None) -> torch.Tensor:
+    """One MoE layer with a shared expert (shared may be None)."""
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, layer.H), dtype=torch.bfloat16, device=x.device)
+    own_ws = ws is None
+    if own_ws:
+        ws = alloc_workspace(forward_ex_workspace(layer, shared, T, k), x.device)
+    st = layer.struct()
+    ss = shared.struct() if shared is not None else None
+    _check(lib().moe_q4_forward_ex(ctypes.byref(st), ctypes.byref(ss) if ss is not None else None, _ptr(x),
+                                   _ptr(logits), T, k, _ptr(out), _ptr(out_f32), _ptr(topk_ids), _ptr(topk_w),
+                                   _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)), "moe_q4_forward_ex")
     if own_ws:
         _hold(stream, ws)
     return out

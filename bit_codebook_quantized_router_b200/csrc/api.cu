@@ -65,11 +65,18 @@ bool shape_ok(const moe_q4_layer* L, int T, int top_k) {
 //   gate/up then down)
 struct Layout {
   size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, tiles, h, h_lo, y, xg, dk_counter,
-      dk_partial, end;
+      dk_partial, h_s, y_s, sx_partial, end;
   int dk_units_gu, dk_units_dn, n_max;
 };
 
-Layout layout(const moe_q4_layer* L, int T, int k) {
+bool shared_ok(const moe_q4_layer* L, const moe_q4_shared* S) {
+  if (!S) return true;
+  if (S->I <= 0 || (S->I % 128) || !S->gate_up || !S->down) return false;
+  if (((uintptr_t)S->gate_up & 15) || ((uintptr_t)S->down & 15)) return false;
+  return L->H % 64 == 0;
+}
+
+Layout layout(const moe_q4_layer* L, int T, int k, const moe_q4_shared* S = nullptr) {
   const size_t R = (size_t)T * k;
   Layout o;
   size_t p = 0;
@@ -113,6 +120,17 @@ Layout layout(const moe_q4_layer* L, int T, int k) {
   p = align_up(p + sizeof(int32_t) * (size_t)(o.dk_units_gu + o.dk_units_dn) * kDkSlabs);
   o.dk_partial = p;
   p = align_up(p + sizeof(float) * (size_t)2 * kDkMaxGrid * 4 * o.n_max * 128);  // 2 tiles per unit, both kernels
+  // shared expert: h_s bf16 [T][I_s] | y_s f32 [T][H] | split-K partial sums
+  o.h_s = o.y_s = o.sx_partial = 0;
+  if (S) {
+    o.h_s = p;
+    p = align_up(p + sizeof(__nv_bfloat16) * (size_t)T * S->I);
+    o.y_s = p;
+    p = align_up(p + sizeof(float) * (size_t)T * L->H);
+    const size_t pa = q4_dense_partial_bytes(T, S->I, L->H, 2), pb = q4_dense_partial_bytes(T, L->H, S->I, 1);
+    o.sx_partial = p;
+    p = align_up(p + (pa > pb ? pa : pb));
+  }
   o.end = p;
   return o;
 }
@@ -137,8 +155,9 @@ HostStage host_stage(const moe_q4_layer* L, int T, size_t base) {
 
 int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, const float* logits,
                 int T, int k, void* out, float* out_f32, int32_t* topk_ids, float* topk_w,
-                int32_t* counts, char* ws, cudaStream_t s, void* const* events = nullptr) {
-  const Layout o = layout(L, T, k);
+                int32_t* counts, char* ws, cudaStream_t s, void* const* events = nullptr,
+                const moe_q4_shared* S = nullptr) {
+  const Layout o = layout(L, T, k, S);
   FwdArgs a;
   memset(&a, 0, sizeof a);
   a.T = T;
@@ -168,6 +187,7 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   a.h_lo = (__nv_bfloat16*)(ws + o.h_lo);
   a.y = (float*)(ws + o.y);
   a.out_f32 = out_f32;
+  a.y_s = S ? (const float*)(ws + o.y_s) : nullptr;
   a.user_ids = topk_ids;
   a.user_w = topk_w;
   a.user_counts = counts;
@@ -203,6 +223,16 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, false, s);
   if (rc == MOE_Q4_OK) rc = mark(5);
   if (rc == MOE_Q4_OK) rc = q4_launch_decode(a, tp, false, part_dn, cnt_dn, grid, s);
+  if (rc == MOE_Q4_OK && S) {
+    // the shared expert: merged gate+up with the SwiGLU, then down (its time
+    // falls between events 6 and 7, with the combine)
+    __nv_bfloat16* h_s = (__nv_bfloat16*)(ws + o.h_s);
+    float* y_s = (float*)(ws + o.y_s);
+    float* part = (float*)(ws + o.sx_partial);
+    rc = q4_launch_dense(S->gate_up, 2, S->I, S->I, L->H, x, T, h_s, nullptr, S->I, part, a.hdr + kStatus, s);
+    if (rc == MOE_Q4_OK)
+      rc = q4_launch_dense(S->down, 1, 0, L->H, S->I, h_s, T, nullptr, y_s, L->H, part, a.hdr + kStatus, s);
+  }
   if (rc == MOE_Q4_OK) rc = mark(6);
   if (rc == MOE_Q4_OK) rc = q4_launch_combine(a, s);
   if (rc == MOE_Q4_OK) rc = mark(7);
@@ -273,6 +303,32 @@ extern "C" int moe_q4_forward(const moe_q4_layer* layer, const void* x, const fl
     return MOE_Q4_EWORKSPACE;
   return run_forward(layer, tp, x, logits, T, top_k, out, out_f32, topk_ids, topk_w, counts,
                      (char*)ws, (cudaStream_t)stream);
+}
+
+extern "C" size_t moe_q4_forward_ex_workspace(const moe_q4_layer* layer, const moe_q4_shared* shared, int T,
+                                              int top_k) {
+  if (!shape_ok(layer, T, top_k) || !shared_ok(layer, shared)) return 0;
+  return layout(layer, T, top_k, shared).end;
+}
+
+extern "C" int moe_q4_forward_ex(const moe_q4_layer* layer, const moe_q4_shared* shared, const void* x,
+                                 const float* logits, int T, int top_k, void* out, float* out_f32,
+                                 int32_t* topk_ids, float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  if (!shared)
+    return moe_q4_forward(layer, x, logits, T, top_k, out, out_f32, topk_ids, topk_w, counts, ws, ws_bytes, stream);
+  if (!shape_ok(layer, T, top_k) || !shared_ok(layer, shared)) return MOE_Q4_EINVAL;
+  TableParams tp;
+  int rc = q4_fill_tables(&tp, layer->tables, layer->n_tables, layer->table_id, layer->E);
+  if (rc != MOE_Q4_OK) return rc;
+  if (T == 0) return MOE_Q4_OK;
+  if (!x || !logits || !out || ((uintptr_t)x & 15) || ((uintptr_t)out & 15) || ((uintptr_t)logits & 3) ||
+      ((uintptr_t)out_f32 & 15))
+    return MOE_Q4_EINVAL;
+  if (!ws || ((uintptr_t)ws & (kAlign - 1)) || ws_bytes < layout(layer, T, top_k, shared).end)
+    return MOE_Q4_EWORKSPACE;
+  return run_forward(layer, tp, x, logits, T, top_k, out, out_f32, topk_ids, topk_w, counts, (char*)ws,
+                     (cudaStream_t)stream, nullptr, shared);
 }
 
 extern "C" int moe_q4_forward_stages(const moe_q4_layer* layer, const void* x, const float* logits,

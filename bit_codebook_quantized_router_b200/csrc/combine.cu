@@ -2,7 +2,8 @@
 //   out[t] = sum_{j=0..k-1} w[t][j] * y[inv[t][j]]
 // ("GLM-5.2 EXL3 TR3 v4" README, "Shared residual rotations, private
 // intermediate rotations": expert outputs are routing-weighted and summed
-// back into the residual space).  Each output element is summed by one
+// back into the residual space), plus the shared expert's output when the
+// layer has one.  Each output element is summed by one
 // thread in slot order in fp32, then rounded to bf16: deterministic, no
 // atomics.
 #include "q4_api_internal.h"
@@ -25,6 +26,14 @@ __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ Fw
     acc.y = fmaf(wj, v.y, acc.y);
     acc.z = fmaf(wj, v.z, acc.z);
     acc.w = fmaf(wj, v.w, acc.w);
+  }
+  if (a.y_s) {
+    // the shared expert's output, weight 1, after the routed slots
+    const float4 v = *reinterpret_cast<const float4*>(a.y_s + (size_t)t * a.H + n4);
+    acc.x += v.x;
+    acc.y += v.y;
+    acc.z += v.z;
+    acc.w += v.w;
   }
   if (a.out_f32) *reinterpret_cast<float4*>(a.out_f32 + (size_t)t * a.H + n4) = acc;
   __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);

@@ -33,6 +33,7 @@ struct FwdArgs {
   __nv_bfloat16* h_lo;     // [T*k][I] bf16 rounding of the remainder silu(g)*u - h
   float* y;                // [T*k][H]
   float* out_f32;          // optional [T][H] fp32 combine result
+  const float* y_s;        // optional [T][H] shared-expert output, added by the combine
   __nv_bfloat16* xg;       // [T*k][H] expert-grouped activations
   int32_t* dk_counter;     // [dk_counter_n] split-tile arrival counters (small-M path)
   int dk_counter_n;
@@ -55,5 +56,10 @@ int q4_launch_prefill(const q4::FwdArgs& a, const q4::TableParams& tp, bool gate
 int q4_prefill_tile_n();
 int q4_launch_decode(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, float* partial,
                         int32_t* counter, int grid, cudaStream_t s);
+// Dense bf16 GEMM on the tensor cores (shared.cu): see q4_launch_dense.
+size_t q4_dense_partial_bytes(int T, int rows, int K, int mats);
+int q4_launch_dense(const void* w, int mats, int mat1_off, int rows, int K, const void* act, int T,
+                    __nv_bfloat16* out_bf16, float* out_f32, int ld, float* partial, int32_t* status,
+                    cudaStream_t s);
 int q4_forward_in_workspace(const moe_q4_layer* layer, const void* x, const float* logits, int T, int top_k,
                             void* out, float* out_f32, void* ws, size_t ws_bytes, cudaStream_t stream);

@@ -154,6 +154,19 @@ def expert_weight(w: Workload, e: int, proj: str, device="cpu") -> torch.Tensor:
     return (t * WEIGHT_STD).to(torch.bfloat16)
 
 
+def shared_expert_weights(w: Workload, I: int | None = None, device="cpu"):
+    """BF16 shared expert of the workload's layer: (gate_up [2I, H], down
+    [H, I]), N(0, 0.02), gate rows first; I defaults to the routed experts'
+    intermediate size (the GLM-5.2 shared expert's, 75.5 MB of BF16 per
+    layer at H = 6144)."""
+    I = w.shape.I if I is None else I
+    H = w.shape.H
+    g = _gen(w.seed_weights * 7919 + 11, device)
+    gu = torch.randn((2 * I, H), generator=g, device=device, dtype=torch.float32) * WEIGHT_STD
+    dn = torch.randn((H, I), generator=g, device=device, dtype=torch.float32) * WEIGHT_STD
+    return gu.to(torch.bfloat16).contiguous(), dn.to(torch.bfloat16).contiguous()
+
+
 def activations(w: Workload, device="cpu", T: int | None = None, variant: int = 0) -> torch.Tensor:
     """bf16 [T, H] activations, N(0, 1); `variant` > 0 draws another batch."""
     T = w.T if T is None else T

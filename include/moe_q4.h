@@ -199,6 +199,38 @@ MOE_Q4_API int moe_q4_forward(const moe_q4_layer* layer, const void* x, const fl
                               float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
                               void* stream);
 
+/* ---------------------------------------------------------------------------
+ * A shared expert beside the routed ones ("GLM-5.2 EXL3 TR3 v4" README,
+ * "Checkpoint layout update"; HF discussion #2 "Store shared experts in
+ * BF16"): the shared-expert MLP kept as its original BF16 weights, gate and
+ * up concatenated into one payload so that one launch computes both.
+ * Every token goes through it with weight 1:
+ *   out[t] = sum_j w_j * y_j[t] + Wd (silu(Wg x_t) * (Wu x_t)).
+ * ------------------------------------------------------------------------- */
+typedef struct moe_q4_shared {
+  int I;                 /* intermediate size of the shared expert, % 128 == 0 */
+  const void* gate_up;   /* device bf16 [2I][H], 16-byte aligned: rows 0..I-1 the
+                            gate, rows I..2I-1 the up projection */
+  const void* down;      /* device bf16 [H][I], 16-byte aligned */
+} moe_q4_shared;
+
+/* Workspace of moe_q4_forward_ex (0 if the arguments are invalid); with
+ * shared == NULL it equals moe_q4_forward_workspace. */
+MOE_Q4_API size_t moe_q4_forward_ex_workspace(const moe_q4_layer* layer, const moe_q4_shared* shared, int T,
+                                              int top_k);
+
+/* moe_q4_forward plus the shared expert (shared may be NULL: then exactly
+ * moe_q4_forward).  The shared expert runs on the tensor cores in two
+ * launches (merged gate+up with the SwiGLU, then down; at decode sizes each
+ * splits its K range over the SMs and adds the split partial sums in a fixed
+ * order), and the combine adds its output after the k routed slots, in fp32:
+ * deterministic.  Arguments and errors as for moe_q4_forward; the workspace
+ * must hold moe_q4_forward_ex_workspace(layer, shared, T, top_k) bytes. */
+MOE_Q4_API int moe_q4_forward_ex(const moe_q4_layer* layer, const moe_q4_shared* shared, const void* x,
+                                 const float* logits, int T, int top_k, void* out, float* out_f32,
+                                 int32_t* topk_ids, float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                                 void* stream);
+
 /* Synchronise `stream`, then return the status recorded in the workspace by
  * the last moe_q4_forward on it (MOE_Q4_OK, MOE_Q4_EDEVICE, MOE_Q4_ETIMEOUT),
  * or MOE_Q4_ECUDA if the stream itself reports an error. */

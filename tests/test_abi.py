@@ -139,3 +139,16 @@ def test_lloyd_host_checks(L):
     assert L.moe_q4_lloyd_solve(g.ctypes.data, -1, 0.0, out, out, fake, ws_n, None) == _lib.EINVAL
     assert L.moe_q4_lloyd_solve(g.ctypes.data, 5, -1.0, out, out, fake, ws_n, None) == _lib.EINVAL
     assert L.moe_q4_lloyd_solve(g.ctypes.data, 5, 0.0, None, out, fake, ws_n, None) == _lib.EINVAL
+
+
+def test_shared_expert_host_checks(L):
+    st, keep = _layer()
+    base = L.moe_q4_forward_workspace(ctypes.byref(st), 4, 2)
+    assert L.moe_q4_forward_ex_workspace(ctypes.byref(st), None, 4, 2) == base
+    ok = _lib._SharedStruct(128, 1 << 20, 1 << 21)
+    assert L.moe_q4_forward_ex_workspace(ctypes.byref(st), ctypes.byref(ok), 4, 2) > base
+    for bad in (_lib._SharedStruct(96, 1 << 20, 1 << 21), _lib._SharedStruct(128, 0, 1 << 21),
+                _lib._SharedStruct(128, (1 << 20) + 8, 1 << 21), _lib._SharedStruct(0, 1 << 20, 1 << 21)):
+        assert L.moe_q4_forward_ex_workspace(ctypes.byref(st), ctypes.byref(bad), 4, 2) == 0
+        assert L.moe_q4_forward_ex(ctypes.byref(st), ctypes.byref(bad), None, None, 4, 2, None, None, None, None,
+                                   None, None, 0, None) == _lib.EINVAL
