@@ -538,13 +538,17 @@ def measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream, reps=20):
     gbs = nbytes / (ms / 1e3) / 1e9
     tfs = flop / (ms / 1e3) / 1e12
     hbm_bound = T <= 256
-    kernel = ("router_few_kernel (one clustered launch)" if T <= 32 and sh.H % 128 == 0
-              else "router_kernel" + (" + router_reduce_kernel (K split)" if need else ""))
+    if T <= 32 and sh.H % 128 == 0:
+        kernel, how = "router_few_kernel (one clustered launch)", "mma.sync bf16"
+    elif sh.E % 128 == 0 and sh.H % 64 == 0:
+        kernel, how = "sx_gemm_kernel<1> (tcgen05 dense GEMM) + sx_reduce_kernel (K split)", "tcgen05 bf16"
+    else:
+        kernel, how = "router_kernel" + (" + router_reduce_kernel (K split)" if need else ""), "mma.sync bf16"
     return {"kernel": kernel, "ms": ms, "bytes": nbytes,
             "flop": flop, "gbs": gbs, "tflops": tfs, "bound": "hbm" if hbm_bound else "tensor",
             "frac": gbs / hbm_peak if hbm_bound else tfs / tf_peak,
             "frac_of_datasheet": gbs / DATASHEET_HBM_GBS if hbm_bound else tfs / DATASHEET_BF16_TFLOPS,
-            "note": "mma.sync bf16 GEMM; not part of the step (the layer's input is the logits)"}
+            "note": how + " GEMM; not part of the step (the layer's input is the logits)"}
 
 
 def measure_workload(q4, w, args, steps, warmup, world, dev, local, stream, flush_l2, barrier, full):

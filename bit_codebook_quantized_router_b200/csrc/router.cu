@@ -253,8 +253,16 @@ static int router_few_cluster(int chunks) {
   return c < 1 ? 1 : (c > 8 ? 8 : c);
 }
 
+// Above the decode sizes, with E a multiple of 128 and H of 64, the gate runs
+// as a dense GEMM on the tensor cores (q4_launch_dense: tcgen05, fp32
+// accumulators in TMEM, K split over the SMs when there are few token tiles,
+// the split partial sums added in a fixed order).  Its workspace: a status
+// word (256 bytes) then the split partial sums.
+static bool router_dense(int T, int H, int E) { return !router_few(T, H) && T > 32 && E % 128 == 0 && H % 64 == 0; }
+
 extern "C" size_t moe_q4_router_workspace(int T, int H, int E) {
   if (!router_args_ok(T, H, E) || T == 0 || router_few(T, H)) return 0;
+  if (router_dense(T, H, E)) return 256 + q4_dense_partial_bytes(T, E, H, 1);
   const RouterPlan p = router_plan(T, H, E);
   return p.chunks > 1 ? sizeof(float) * (size_t)p.chunks * T * E : 0;
 }
@@ -296,6 +304,13 @@ extern "C" int moe_q4_router(const void* x, const void* w, int T, int H, int E, 
   }
   const size_t need = moe_q4_router_workspace(T, H, E);
   if (need > 0 && (!ws || ws_bytes < need || ((uintptr_t)ws & 15))) return MOE_Q4_EWORKSPACE;
+  if (router_dense(T, H, E)) {
+    if ((uintptr_t)ws & 255) return MOE_Q4_EWORKSPACE;
+    int32_t* status = reinterpret_cast<int32_t*>(ws);
+    if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_Q4_ECUDA;
+    float* part = need > 256 ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 256) : nullptr;
+    return q4_launch_dense(w, 1, 0, E, H, x, T, nullptr, logits, E, part, status, s);
+  }
   const long long units = (long long)p.e_tiles * p.t_tiles * p.chunks;
   const long long want = (units + rt::kWarps - 1) / rt::kWarps;
   const int grid = (int)(want < 148 * 8 ? want : 148 * 8);

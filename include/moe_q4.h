@@ -62,6 +62,15 @@ extern "C" {
 #define MOE_Q4_ETIMEOUT 4    /* a bounded device-side wait gave up */
 #define MOE_Q4_EDEVICE 5     /* the device flagged bad data (non-finite logit / weight) */
 #define MOE_Q4_ENOTSUP 6     /* a size beyond what this build supports */
+#define MOE_Q4_EBOUNDS 7     /* a device-side index check failed (debug build only, see below) */
+
+/* Debug build: libmoe_q4 compiled with MOE_Q4_DEBUG defined (the package's
+ * build step writes it as libmoe_q4_debug.so beside the release library)
+ * checks on the device every index it reads from a routing table or the
+ * workspace before using it (token and row numbers, expert ids, grouped-row
+ * offsets).  A failing check records MOE_Q4_EBOUNDS in the status word and
+ * skips the access; no kernel traps.  The release build makes no such checks
+ * and computes the same bits. */
 
 /* Limits of this build. */
 #define MOE_Q4_MAX_TABLES 16
@@ -130,9 +139,13 @@ MOE_Q4_API int moe_q4_dequant(const uint8_t* weight, const uint8_t* weight_scale
  *   T >= 0; H > 0, H % 32 == 0; E > 0;
  *   logits    device, fp32 [T][E] (out): the input of moe_q4_forward;
  *   ws        device workspace of at least moe_q4_router_workspace(T, H, E)
- *             bytes (16-byte aligned; may be NULL when that is 0, as it is
- *             for T <= 32 with H % 128 == 0), owned by the call until the
- *             enqueued work completes;
+ *             bytes (16-byte aligned, 256-byte aligned above T = 32; may be
+ *             NULL when that is 0, as it is for T <= 32 with H % 128 == 0),
+ *             owned by the call until the enqueued work completes.  Above
+ *             T = 32 with E % 128 == 0 and H % 64 == 0 the gate runs on the
+ *             tensor cores (tcgen05) and the workspace's first int32 is a
+ *             status word (MOE_Q4_ETIMEOUT if a bounded device wait gave up;
+ *             read it with moe_q4_read_status);
  *   ws_bytes  size of ws.
  * Returns MOE_Q4_EINVAL for bad sizes or pointers, MOE_Q4_EWORKSPACE for a
  * missing or short workspace; no host synchronisation, no allocation.
@@ -355,6 +368,19 @@ MOE_Q4_API int moe_q4_lloyd_hist(const void* w, long long n_blocks, const float*
                                  size_t ws_bytes, void* stream);
 MOE_Q4_API int moe_q4_lloyd_solve(const float* grid0, int max_iter, double tol, float* grid, int32_t* iters,
                                   const void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * moe_q4_selftest_wait -- test support: checks that a bounded device wait
+ * gives up and reports instead of hanging.  One CTA: a producer warp that
+ * issues nothing and a consumer warp waiting on the stage barrier it would
+ * have completed, with the same bounded wait and teardown as the layer's
+ * kernels.  After limit_us microseconds (1 .. 2,000,000) the wait gives up
+ * and MOE_Q4_ETIMEOUT is recorded in *status (device int32, left unchanged
+ * otherwise; it records only over MOE_Q4_OK).  The kernel returns normally:
+ * the context stays usable for the next call.  Not part of the layer; the
+ * pages have no counterpart.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API int moe_q4_selftest_wait(int32_t* status, unsigned limit_us, void* stream);
 
 /* Synchronise `stream` and return the int32 at device address `status`
  * (as written by moe_q4_pack), or MOE_Q4_ECUDA. */
