@@ -10,9 +10,10 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe_q4.so")
+# MOE_Q4_LIB=debug selects the bounds-checking build (libmoe_q4_debug.so)
+LIB_PATH = os.path.join(_HERE, "libmoe_q4_debug.so" if os.environ.get("MOE_Q4_LIB") == "debug" else "libmoe_q4.so")
 
-OK, EINVAL, ECUDA, EWORKSPACE, ETIMEOUT, EDEVICE, ENOTSUP = range(7)
+OK, EINVAL, ECUDA, EWORKSPACE, ETIMEOUT, EDEVICE, ENOTSUP, EBOUNDS = range(8)
 MAX_TABLES, MAX_EXPERTS, MAX_TOPK = 16, 512, 16
 
 
@@ -74,6 +75,8 @@ def lib():
         L.moe_q4_forward_ex.argtypes = [ctypes.POINTER(_LayerStruct), ctypes.POINTER(_SharedStruct), vp, vp, ci, ci,
                                         vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_q4_forward_ex.restype = ci
+        L.moe_q4_selftest_wait.argtypes = [vp, ctypes.c_uint, vp]
+        L.moe_q4_selftest_wait.restype = ci
         L.moe_q4_lloyd_workspace.argtypes = [vp]
         L.moe_q4_lloyd_workspace.restype = sz
         L.moe_q4_lloyd_hist.argtypes = [vp, ctypes.c_longlong, vp, ci, vp, sz, vp]
