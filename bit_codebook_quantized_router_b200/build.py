@@ -19,37 +19,50 @@ NVCC_FLAGS = [
 ]
 
 
+LIB_DEBUG = os.path.join(PKG, "libmoe_q4_debug.so")
+
+
 def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale():
-    if not os.path.exists(LIB):
+def _stale(lib):
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")) \
         + glob.glob(os.path.join(ROOT, "include", "*.h"))
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not _stale():
-        return LIB
+def _build_one(lib, objdir, flags, verbose):
+    from concurrent.futures import ThreadPoolExecutor
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-    objdir = os.path.join(PKG, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
-    for src in sources():
+
+    def compile_one(src):
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc, "-c", src, "-o", obj, *NVCC_FLAGS, *extra]
+        cmd = [nvcc, "-c", src, "-o", obj, *NVCC_FLAGS, *flags]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.check_call(cmd)
-        objs.append(obj)
-    tmp = LIB + f".tmp{os.getpid()}"
+        return obj
+
+    with ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
+        objs = list(ex.map(compile_one, sources()))
+    tmp = lib + f".tmp{os.getpid()}"
     subprocess.check_call([nvcc, "-shared", "-o", tmp, *objs, "-gencode", "arch=compute_100a,code=sm_100a",
                            "-Xcompiler", "-fPIC"])
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False, extra=(), debug: bool = True) -> str:
+    """Build the release library (and, with debug=True, the bounds-checking
+    debug library beside it: MOE_Q4_DEBUG defined)."""
+    if force or _stale(LIB):
+        _build_one(LIB, os.path.join(PKG, "_build"), list(extra), verbose)
+    if debug and (force or _stale(LIB_DEBUG)):
+        _build_one(LIB_DEBUG, os.path.join(PKG, "_build_debug"), ["-DMOE_Q4_DEBUG", *extra], verbose)
     return LIB
 
 

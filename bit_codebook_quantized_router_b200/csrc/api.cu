@@ -274,6 +274,7 @@ extern "C" const char* moe_q4_status_string(int status) {
     case MOE_Q4_ETIMEOUT: return "bounded device wait timed out";
     case MOE_Q4_EDEVICE: return "device detected invalid data (non-finite input)";
     case MOE_Q4_ENOTSUP: return "size not supported by this build";
+    case MOE_Q4_EBOUNDS: return "device index check failed (debug build)";
     default: return "unknown status";
   }
 }

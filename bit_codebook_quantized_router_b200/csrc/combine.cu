@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ Fw
   for (int j = 0; j < a.k; ++j) {
     const int r = a.inv[t * a.k + j];
     const float wj = a.w[t * a.k + j];
+    if (!q4_check((unsigned)r < (unsigned)(a.T * a.k), a.hdr + kStatus)) continue;
     const float4 v = *reinterpret_cast<const float4*>(a.y + (size_t)r * a.H + n4);
     acc.x = fmaf(wj, v.x, acc.x);
     acc.y = fmaf(wj, v.y, acc.y);

@@ -474,12 +474,14 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       const int unit = g / P.stages;
       const int st0 = g - unit * P.stages;
       const int seg_end = min(k1, (unit + 1) * P.stages);
-      const int e = unit_expert(unit);
+      int e = unit_expert(unit);
+      if (!q4_check((unsigned)e < (unsigned)a.E, a.hdr + kStatus)) e = 0;
       const int t = unit % P.tiles_per_e;
       const int wrow = e * rows_total + t * C::kUnitRows;
       // down: the unit's second row tile exists unless H is an odd number of 128s
       const bool two = GATEUP || t * C::kUnitRows + dk::kRows < rows_total;
       const int row0 = expert_row0(unit, e);
+      if (!q4_check(row0 >= 0 && row0 + expert_rows(e) <= a.T * a.k, a.hdr + kStatus)) break;
       // Activation rows by untiled bulk copies (a tiled TMA would need a
       // 128-byte-aligned destination), one per row and stage: the stage's
       // 32 * subs * 4 bytes of x[token] (gate/up, lane n: row n) or of h / h_lo
@@ -490,8 +492,11 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
       const __nv_bfloat16* my_src = nullptr;
       if (GATEUP) {
         if (lane < n_e) {
-          my_slot = lane;
-          my_src = a.x + (self ? (size_t)0 : (size_t)a.row_token[row0 + lane] * a.H);
+          const int tok = self ? 0 : a.row_token[row0 + lane];
+          if (q4_check((unsigned)tok < (unsigned)a.T, a.hdr + kStatus)) {
+            my_slot = lane;
+            my_src = a.x + (size_t)tok * a.H;
+          }
         }
       } else {
         const int n = lane & 15;
@@ -774,6 +779,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
           const int n = 8 * tt + 2 * tq + (i & 1);
           if (n >= n_e) continue;
           const size_t row = (size_t)row0 + n;
+          if (!q4_check(row < (size_t)a.T * a.k, a.hdr + kStatus)) continue;
           const int wr = tile * C::kUnitRows + ((i >> 1) ? r1 : r0);
           if (GATEUP) {
             const float hv = silu_mul(acc[0][tt][i], acc[1][tt][i]);

@@ -158,7 +158,8 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
         int p, m, nt;
         tile_coords(a, P.m_tiles, np, tile, p, m, nt);
-        const int e = a.pre_list[p];
+        int e = a.pre_list[p];
+        if (!q4_check((unsigned)e < (unsigned)a.E, a.hdr + kStatus)) e = 0;
         const int wrow = e * rows_total + m * kBM;
         const int brow = a.offsets[e] + nt * kBN;
         for (int ks = 0; ks < P.k_steps; ++ks, ++it) {
@@ -289,9 +290,12 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
     for (int tile = blockIdx.x; tile < total && !warp_aborted(abort_flag); tile += gridDim.x, ++tcount) {
       int p, m, nt;
       tile_coords(a, P.m_tiles, np, tile, p, m, nt);
-      const int e = a.pre_list[p];
-      const int n_e = a.counts[e];
+      int e = a.pre_list[p];
+      if (!q4_check((unsigned)e < (unsigned)a.E, a.hdr + kStatus)) e = 0;
+      int n_e = a.counts[e];
       const int row0 = a.offsets[e];
+      // (a failed check leaves the tile's rows unwritten)
+      if (!q4_check(row0 >= 0 && n_e >= 0 && row0 + n_e <= a.T * a.k, a.hdr + kStatus)) n_e = nt * kBN;
       const int buf = (int)(tcount % C::kAccBufs);
       const uint32_t use = tcount / C::kAccBufs;
       if (!mbar_wait_warp(&acc_full[buf], use & 1, abort_flag, kWaitLimitNs)) break;

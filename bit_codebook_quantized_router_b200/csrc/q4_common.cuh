@@ -42,6 +42,18 @@ __device__ __forceinline__ void record_error(int32_t* status, int code) {
   atomicCAS(reinterpret_cast<int*>(status), 0, code);
 }
 
+// Device-side index check of the debug build (MOE_Q4_DEBUG): true when `ok`;
+// else records MOE_Q4_EBOUNDS and the caller skips the access.  The release
+// build compiles it to `true`.
+#ifdef MOE_Q4_DEBUG
+__device__ __forceinline__ bool q4_check(bool ok, int32_t* status) {
+  if (!ok) record_error(status, MOE_Q4_EBOUNDS);
+  return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool q4_check(bool, int32_t*) { return true; }
+#endif
+
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));

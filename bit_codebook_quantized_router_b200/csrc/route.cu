@@ -291,6 +291,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant_
   for (int64_t v = blockIdx.x * 256 + threadIdx.x; v < n; v += (int64_t)gridDim.x * 256) {
     const int r = (int)(v / vec_per_row);
     const int q = (int)(v % vec_per_row);
+    if (!q4_check((unsigned)a.row_token[r] < (unsigned)a.T, a.hdr + kStatus)) continue;
     const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)a.row_token[r] * a.H) + q;
     reinterpret_cast<uint4*>(a.xg + (size_t)r * a.H)[q] = *src;
   }

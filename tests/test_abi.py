@@ -152,3 +152,13 @@ def test_shared_expert_host_checks(L):
         assert L.moe_q4_forward_ex_workspace(ctypes.byref(st), ctypes.byref(bad), 4, 2) == 0
         assert L.moe_q4_forward_ex(ctypes.byref(st), ctypes.byref(bad), None, None, 4, 2, None, None, None, None,
                                    None, None, 0, None) == _lib.EINVAL
+
+
+def test_debug_build_exports_every_declared_symbol(L):
+    from bit_codebook_quantized_router_b200 import build
+    assert os.path.exists(build.LIB_DEBUG)
+    D = ctypes.CDLL(build.LIB_DEBUG)
+    for s in declared_symbols():
+        assert hasattr(D, s), s
+    D.moe_q4_status_string.restype = ctypes.c_char_p
+    assert b"debug" in D.moe_q4_status_string(_lib.EBOUNDS)
