@@ -75,6 +75,8 @@ def lib():
         L.moe_q4_forward_ex.argtypes = [ctypes.POINTER(_LayerStruct), ctypes.POINTER(_SharedStruct), vp, vp, ci, ci,
                                         vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_q4_forward_ex.restype = ci
+        L.moe_q4_combine.argtypes = [vp, vp, vp, ci, ci, ci, vp, vp, vp]
+        L.moe_q4_combine.restype = ci
         L.moe_q4_selftest_wait.argtypes = [vp, ctypes.c_uint, vp]
         L.moe_q4_selftest_wait.restype = ci
         L.moe_q4_lloyd_workspace.argtypes = [vp]
@@ -367,3 +369,17 @@ def lloyd_fit(weights, grid0, max_iter: int = 300, tol: float = 1e-12, stream=No
     _hold(stream, ws)
     status = int(lib().moe_q4_read_status(_ptr(ws), _stream(stream)))
     return grid, iters, status
+
+
+def combine(y: torch.Tensor, w: torch.Tensor, inv=None, out=None, out_f32=None, stream=None) -> torch.Tensor:
+    """Weighted combine: y fp32 [T*k, H] (rows in (token, slot) order unless
+    inv [T, k] places them), w fp32 [T, k] -> bf16 [T, H]."""
+    T, k = w.shape
+    H = y.shape[1]
+    if out is None:
+        out = torch.empty((T, H), dtype=torch.bfloat16, device=y.device)
+    y, w = y.contiguous(), w.contiguous()
+    _check(lib().moe_q4_combine(_ptr(y), _ptr(w), _ptr(inv), T, k, H, _ptr(out), _ptr(out_f32), _stream(stream)),
+           "moe_q4_combine")
+    _hold(stream, y, w)
+    return out

@@ -6,6 +6,8 @@
 // layer has one.  Each output element is summed by one
 // thread in slot order in fp32, then rounded to bf16: deterministic, no
 // atomics.
+#include <string.h>
+
 #include "q4_api_internal.h"
 #include "q4_common.cuh"
 
@@ -19,9 +21,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ Fw
   for (int t = blockIdx.y; t < a.T; t += gridDim.y) {
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int j = 0; j < a.k; ++j) {
-    const int r = a.inv[t * a.k + j];
+    // (no inverse map: the rows are in (token, slot) order)
+    const int r = a.inv ? a.inv[t * a.k + j] : t * a.k + j;
     const float wj = a.w[t * a.k + j];
-    if (!q4_check((unsigned)r < (unsigned)(a.T * a.k), a.hdr + kStatus)) continue;
+    if (!q4_check((unsigned)r < (unsigned)(a.T * a.k), a.hdr ? a.hdr + kStatus : nullptr)) continue;
     const float4 v = *reinterpret_cast<const float4*>(a.y + (size_t)r * a.H + n4);
     acc.x = fmaf(wj, v.x, acc.x);
     acc.y = fmaf(wj, v.y, acc.y);
@@ -62,4 +65,26 @@ int q4_launch_combine(const FwdArgs& a, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, combine_kernel, a) == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
+}
+
+// The combine alone: y fp32 [T*k][H] (rows in (token, slot) order, or placed
+// by inv), w fp32 [T][k] -> out bf16 [T][H] and optionally out_f32.
+extern "C" int moe_q4_combine(const float* y, const float* w, const int32_t* inv, int T, int k, int H, void* out,
+                              float* out_f32, void* stream) {
+  if (T < 0 || k < 1 || k > MOE_Q4_MAX_TOPK || H <= 0 || H % 4) return MOE_Q4_EINVAL;
+  if (T == 0) return MOE_Q4_OK;
+  if (!y || !w || !out || ((uintptr_t)y & 15) || ((uintptr_t)out & 7) || ((uintptr_t)out_f32 & 15) ||
+      ((uintptr_t)w & 3))
+    return MOE_Q4_EINVAL;
+  FwdArgs a;
+  memset(&a, 0, sizeof a);
+  a.T = T;
+  a.k = k;
+  a.H = H;
+  a.y = const_cast<float*>(y);
+  a.w = const_cast<float*>(w);
+  a.inv = const_cast<int32_t*>(inv);
+  a.out = (__nv_bfloat16*)out;
+  a.out_f32 = out_f32;
+  return q4_launch_combine(a, (cudaStream_t)stream);
 }

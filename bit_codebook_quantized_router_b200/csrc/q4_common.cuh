@@ -39,7 +39,7 @@ enum HeaderWord : int {
 };
 
 __device__ __forceinline__ void record_error(int32_t* status, int code) {
-  atomicCAS(reinterpret_cast<int*>(status), 0, code);
+  if (status) atomicCAS(reinterpret_cast<int*>(status), 0, code);
 }
 
 // Device-side index check of the debug build (MOE_Q4_DEBUG): true when `ok`;

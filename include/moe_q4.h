@@ -370,6 +370,20 @@ MOE_Q4_API int moe_q4_lloyd_solve(const float* grid0, int max_iter, double tol, 
                                   const void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * moe_q4_combine -- the layer's weighted combine alone (used by the expert-
+ * parallel forward, where the expert outputs come back from other ranks):
+ *   out[t] = sum_{j<k} w[t][j] * y[r(t, j)],  r(t, j) = inv ? inv[t*k+j] : t*k+j,
+ * summed in slot order in fp32, rounded to bf16 (the same arithmetic as the
+ * forward's combine: deterministic).
+ *   y        device fp32 [T*k][H], 16-byte aligned;   w  device fp32 [T][k];
+ *   inv      optional device int32 [T][k] (NULL: rows in (token, slot) order);
+ *   out      device bf16 [T][H] (out);  out_f32  optional device fp32 [T][H];
+ *   H % 4 == 0, 1 <= k <= MOE_Q4_MAX_TOPK.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API int moe_q4_combine(const float* y, const float* w, const int32_t* inv, int T, int k, int H, void* out,
+                              float* out_f32, void* stream);
+
+/* ---------------------------------------------------------------------------
  * moe_q4_selftest_wait -- test support: checks that a bounded device wait
  * gives up and reports instead of hanging.  One CTA: a producer warp that
  * issues nothing and a consumer warp waiting on the stage barrier it would
