@@ -510,6 +510,43 @@ def measure_lloyd(q4, w, hbm_peak, flush_l2, stream, reps=3, max_iter=100):
             "frac_of_datasheet": gbs / DATASHEET_HBM_GBS, "status_ok": bool(ok)}
 
 
+def measure_shared(q4, w, layer, xs, lgs, hbm_peak, flush_l2, stream, steps=50):
+    """The layer with its BF16 shared expert (moe_q4_forward_ex): the same
+    steps back to back; bytes = the routed experts touched + the shared
+    expert's BF16 weights (3 I H * 2) + x and out."""
+    sh = w.shape
+    gu, dn = inputs.shared_expert_weights(w, device="cuda")
+    shared = q4.Shared(gu, dn)
+    T, k = w.T, sh.k
+    ws = q4.alloc_workspace(q4.forward_ex_workspace(layer, shared, T, k))
+    out = torch.empty((T, sh.H), dtype=torch.bfloat16, device="cuda")
+    for i in range(5):
+        q4.forward_ex(layer, shared, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)
+    torch.cuda.synchronize()
+    ok = q4.forward_status(ws) == 0
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    # back to back behind a device-side sleep, as the main timed loop: the host
+    # enqueues every step before the GPU reaches the first
+    torch.cuda._sleep(int(steps * 400_000))
+    a.record(stream)
+    for i in range(steps):
+        q4.forward_ex(layer, shared, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    touched = float(np.mean([torch.unique(torch.topk(l, k, dim=1).indices).numel() for l in lgs]))
+    gu_b, dn_b = expert_bytes(sh)
+    nbytes = touched * (gu_b + dn_b) + 3 * sh.I * sh.H * 2 + T * sh.H * 2 * 2
+    gbs = nbytes / (ms / 1e3) / 1e9
+    del ws, shared, gu, dn
+    return {"kernel": "forward with the shared expert: routed kernels + sx_gemm_kernel<2> (merged gate+up, SwiGLU) + "
+                      "sx_gemm_kernel<1> (down) (+ split reduction) + combine",
+            "ms_per_step": ms, "value": T / (ms / 1e3), "unit": UNIT, "bytes_per_step": nbytes, "gbs": gbs,
+            "frac_of_peak": gbs / hbm_peak, "status_ok": bool(ok),
+            "shared_bytes": 3 * sh.I * sh.H * 2}
+
+
 def measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream, reps=20):
     """The router gate ahead of the layer (moe_q4_router): bf16 x [T, H] times
     the bf16 gate [E, H] -> fp32 logits.  Algorithmic work: the gate and x read
@@ -524,15 +561,17 @@ def measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream, reps=20):
     for i in range(3):
         q4.router(xs[i % len(xs)], gate, out=out, ws=ws)
     torch.cuda.synchronize()
-    st = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
-    en = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    # back to back behind a device-side sleep (the host enqueues every call
+    # before the GPU reaches the first: its launch overhead is not timed);
+    # the rotating x batches and the 3 MB gate stay in L2 between calls
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(reps * 400_000))
+    a.record(stream)
     for i in range(reps):
-        flush_l2(i)
-        st[i].record(stream)
         q4.router(xs[i % len(xs)], gate, out=out, ws=ws)
-        en[i].record(stream)
+    b.record(stream)
     torch.cuda.synchronize()
-    ms = sum(a.elapsed_time(b) for a, b in zip(st, en)) / reps
+    ms = a.elapsed_time(b) / reps
     nbytes = sh.E * sh.H * 2 + T * sh.H * 2 + T * sh.E * 4
     flop = 2.0 * T * sh.E * sh.H
     gbs = nbytes / (ms / 1e3) / 1e9
@@ -675,6 +714,9 @@ def measure_workload(q4, w, args, steps, warmup, world, dev, local, stream, flus
         "gpu_launches": kernels_per_step * steps,
         "clocks": clk.summary(),
     }
+    res["router"] = measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream)
+    res["shared_expert"] = measure_shared(q4, w, layer, xs, lgs, hbm_peak, flush_l2, stream,
+                                          steps=min(steps, 50))
     if full:
         res["flushed"] = {"value": T * world / (flushed_ms / 1e3), "unit": UNIT, "ms_per_step": flushed_ms,
                           "steps": n_fl,
@@ -684,7 +726,6 @@ def measure_workload(q4, w, args, steps, warmup, world, dev, local, stream, flus
                          "note": "same forward replayed from CUDA graphs, L2 flushed outside the events"}
                         if graph_ms else {"value": None, "unavailable": graph_why})
         res["dequant"] = measure_dequant(q4, layer, hbm_peak, flush_l2, stream) if not args.no_dequant else None
-        res["router"] = measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream)
         if not args.no_lloyd:
             res["lloyd"] = measure_lloyd(q4, w, hbm_peak, flush_l2, stream)
         res["_cpu_inputs"] = (inputs.bf16_bits(xs[0]), lgs[0].cpu().numpy())
