@@ -559,6 +559,45 @@ def measure_shared(q4, w, layer, xs, lgs, hbm_peak, flush_l2, stream, steps=50):
             "shared_bytes": 3 * sh.I * sh.H * 2}
 
 
+def measure_gated(q4, w, layer, xs, stream, steps=50):
+    """The layer from the hidden states (moe_q4_forward_gated): the bf16
+    router gate, the routing and the routed experts, steps back to back.
+    The logits-input forward is timed on the same router logits (the same
+    routing) beside it: `router_added_ms` is the difference."""
+    sh = w.shape
+    gate = inputs.router_weight(w, device="cuda")
+    T, k = w.T, sh.k
+    ws = q4.alloc_workspace(q4.forward_gated_workspace(layer, None, T, k))
+    out = torch.empty((T, sh.H), dtype=torch.bfloat16, device="cuda")
+    lgs = [q4.router(x, gate) for x in xs]
+    runs = {"gated": lambda i: q4.forward_gated(layer, None, gate, xs[i % ROTATE], k, out=out, ws=ws),
+            "plain": lambda i: q4.forward(layer, xs[i % ROTATE], lgs[i % ROTATE], k, out=out, ws=ws)}
+    ms = {}
+    for name, run in runs.items():
+        for i in range(5):
+            run(i)
+        torch.cuda.synchronize()
+        assert q4.forward_status(ws) == 0
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(int(steps * 400_000))
+        a.record(stream)
+        for i in range(steps):
+            run(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms[name] = a.elapsed_time(b) / steps
+    ok = q4.forward_status(ws) == 0
+    touched = float(np.mean([torch.unique(torch.topk(l, k, dim=1).indices).numel() for l in lgs]))
+    fused = T <= 32 and sh.H % 128 == 0 and T * k <= 4096
+    first = ("router_route_kernel (router gate + routing + grouping, one clustered launch)" if fused else
+             "router kernels, then the routing kernels")
+    del ws, gate, out, lgs
+    return {"kernel": first + ", then the layer's kernels", "ms_per_step": ms["gated"],
+            "value": T / (ms["gated"] / 1e3), "unit": UNIT, "logits_input_ms_per_step": ms["plain"],
+            "router_added_ms": ms["gated"] - ms["plain"], "touched_experts": touched, "status_ok": bool(ok),
+            "note": "routing from a random bf16 gate (no Zipf skew); both steps on the same logits"}
+
+
 def measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream, reps=20):
     """The router gate ahead of the layer (moe_q4_router): bf16 x [T, H] times
     the bf16 gate [E, H] -> fp32 logits.  Algorithmic work: the gate and x read
@@ -744,6 +783,7 @@ def measure_workload(q4, w, args, steps, warmup, world, dev, local, stream, flus
     res["router"] = measure_router(q4, w, xs, hbm_peak, tf_peak, flush_l2, stream)
     res["shared_expert"] = measure_shared(q4, w, layer, xs, lgs, hbm_peak, flush_l2, stream,
                                           steps=min(steps, 50))
+    res["gated"] = measure_gated(q4, w, layer, xs, stream, steps=min(steps, 50))
     if full:
         res["flushed"] = {"value": T * world / (flushed_ms / 1e3), "unit": UNIT, "ms_per_step": flushed_ms,
                           "steps": n_fl,

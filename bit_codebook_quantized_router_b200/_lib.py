@@ -75,6 +75,12 @@ def lib():
         L.moe_q4_forward_ex.argtypes = [ctypes.POINTER(_LayerStruct), ctypes.POINTER(_SharedStruct), vp, vp, ci, ci,
                                         vp, vp, vp, vp, vp, vp, sz, vp]
         L.moe_q4_forward_ex.restype = ci
+        L.moe_q4_forward_gated_workspace.argtypes = [ctypes.POINTER(_LayerStruct), ctypes.POINTER(_SharedStruct),
+                                                     ci, ci]
+        L.moe_q4_forward_gated_workspace.restype = sz
+        L.moe_q4_forward_gated.argtypes = [ctypes.POINTER(_LayerStruct), ctypes.POINTER(_SharedStruct), vp, vp, ci,
+                                           ci, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.moe_q4_forward_gated.restype = ci
         L.moe_q4_combine.argtypes = [vp, vp, vp, ci, ci, ci, vp, vp, vp]
         L.moe_q4_combine.restype = ci
         L.moe_q4_selftest_wait.argtypes = [vp, ctypes.c_uint, vp]
@@ -266,6 +272,35 @@ def forward_ex(layer: Layer, shared, x: torch.Tensor, logits: torch.Tensor, k: i
     _check(lib().moe_q4_forward_ex(ctypes.byref(st), ctypes.byref(ss) if ss is not None else None, _ptr(x),
                                    _ptr(logits), T, k, _ptr(out), _ptr(out_f32), _ptr(topk_ids), _ptr(topk_w),
                                    _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)), "moe_q4_forward_ex")
+    if own_ws:
+        _hold(stream, ws)
+    return out
+
+
+def forward_gated_workspace(layer: Layer, shared, T: int, k: int) -> int:
+    sh = ctypes.byref(shared.struct()) if shared is not None else None
+    return int(lib().moe_q4_forward_gated_workspace(ctypes.byref(layer.struct()), sh, T, k))
+
+
+def forward_gated(layer: Layer, shared, router_w: torch.Tensor, x: torch.Tensor, k: int, out=None, ws=None,
+                  logits=None, topk_ids=None, topk_w=None, counts=None, out_f32=None, stream=None) -> torch.Tensor:
+    """One MoE layer from the hidden states: the bf16 router gate router_w
+    [E, H] computes the logits (into `logits` [T, E] fp32 when given), then
+    the layer as forward_ex (shared may be None)."""
+    if router_w.dtype != torch.bfloat16 or tuple(router_w.shape) != (layer.E, layer.H):
+        raise ValueError(f"router_w must be bf16 [{layer.E}, {layer.H}]")
+    T = x.shape[0]
+    if out is None:
+        out = torch.empty((T, layer.H), dtype=torch.bfloat16, device=x.device)
+    own_ws = ws is None
+    if own_ws:
+        ws = alloc_workspace(forward_gated_workspace(layer, shared, T, k), x.device)
+    st = layer.struct()
+    ss = shared.struct() if shared is not None else None
+    _check(lib().moe_q4_forward_gated(ctypes.byref(st), ctypes.byref(ss) if ss is not None else None,
+                                      _ptr(router_w), _ptr(x), T, k, _ptr(out), _ptr(out_f32), _ptr(logits),
+                                      _ptr(topk_ids), _ptr(topk_w), _ptr(counts), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "moe_q4_forward_gated")
     if own_ws:
         _hold(stream, ws)
     return out

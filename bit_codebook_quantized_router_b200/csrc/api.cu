@@ -62,10 +62,11 @@ bool shape_ok(const moe_q4_layer* L, int T, int top_k) {
 //   h_lo bf16[T*k][I] | y f32[T*k][H] | xg bf16[T*k][H] (activation rows in
 //   expert order, T > 16 only) | split-tile counters int32[units] | partial sums of the
 //   small-M kernels f32[2*160][4][min(16,T)][128] (two 128-row tiles per unit,
-//   gate/up then down)
+//   gate/up then down) | with a shared expert: h_s | y_s | its split partial
+//   sums | with the router gate in front: logits f32[T][E] | its partial sums
 struct Layout {
   size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, tiles, h, h_lo, y, xg, dk_counter,
-      dk_partial, h_s, y_s, sx_partial, end;
+      dk_partial, h_s, y_s, sx_partial, logits, router_partial, end;
   int dk_units_gu, dk_units_dn, n_max;
 };
 
@@ -76,7 +77,7 @@ bool shared_ok(const moe_q4_layer* L, const moe_q4_shared* S) {
   return L->H % 64 == 0;
 }
 
-Layout layout(const moe_q4_layer* L, int T, int k, const moe_q4_shared* S = nullptr) {
+Layout layout(const moe_q4_layer* L, int T, int k, const moe_q4_shared* S = nullptr, bool gated = false) {
   const size_t R = (size_t)T * k;
   Layout o;
   size_t p = 0;
@@ -131,6 +132,14 @@ Layout layout(const moe_q4_layer* L, int T, int k, const moe_q4_shared* S = null
     o.sx_partial = p;
     p = align_up(p + (pa > pb ? pa : pb));
   }
+  // router gate in front (moe_q4_forward_gated): logits f32 [T][E] | its partial sums
+  o.logits = o.router_partial = 0;
+  if (gated) {
+    o.logits = p;
+    p = align_up(p + sizeof(float) * (size_t)T * L->E);
+    o.router_partial = p;
+    p = align_up(p + q4_router_partial_bytes(T, L->H, L->E));
+  }
   o.end = p;
   return o;
 }
@@ -156,8 +165,8 @@ HostStage host_stage(const moe_q4_layer* L, int T, size_t base) {
 int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, const float* logits,
                 int T, int k, void* out, float* out_f32, int32_t* topk_ids, float* topk_w,
                 int32_t* counts, char* ws, cudaStream_t s, void* const* events = nullptr,
-                const moe_q4_shared* S = nullptr) {
-  const Layout o = layout(L, T, k, S);
+                const moe_q4_shared* S = nullptr, const void* router_w = nullptr) {
+  const Layout o = layout(L, T, k, S, router_w != nullptr);
   FwdArgs a;
   memset(&a, 0, sizeof a);
   a.T = T;
@@ -205,7 +214,23 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   // path takes, so the tensor-core kernels are not launched at all.
   const bool pre = uses_prefill(T);
   int rc = mark(0);
-  if (rc == MOE_Q4_OK) rc = q4_launch_route(a, s);
+  if (rc == MOE_Q4_OK && router_w) {
+    // the router gate in front: the logits land in `logits` (the caller's
+    // buffer or the workspace's); the status word and the fused kernel's
+    // ticket start at zero, and the routing leaves the status alone
+    a.keep_status = 1;
+    a.logits_in_forward = 1;
+    if (cudaMemsetAsync(a.hdr, 0, 8 * sizeof(int32_t), s) != cudaSuccess) rc = MOE_Q4_ECUDA;
+    if (rc == MOE_Q4_OK && q4_router_route_fused(T, L->H, k)) {
+      rc = q4_launch_router_route(a, router_w, s);
+    } else if (rc == MOE_Q4_OK) {
+      rc = q4_launch_router(x, router_w, T, L->H, L->E, const_cast<float*>(logits), ws + o.router_partial,
+                            a.hdr + kStatus, s);
+      if (rc == MOE_Q4_OK) rc = q4_launch_route(a, s);
+    }
+  } else if (rc == MOE_Q4_OK) {
+    rc = q4_launch_route(a, s);
+  }
   if (rc == MOE_Q4_OK) rc = mark(1);
   const int grid = dk_grid();
   float* part_gu = (float*)(ws + o.dk_partial);
@@ -330,6 +355,31 @@ extern "C" int moe_q4_forward_ex(const moe_q4_layer* layer, const moe_q4_shared*
     return MOE_Q4_EWORKSPACE;
   return run_forward(layer, tp, x, logits, T, top_k, out, out_f32, topk_ids, topk_w, counts, (char*)ws,
                      (cudaStream_t)stream, nullptr, shared);
+}
+
+extern "C" size_t moe_q4_forward_gated_workspace(const moe_q4_layer* layer, const moe_q4_shared* shared, int T,
+                                                 int top_k) {
+  if (!shape_ok(layer, T, top_k) || !shared_ok(layer, shared)) return 0;
+  return layout(layer, T, top_k, shared, true).end;
+}
+
+extern "C" int moe_q4_forward_gated(const moe_q4_layer* layer, const moe_q4_shared* shared, const void* router_w,
+                                    const void* x, int T, int top_k, void* out, float* out_f32, float* logits,
+                                    int32_t* topk_ids, float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                                    void* stream) {
+  if (!shape_ok(layer, T, top_k) || !shared_ok(layer, shared)) return MOE_Q4_EINVAL;
+  TableParams tp;
+  int rc = q4_fill_tables(&tp, layer->tables, layer->n_tables, layer->table_id, layer->E);
+  if (rc != MOE_Q4_OK) return rc;
+  if (T == 0) return MOE_Q4_OK;
+  if (!router_w || !x || !out || ((uintptr_t)router_w & 15) || ((uintptr_t)x & 15) || ((uintptr_t)out & 15) ||
+      ((uintptr_t)out_f32 & 15) || ((uintptr_t)logits & 3))
+    return MOE_Q4_EINVAL;
+  const Layout o = layout(layer, T, top_k, shared, true);
+  if (!ws || ((uintptr_t)ws & (kAlign - 1)) || ws_bytes < o.end) return MOE_Q4_EWORKSPACE;
+  float* lg = logits ? logits : reinterpret_cast<float*>((char*)ws + o.logits);
+  return run_forward(layer, tp, x, lg, T, top_k, out, out_f32, topk_ids, topk_w, counts, (char*)ws,
+                     (cudaStream_t)stream, nullptr, shared, router_w);
 }
 
 extern "C" int moe_q4_forward_stages(const moe_q4_layer* layer, const void* x, const float* logits,

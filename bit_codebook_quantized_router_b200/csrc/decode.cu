@@ -860,7 +860,9 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   using Geo = typename C::template Geom<SUBS>;
   P.partial = partial;
   P.counter = counter;
-  P.self_k = GATEUP && a.T == 1 ? a.k : 0;
+  // (one token routed by the kernel itself reads the logits before its
+  // dependency wait: only when they are an input of the forward)
+  P.self_k = GATEUP && a.T == 1 && !a.logits_in_forward ? a.k : 0;
 
   // deepest ring that fits; the dynamic window starts after the reserved bytes
   // (the kernel has no static shared memory)

@@ -37,6 +37,8 @@ struct FwdArgs {
   __nv_bfloat16* xg;       // [T*k][H] expert-grouped activations
   int32_t* dk_counter;     // [dk_counter_n] split-tile arrival counters (small-M path)
   int dk_counter_n;
+  int keep_status;         // the status word was cleared before this forward's first kernel
+  int logits_in_forward;   // the logits are computed by this forward's first kernel
   int32_t* user_ids;
   float* user_w;
   int32_t* user_counts;
@@ -51,6 +53,15 @@ int q4_fill_tables(q4::TableParams* tp, const float* tables, int n_tables, const
 // Kernel launchers (return MOE_Q4_OK or MOE_Q4_ECUDA).
 int q4_launch_route(const q4::FwdArgs& a, cudaStream_t s);
 int q4_launch_combine(const q4::FwdArgs& a, cudaStream_t s);
+// Router gate (router.cu): logits = x . w^T at any T (part: the partial sums,
+// q4_router_partial_bytes; status: the dense GEMM's status word), and at
+// decode sizes the router with the routing fused behind it (a.logits is the
+// logits buffer it writes; a.hdr[kRouterTicket] must be 0 at launch).
+size_t q4_router_partial_bytes(int T, int H, int E);
+int q4_launch_router(const void* x, const void* w, int T, int H, int E, float* logits, void* part, int32_t* status,
+                     cudaStream_t s);
+bool q4_router_route_fused(int T, int H, int k);
+int q4_launch_router_route(const q4::FwdArgs& a, const void* w, cudaStream_t s);
 int q4_launch_gather(const q4::FwdArgs& a, cudaStream_t s);
 int q4_launch_prefill(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, cudaStream_t s);
 int q4_prefill_tile_n();

@@ -34,7 +34,7 @@ enum HeaderWord : int {
   kNumDecode = 1,  // experts on the small-M streaming path
   kNumPrefill = 2, // experts on the tensor-core path
   kNumTiles = 3,   // tensor-core path work tiles
-  kTileCursor = 4, // dynamic tile scheduler cursor
+  kRouterTicket = 4,  // CTAs of the fused router + routing kernel done with their logits
   kHeaderWords = 64,
 };
 
@@ -169,6 +169,9 @@ constexpr int kMaxLogitsPerLane = kMaxExperts / 32;
 // Each of the k rounds takes the best remaining (value, then lower id) by a
 // warp argmax; lane j ends up holding slot j.  Non-finite logits are
 // treated as -inf and recorded as a device error (unless status is null).
+// L2_ONLY: read the logits through L2 only (ld.global.cg), for logits that
+// other CTAs of the same grid wrote.
+template <bool L2_ONLY = false>
 __device__ __forceinline__ void topk_warp(const float* __restrict__ row, int E, int k, int lane,
                                           int32_t* status, int& my_id, float& my_w) {
   float v[kMaxLogitsPerLane];
@@ -179,7 +182,7 @@ __device__ __forceinline__ void topk_warp(const float* __restrict__ row, int E, 
     const int id = lane + 32 * i;
     v[i] = -INFINITY;
     if (id < E) {
-      float x = row[id];
+      float x = L2_ONLY ? __ldcg(row + id) : row[id];
       if (!isfinite(x)) {
         bad = true;
         x = -INFINITY;

@@ -11,22 +11,13 @@
 
 #include "q4_api_internal.h"
 #include "q4_common.cuh"
+#include "route_small.cuh"
 
 namespace q4 {
 
 constexpr int kRouteThreads = 1024;
 constexpr int kRouteWarps = kRouteThreads / 32;
 constexpr int kFusedMaxT = 256;  // above this, top-k runs on many CTAs first
-
-__device__ __forceinline__ void store_route(const FwdArgs& a, int t, int lane, int id, float w) {
-  if (lane < a.k) {
-    const int r = t * a.k + lane;
-    a.ids[r] = id;
-    a.w[r] = w;
-    if (a.user_ids) a.user_ids[r] = id;
-    if (a.user_w) a.user_w[r] = w;
-  }
-}
 
 // Block-wide exclusive scan of one value per thread (kRouteThreads threads).
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
@@ -150,111 +141,16 @@ __device__ void group_rows(const FwdArgs& a, int* sm) {
   }
 }
 
-// Small T (<= kFusedMaxT): one CTA routes every token and groups, with the
-// ids kept in shared memory.  A row's place within its expert is the number
-// of earlier tokens that chose the same expert, read from a per-expert
-// bitmask of tokens (tokens pick an expert at most once, so token order is
-// row order within an expert).  One packed scan gives the offsets, both
-// expert lists and the tensor-core tile offsets.
-// Shared memory: ids[T*k] | counts[E] | offs[E] | tokmask[E][W], W = ceil(T/32).
+// Small T (<= kFusedMaxT): one CTA routes every token and groups
+// (route_small, ids kept in shared memory).
 __global__ void __launch_bounds__(kRouteThreads) route_fused_kernel(const __grid_constant__ FwdArgs a) {
   extern __shared__ int sm[];
-  const int E = a.E, T = a.T, k = a.k;
-  const int W = (T + 31) >> 5;
-  int* ids_s = sm;
-  int* counts = ids_s + T * k;
-  int* offs = counts + E;
-  uint32_t* tokmask = reinterpret_cast<uint32_t*>(offs + E);
-  __shared__ unsigned long long warp_tot[33];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int e = tid; e < E; e += kRouteThreads) counts[e] = 0;
-  for (int i = tid; i < E * W; i += kRouteThreads) tokmask[i] = 0u;
   pdl_wait();
   // The next kernel may be scheduled now.  Its own wait still covers this
   // kernel's results; what it reads before that wait (the layer's inputs x
   // and logits, the weights) is complete once this kernel's wait returned.
   pdl_trigger();
-  if (tid == 0) a.hdr[kStatus] = MOE_Q4_OK;
-  // per-tile arrival counters of the small-M kernels start at zero every call
-  for (int i = tid; i < a.dk_counter_n; i += kRouteThreads) a.dk_counter[i] = 0;
-  __syncthreads();
-  for (int t = warp; t < T; t += kRouteWarps) {
-    int id;
-    float w;
-    topk_warp(a.logits + (size_t)t * E, E, k, lane, a.hdr + kStatus, id, w);
-    store_route(a, t, lane, id, w);
-    if (lane < k) {
-      ids_s[t * k + lane] = id;
-      if ((unsigned)id < (unsigned)E) {
-        atomicAdd(&counts[id], 1);
-        atomicOr(&tokmask[id * W + (t >> 5)], 1u << (t & 31));
-      } else {
-        record_error(a.hdr + kStatus, MOE_Q4_EDEVICE);
-      }
-    }
-  }
-  __syncthreads();
-  // one exclusive scan over experts of four 16-bit fields:
-  //   rows | small-M experts | tensor-core experts | tensor-core tiles
-  // (T*k <= 4096 rows and E <= 512 experts: no field overflows)
-  const int c = tid < E ? counts[tid] : 0;
-  const bool fd = c > 0 && c <= a.dec_max, fp = c > a.dec_max;
-  const int ntl = fp ? (c + a.tile_n - 1) / a.tile_n : 0;
-  const unsigned long long v = (unsigned long long)c | ((unsigned long long)(fd ? 1 : 0) << 16) |
-                               ((unsigned long long)(fp ? 1 : 0) << 32) | ((unsigned long long)ntl << 48);
-  unsigned long long inc = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long u = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += u;
-  }
-  if (lane == 31) warp_tot[warp] = inc;
-  __syncthreads();
-  if (warp == 0) {
-    const unsigned long long wv = warp_tot[lane];
-    unsigned long long winc = wv;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned long long u = __shfl_up_sync(0xffffffffu, winc, o);
-      if (lane >= o) winc += u;
-    }
-    warp_tot[lane] = winc - wv;
-    if (lane == 31) warp_tot[32] = winc;
-  }
-  __syncthreads();
-  const unsigned long long ex = warp_tot[warp] + inc - v, tot = warp_tot[32];
-  const int off = (int)(ex & 0xffffu), pd = (int)((ex >> 16) & 0xffffu);
-  const int pp = (int)((ex >> 32) & 0xffffu), ntoff = (int)(ex >> 48);
-  if (tid < E) {
-    offs[tid] = off;
-    a.offsets[tid] = off;
-    a.counts[tid] = c;
-    if (a.user_counts) a.user_counts[tid] = c;
-    if (fd) a.dec_list[pd] = tid;
-    if (fp) a.pre_list[pp] = tid;
-    if (fp && a.tiles) a.tiles[pp] = ntoff;
-  }
-  if (tid == 0) {
-    const int total = (int)(tot & 0xffffu), nd = (int)((tot >> 16) & 0xffffu);
-    const int np = (int)((tot >> 32) & 0xffffu), ntot = (int)(tot >> 48);
-    a.offsets[E] = total;
-    a.hdr[kNumDecode] = nd;
-    a.hdr[kNumPrefill] = np;
-    a.hdr[kNumTiles] = ntot;
-    if (a.tiles) a.tiles[np] = ntot;
-  }
-  __syncthreads();
-  // stable placement: rank of token t among the tokens that chose expert e
-  for (int r = tid; r < T * k; r += kRouteThreads) {
-    const int t = r / k, e = ids_s[r];
-    if ((unsigned)e >= (unsigned)E) continue;
-    const uint32_t* m = tokmask + e * W;
-    int rank = __popc(m[t >> 5] & ((1u << (t & 31)) - 1u));
-    for (int q = 0; q < (t >> 5); ++q) rank += __popc(m[q]);
-    const int pos = offs[e] + rank;
-    a.row_token[pos] = t;
-    a.inv[r] = pos;
-  }
+  route_small<kRouteThreads, false>(a, sm);
 }
 
 // Large T: top-k on many CTAs (one warp per token; the host clears the
@@ -302,12 +198,9 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant_
 using namespace q4;
 
 static size_t group_smem_bytes(int E) { return sizeof(int) * ((size_t)3 * E + 1 + (size_t)2 * kRouteWarps * E); }
-static size_t fused_smem_bytes(int E, int T, int k) {
-  return sizeof(int) * ((size_t)T * k + 2 * (size_t)E + (size_t)E * ((T + 31) / 32));
-}
 
 int q4_launch_route(const FwdArgs& a, cudaStream_t s) {
-  const size_t smem = a.T <= kFusedMaxT ? fused_smem_bytes(a.E, a.T, a.k) : group_smem_bytes(a.E);
+  const size_t smem = a.T <= kFusedMaxT ? route_small_smem_bytes(a.E, a.T, a.k) : group_smem_bytes(a.E);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -327,7 +220,8 @@ int q4_launch_route(const FwdArgs& a, cudaStream_t s) {
     if (cudaFuncSetAttribute(route_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return MOE_Q4_ECUDA;
-    if (cudaMemsetAsync(a.hdr + kStatus, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_Q4_ECUDA;
+    if (!a.keep_status && cudaMemsetAsync(a.hdr + kStatus, 0, sizeof(int32_t), s) != cudaSuccess)
+      return MOE_Q4_ECUDA;
     cfg.gridDim = dim3((a.T + 7) / 8);
     cfg.blockDim = dim3(256);
     cfg.dynamicSmemBytes = 0;

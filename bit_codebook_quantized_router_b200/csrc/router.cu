@@ -16,6 +16,7 @@
 
 #include "q4_api_internal.h"
 #include "q4_common.cuh"
+#include "route_small.cuh"
 
 namespace cg = cooperative_groups;
 
@@ -155,9 +156,8 @@ __global__ void __launch_bounds__(rt::kThreads) router_kernel(const uint16_t* __
 // adding the C CTA sums in rank order through distributed shared memory.  The order of every sum is
 // fixed by (H, C), so the result does not depend on scheduling.
 template <int NT>
-__global__ void __launch_bounds__(rt::kThreads, 1) router_few_kernel(const uint16_t* __restrict__ x,
-                                                                  const uint16_t* __restrict__ w, int T, int H, int E,
-                                                                  int chunks, float* __restrict__ logits) {
+__device__ __forceinline__ void router_few_body(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w, int T,
+                                                int H, int E, int chunks, float* __restrict__ logits) {
   constexpr int kTile = rt::kRows * rt::kTokens;  // 512 logits: [gate row][token]
   __shared__ float part[rt::kWarps][kTile];
   __shared__ float cta_sum[kTile];
@@ -211,6 +211,37 @@ __global__ void __launch_bounds__(rt::kThreads, 1) router_few_kernel(const uint1
   cluster.sync();  // no CTA leaves while another still reads its shared memory
 }
 
+template <int NT>
+__global__ void __launch_bounds__(rt::kThreads, 1) router_few_kernel(const uint16_t* __restrict__ x,
+                                                                  const uint16_t* __restrict__ w, int T, int H, int E,
+                                                                  int chunks, float* __restrict__ logits) {
+  router_few_body<NT>(x, w, T, H, E, chunks, logits);
+}
+
+// The same with the routing fused behind it ("GLM-5.2-EXL3-DENSE6-MTP78",
+// "Quant recipe": the BF16 mlp.gate in front of the routed experts): every
+// CTA writes its share of the logits, makes it visible device-wide and takes
+// a ticket; the CTA holding the last ticket (no CTA waits for another) reads
+// all the logits through L2 and routes and groups the T tokens (route_small),
+// then clears the ticket for the next call.  One launch from hidden states
+// to the grouped rows; the logits stay in L2.
+template <int NT>
+__global__ void __launch_bounds__(rt::kThreads, 1) router_route_kernel(const __grid_constant__ FwdArgs a,
+                                                                    const uint16_t* __restrict__ w, int chunks) {
+  extern __shared__ int route_sm[];
+  __shared__ int last;
+  pdl_trigger();  // scheduling only: the next kernel's wait covers this whole grid
+  router_few_body<NT>(reinterpret_cast<const uint16_t*>(a.x), w, a.T, a.H, a.E, chunks, const_cast<float*>(a.logits));
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(a.hdr + kRouterTicket, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  route_small<rt::kThreads, true>(a, route_sm);
+  if (threadIdx.x == 0) a.hdr[kRouterTicket] = 0;
+}
+
 // logits = the chunks' partial sums, added in a fixed order: one thread per
 // logit in chunk order, or (many chunks) one warp per logit, lane l adding
 // chunks l, l + 32, ... and the lanes' sums combined by a fixed butterfly.
@@ -260,61 +291,58 @@ static int router_few_cluster(int chunks) {
 // word (256 bytes) then the split partial sums.
 static bool router_dense(int T, int H, int E) { return !router_few(T, H) && T > 32 && E % 128 == 0 && H % 64 == 0; }
 
-extern "C" size_t moe_q4_router_workspace(int T, int H, int E) {
-  if (!router_args_ok(T, H, E) || T == 0 || router_few(T, H)) return 0;
-  if (router_dense(T, H, E)) return 256 + q4_dense_partial_bytes(T, E, H, 1);
+size_t q4_router_partial_bytes(int T, int H, int E) {
+  if (T == 0 || router_few(T, H)) return 0;
+  if (router_dense(T, H, E)) return q4_dense_partial_bytes(T, E, H, 1);
   const RouterPlan p = router_plan(T, H, E);
   return p.chunks > 1 ? sizeof(float) * (size_t)p.chunks * T * E : 0;
 }
 
-extern "C" int moe_q4_router(const void* x, const void* w, int T, int H, int E, float* logits, void* ws,
-                             size_t ws_bytes, void* stream) {
-  if (!router_args_ok(T, H, E)) return MOE_Q4_EINVAL;
+// Cluster launch of a decode-size kernel over the gate tiles.
+template <typename... Args>
+static cudaError_t launch_few(void (*kern)(Args...), const RouterPlan& p, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  const int C = router_few_cluster(p.chunks);
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.e_tiles * C);
+  cfg.blockDim = dim3(rt::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
+int q4_launch_router(const void* x, const void* w, int T, int H, int E, float* logits, void* part, int32_t* status,
+                     cudaStream_t s) {
   if (T == 0) return MOE_Q4_OK;
-  if (!x || !w || !logits) return MOE_Q4_EINVAL;
-  if (((uintptr_t)x & 15) || ((uintptr_t)w & 15)) return MOE_Q4_EINVAL;
   const RouterPlan p = router_plan(T, H, E);
-  cudaStream_t s = (cudaStream_t)stream;
   const uint16_t* xb = static_cast<const uint16_t*>(x);
   const uint16_t* wb = static_cast<const uint16_t*>(w);
   if (router_few(T, H)) {
-    const int C = router_few_cluster(p.chunks);
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.e_tiles * C);
-    cfg.blockDim = dim3(rt::kThreads);
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     const int nt = (T + 7) / 8;
     cudaError_t e;
     if (nt == 1)
-      e = cudaLaunchKernelEx(&cfg, router_few_kernel<1>, xb, wb, T, H, E, p.chunks, logits);
+      e = launch_few(router_few_kernel<1>, p, 0, s, xb, wb, T, H, E, p.chunks, logits);
     else if (nt == 2)
-      e = cudaLaunchKernelEx(&cfg, router_few_kernel<2>, xb, wb, T, H, E, p.chunks, logits);
+      e = launch_few(router_few_kernel<2>, p, 0, s, xb, wb, T, H, E, p.chunks, logits);
     else if (nt == 3)
-      e = cudaLaunchKernelEx(&cfg, router_few_kernel<3>, xb, wb, T, H, E, p.chunks, logits);
+      e = launch_few(router_few_kernel<3>, p, 0, s, xb, wb, T, H, E, p.chunks, logits);
     else
-      e = cudaLaunchKernelEx(&cfg, router_few_kernel<4>, xb, wb, T, H, E, p.chunks, logits);
+      e = launch_few(router_few_kernel<4>, p, 0, s, xb, wb, T, H, E, p.chunks, logits);
     return e == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
   }
-  const size_t need = moe_q4_router_workspace(T, H, E);
-  if (need > 0 && (!ws || ws_bytes < need || ((uintptr_t)ws & 15))) return MOE_Q4_EWORKSPACE;
-  if (router_dense(T, H, E)) {
-    if ((uintptr_t)ws & 255) return MOE_Q4_EWORKSPACE;
-    int32_t* status = reinterpret_cast<int32_t*>(ws);
-    if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_Q4_ECUDA;
-    float* part = need > 256 ? reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + 256) : nullptr;
-    return q4_launch_dense(w, 1, 0, E, H, x, T, nullptr, logits, E, part, status, s);
-  }
+  if (router_dense(T, H, E))
+    return q4_launch_dense(w, 1, 0, E, H, x, T, nullptr, logits, E, static_cast<float*>(part), status, s);
   const long long units = (long long)p.e_tiles * p.t_tiles * p.chunks;
   const long long want = (units + rt::kWarps - 1) / rt::kWarps;
   const int grid = (int)(want < 148 * 8 ? want : 148 * 8);
-  float* dst = p.chunks > 1 ? reinterpret_cast<float*>(ws) : logits;
+  float* dst = p.chunks > 1 ? static_cast<float*>(part) : logits;
   router_kernel<<<grid, rt::kThreads, 0, s>>>(xb, wb, T, H, E, p, dst);
   if (cudaGetLastError() != cudaSuccess) return MOE_Q4_ECUDA;
   if (p.chunks > 1) {
@@ -325,4 +353,49 @@ extern "C" int moe_q4_router(const void* x, const void* w, int T, int H, int E, 
     if (cudaGetLastError() != cudaSuccess) return MOE_Q4_ECUDA;
   }
   return MOE_Q4_OK;
+}
+
+bool q4_router_route_fused(int T, int H, int k) { return T >= 1 && router_few(T, H) && T * k <= 4096; }
+
+int q4_launch_router_route(const FwdArgs& a, const void* w, cudaStream_t s) {
+  const RouterPlan p = router_plan(a.T, a.H, a.E);
+  const size_t smem = route_small_smem_bytes(a.E, a.T, a.k);
+  const uint16_t* wb = static_cast<const uint16_t*>(w);
+  const int nt = (a.T + 7) / 8;
+  cudaError_t e;
+  if (nt == 1)
+    e = launch_few(router_route_kernel<1>, p, smem, s, a, wb, p.chunks);
+  else if (nt == 2)
+    e = launch_few(router_route_kernel<2>, p, smem, s, a, wb, p.chunks);
+  else if (nt == 3)
+    e = launch_few(router_route_kernel<3>, p, smem, s, a, wb, p.chunks);
+  else
+    e = launch_few(router_route_kernel<4>, p, smem, s, a, wb, p.chunks);
+  return e == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
+}
+
+extern "C" size_t moe_q4_router_workspace(int T, int H, int E) {
+  if (!router_args_ok(T, H, E) || T == 0 || router_few(T, H)) return 0;
+  const size_t part = q4_router_partial_bytes(T, H, E);
+  return router_dense(T, H, E) ? 256 + part : part;
+}
+
+extern "C" int moe_q4_router(const void* x, const void* w, int T, int H, int E, float* logits, void* ws,
+                             size_t ws_bytes, void* stream) {
+  if (!router_args_ok(T, H, E)) return MOE_Q4_EINVAL;
+  if (T == 0) return MOE_Q4_OK;
+  if (!x || !w || !logits) return MOE_Q4_EINVAL;
+  if (((uintptr_t)x & 15) || ((uintptr_t)w & 15)) return MOE_Q4_EINVAL;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t need = moe_q4_router_workspace(T, H, E);
+  if (need > 0 && (!ws || ws_bytes < need || ((uintptr_t)ws & 15))) return MOE_Q4_EWORKSPACE;
+  if (router_dense(T, H, E)) {
+    // the dense GEMM's status word at the workspace start, its partial sums after it
+    if ((uintptr_t)ws & 255) return MOE_Q4_EWORKSPACE;
+    int32_t* status = reinterpret_cast<int32_t*>(ws);
+    if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_Q4_ECUDA;
+    void* part = need > 256 ? reinterpret_cast<char*>(ws) + 256 : nullptr;
+    return q4_launch_router(x, w, T, H, E, logits, part, status, s);
+  }
+  return q4_launch_router(x, w, T, H, E, logits, ws, nullptr, s);
 }

@@ -244,6 +244,35 @@ MOE_Q4_API int moe_q4_forward_ex(const moe_q4_layer* layer, const moe_q4_shared*
                                  int32_t* topk_ids, float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
                                  void* stream);
 
+/* ---------------------------------------------------------------------------
+ * moe_q4_forward_gated -- the layer with its router gate in front: from the
+ * hidden states alone ("GLM-5.2-EXL3-DENSE6-MTP78", "Quant recipe": the
+ * mlp.gate linear kept in BF16, ahead of the routed experts).
+ *   logits[t][e] = sum_h x[t][h] * router_w[e][h]   (fp32 accumulation, as
+ *   moe_q4_router computes them, bit for bit), then moe_q4_forward_ex on those
+ *   logits.
+ * For T <= 32 (with T * top_k <= 4096) one launch computes the logits on
+ * every SM and routes and groups the tokens: each CTA adds its logits'
+ * partial sums in a fixed order, publishes them device-wide and takes a
+ * ticket; the last CTA to finish routes (no CTA waits for another).  Larger
+ * T runs moe_q4_router's kernels (tensor cores for E % 128 == 0), then the
+ * routing kernels.
+ * Arguments as for moe_q4_forward_ex, plus:
+ *   router_w   device bf16 [E][H], 16-byte aligned;
+ *   logits     optional device fp32 [T][E] (out), 4-byte aligned: the
+ *              router's logits; NULL keeps them in the workspace;
+ *   ws         at least moe_q4_forward_gated_workspace(layer, shared, T,
+ *              top_k) bytes, 256-byte aligned.
+ * Device errors (a non-finite logit, a timed-out wait of the tensor-core
+ * router) set the workspace status word, as for moe_q4_forward.
+ * ------------------------------------------------------------------------- */
+MOE_Q4_API size_t moe_q4_forward_gated_workspace(const moe_q4_layer* layer, const moe_q4_shared* shared, int T,
+                                                 int top_k);
+MOE_Q4_API int moe_q4_forward_gated(const moe_q4_layer* layer, const moe_q4_shared* shared, const void* router_w,
+                                    const void* x, int T, int top_k, void* out, float* out_f32, float* logits,
+                                    int32_t* topk_ids, float* topk_w, int32_t* counts, void* ws, size_t ws_bytes,
+                                    void* stream);
+
 /* Synchronise `stream`, then return the status recorded in the workspace by
  * the last moe_q4_forward on it (MOE_Q4_OK, MOE_Q4_EDEVICE, MOE_Q4_ETIMEOUT),
  * or MOE_Q4_ECUDA if the stream itself reports an error. */

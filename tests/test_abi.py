@@ -154,6 +154,25 @@ def test_shared_expert_host_checks(L):
                                    None, None, 0, None) == _lib.EINVAL
 
 
+def test_gated_forward_host_checks(L):
+    st, keep = _layer()
+    base = L.moe_q4_forward_workspace(ctypes.byref(st), 4, 2)
+    gated = L.moe_q4_forward_gated_workspace(ctypes.byref(st), None, 4, 2)
+    assert gated > base  # the logits (and any router partial sums) live in the workspace
+    assert L.moe_q4_forward_gated_workspace(ctypes.byref(st), None, 4, 0) == 0
+    fake = ctypes.c_void_p(1 << 20)
+    f = L.moe_q4_forward_gated
+    # no router gate, a misaligned gate, a misaligned logits buffer, a short workspace
+    assert f(ctypes.byref(st), None, None, fake, 4, 2, fake, None, None, None, None, None, fake, gated,
+             None) == _lib.EINVAL
+    assert f(ctypes.byref(st), None, ctypes.c_void_p((1 << 20) + 2), fake, 4, 2, fake, None, None, None, None, None,
+             fake, gated, None) == _lib.EINVAL
+    assert f(ctypes.byref(st), None, fake, fake, 4, 2, fake, None, ctypes.c_void_p((1 << 20) + 2), None, None, None,
+             fake, gated, None) == _lib.EINVAL
+    assert f(ctypes.byref(st), None, fake, fake, 4, 2, fake, None, None, None, None, None, fake, gated - 256,
+             None) == _lib.EWORKSPACE
+
+
 def test_debug_build_exports_every_declared_symbol(L):
     from bit_codebook_quantized_router_b200 import build
     assert os.path.exists(build.LIB_DEBUG)

@@ -62,11 +62,12 @@ def test_tiny_workload_full():
 
 # Edge cases on a small layer (H=256, I=128, E=8): T=1; an expert with
 # exactly the small-M path's limit (16 rows) and one more (17, the tensor-core
-# path); exactly one tensor-core token tile (256) and one more (257); experts
-# with 0 rows; every token on one expert; k = 1; k = E.
+# path); exactly one tensor-core token tile (256) and one more (257), a tile
+# and a half (384, 385), ragged single tiles (192, 193); experts with 0 rows;
+# every token on one expert; k = 1; k = E.
 @pytest.mark.parametrize("T,k,bias", [(1, 2, None), (16, 1, 3), (17, 1, 3), (33, 2, None),
-                                      (40, 2, 5), (64, 8, None), (200, 2, None), (256, 1, 3), (257, 1, 3),
-                                      (300, 3, 0)])
+                                      (40, 2, 5), (64, 8, None), (192, 1, 3), (193, 1, 3), (200, 2, None),
+                                      (256, 1, 3), (257, 1, 3), (300, 3, 0), (384, 1, 3), (385, 1, 3)])
 def test_small_layer_edge_counts(T, k, bias):
     w = inputs.Workload("small", 7, T, inputs.TINY)
     L, dev = _small_device_layer(w)
