@@ -49,6 +49,25 @@ def test_small_layer_with_shared_expert(T, k):
     gpu_support.check_out(out, ref, f"shared T={T} k={k}")
 
 
+# At decode sizes the shared expert's GEMMs split K over the SMs.  A layer
+# with longer K than the tiny one (H = 1024, shared I = 512) makes its gate/up
+# split 16 k-steps in 4 and its down 8 in 2; the split partial sums are added
+# in split order by a second kernel, and a repeat gives the same bits.
+@pytest.mark.parametrize("T", [1, 3, 16])
+def test_shared_expert_with_k_splits(T):
+    w = inputs.Workload("shared_split", 17, T, inputs.Shape(H=1024, I=256, E=8, k=2))
+    L, dev = _small_device_layer(w)
+    gu, dn = inputs.shared_expert_weights(w, I=512, device="cuda")
+    sh = q4.Shared(gu, dn)
+    x = inputs.activations(w)
+    lg = inputs.router_logits(w)
+    out = _run(dev, sh, x.cuda(), lg.cuda(), 2)
+    ref = _ref(L, inputs.bf16_bits(x), lg.numpy(), 2, gu, dn, range(T))
+    gpu_support.check_out(out, ref, f"shared with K splits T={T}")
+    again = _run(dev, sh, x.cuda(), lg.cuda(), 2)
+    assert torch.equal(out, again)
+
+
 def test_without_shared_expert_equals_forward():
     w = inputs.Workload("shared0", 15, 6, inputs.TINY)
     _, dev = _small_device_layer(w)
