@@ -322,7 +322,10 @@ __device__ __forceinline__ void decode_chunk(const uint4 c, const Planes& PL, ui
 
 // SUBS (64-K super-steps per stage, 4 or 2) is a template argument so that a
 // stage's two 128-K halves form one unrolled block the compiler can interleave.
-template <bool GATEUP, int NT, int SUBS>
+// SELF: the one-token routing below is compiled in (only the gate/up kernel
+// of a one-token call uses it; compiled into the others it cost 2.5 us per
+// launch at T = 8 although never run).
+template <bool GATEUP, int NT, int SUBS, bool SELF>
 __global__ void __launch_bounds__(dk::kThreads, 1)
     dk_kernel(const __grid_constant__ DkParams P, const __grid_constant__ TableParams tp,
               const __grid_constant__ CUtensorMap tm_wa, const __grid_constant__ CUtensorMap tm_wb) {
@@ -381,7 +384,7 @@ __global__ void __launch_bounds__(dk::kThreads, 1)
   // only after a wait at the end of each unit; every thread waits again
   // before it exits, so the kernels after this one still find the routing
   // kernel complete.
-  const bool self = GATEUP && P.self_k > 0;
+  const bool self = SELF && GATEUP && P.self_k > 0;
   int* self_e = reinterpret_cast<int*>(bars) + 64;  // [k] expert list (bytes 256.. of the barrier block)
   if (self && warp == 0) {  // (while warps 1..8 build the table below)
     const int k = P.self_k;
@@ -844,7 +847,7 @@ static bool dk_map(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, con
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GATEUP, int NT, int SUBS>
+template <bool GATEUP, int NT, int SUBS, bool SELF>
 static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partial, int32_t* counter, int grid,
                      cudaStream_t s) {
   using C = DkCfg<GATEUP, NT>;
@@ -862,7 +865,7 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   P.counter = counter;
   // (one token routed by the kernel itself reads the logits before its
   // dependency wait: only when they are an input of the forward)
-  P.self_k = GATEUP && a.T == 1 && !a.logits_in_forward ? a.k : 0;
+  P.self_k = SELF && GATEUP && a.T == 1 && !a.logits_in_forward ? a.k : 0;
 
   // deepest ring that fits; the dynamic window starts after the reserved bytes
   // (the kernel has no static shared memory)
@@ -893,7 +896,8 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
     twb = twa;
   }
   if (!ok) return MOE_Q4_ECUDA;
-  if (cudaFuncSetAttribute(dk_kernel<GATEUP, NT, SUBS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+  if (cudaFuncSetAttribute(dk_kernel<GATEUP, NT, SUBS, SELF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) !=
       cudaSuccess)
     return MOE_Q4_ECUDA;
   cudaLaunchAttribute attr[1];
@@ -908,7 +912,7 @@ static int launch_dk_subs(const FwdArgs& a, const TableParams& tp, float* partia
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, dk_kernel<GATEUP, NT, SUBS>, P, tp, twa, twb) == cudaSuccess ? MOE_Q4_OK
+  return cudaLaunchKernelEx(&cfg, dk_kernel<GATEUP, NT, SUBS, SELF>, P, tp, twa, twb) == cudaSuccess ? MOE_Q4_OK
                                                                                                  : MOE_Q4_ECUDA;
 }
 
@@ -917,8 +921,14 @@ template <bool GATEUP, int NT>
 static int launch_dk(const FwdArgs& a, const TableParams& tp, float* partial, int32_t* counter, int grid,
                      cudaStream_t s) {
   const int K = GATEUP ? a.H : a.I;
-  return K % 256 == 0 ? launch_dk_subs<GATEUP, NT, 4>(a, tp, partial, counter, grid, s)
-                      : launch_dk_subs<GATEUP, NT, 2>(a, tp, partial, counter, grid, s);
+  // one token routed by the gate/up kernel itself (logits given as input)
+  if constexpr (GATEUP && NT == 1) {
+    if (a.T == 1 && !a.logits_in_forward)
+      return K % 256 == 0 ? launch_dk_subs<GATEUP, NT, 4, true>(a, tp, partial, counter, grid, s)
+                          : launch_dk_subs<GATEUP, NT, 2, true>(a, tp, partial, counter, grid, s);
+  }
+  return K % 256 == 0 ? launch_dk_subs<GATEUP, NT, 4, false>(a, tp, partial, counter, grid, s)
+                      : launch_dk_subs<GATEUP, NT, 2, false>(a, tp, partial, counter, grid, s);
 }
 
 }  // namespace q4

@@ -64,6 +64,11 @@ struct TcCfg {
   static constexpr int kCTile = kBM * kBK / 2;        // 4 KB codes per matrix
   static constexpr int kStageBytes = kMats * kATile + kBTile + kMats * kCTile;
   static constexpr int kAccBufs = GATEUP ? 1 : 2;     // TMEM holds 512 columns
+  // single-buffered accumulators (gate/up): the dequant warps, idle while the
+  // MMA waits for the drain, drain beside the epilogue warps
+  static constexpr bool kHelp = kAccBufs == 1;
+  static constexpr int kDrainWarps = kEpiWarps + (kHelp ? kDequantThreads / 32 : 0);
+  static constexpr int kWorkersPerQuad = kDrainWarps / 4;
   static constexpr int kTmemCols = kAccBufs * kMats * kBN;
   static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 1024 /*barriers*/;
 };
@@ -111,8 +116,8 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
   uint64_t* empty = a_ready + C::kStages;        // [S] stage consumed by the MMAs
   uint64_t* acc_full = empty + C::kStages;       // [2]
   uint64_t* acc_empty = acc_full + 2;            // [2]
-  uint64_t* drain = acc_empty + 2;               // [1] final MMA completion
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* mma_done = acc_empty + 2;            // [1] final MMA completion
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const FwdArgs& a = P.a;
@@ -127,9 +132,9 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], C::kEpiWarps);
+      mbar_init(&acc_empty[b], C::kDrainWarps);
     }
-    mbar_init(drain, 1);
+    mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tmap(&tm_b);
@@ -150,6 +155,78 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
   const int total = np > 0 ? P.m_tiles * a.tiles[np] : 0;
   const int rows_total = GATEUP ? a.I : a.H;
   const int K = GATEUP ? a.H : a.I;
+
+  // Drain of the accumulators of the tcount-th tile of this CTA by one warp:
+  // worker `wk` of the C::kWorkersPerQuad warps of its TMEM lane quarter takes
+  // a contiguous range of 8-column chunks; tcgen05.ld of the fp32 sums (one
+  // lane = one weight row), SwiGLU (gate/up) or fp32 y (down), stores, then
+  // the warp signs off on acc_empty.  False when a wait gave up.
+  const auto drain = [&](int tile, uint32_t tcount, int wk) -> bool {
+    const int quad = warp & 3;          // TMEM lanes 32*quad .. +31
+    const int row = quad * 32 + lane;   // weight row in the tile
+    int p, m, nt;
+    tile_coords(a, P.m_tiles, np, tile, p, m, nt);
+    int e = a.pre_list[p];
+    if (!q4_check((unsigned)e < (unsigned)a.E, a.hdr + kStatus)) e = 0;
+    int n_e = a.counts[e];
+    const int row0 = a.offsets[e];
+    // (a failed check leaves the tile's rows unwritten)
+    if (!q4_check(row0 >= 0 && n_e >= 0 && row0 + n_e <= a.T * a.k, a.hdr + kStatus)) n_e = nt * kBN;
+    const int buf = (int)(tcount % C::kAccBufs);
+    const uint32_t use = tcount / C::kAccBufs;
+    if (!mbar_wait_warp(&acc_full[buf], use & 1, abort_flag, kWaitLimitNs)) return false;
+    tc_fence_after();
+    const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * (C::kMats * kBN);
+    const int wrow = m * kBM + row;
+    const int n_hi = n_e - nt * kBN < kBN ? n_e - nt * kBN : kBN;  // tokens of this tile
+    // 8 token columns of every matrix per chunk; the next chunk's TMEM loads
+    // are in flight while this chunk is finished (one wait per chunk)
+    constexpr int kCw = 8;
+    uint32_t va[C::kMats][kCw], vb[C::kMats][kCw];
+    const auto issue = [&](uint32_t (*v)[kCw], int c0) {
+#pragma unroll
+      for (int mt = 0; mt < C::kMats; ++mt) tmem_ld8_nowait(tb + mt * kBN + c0, v[mt]);
+    };
+    // this thread's row in the output rows of the tile's tokens: token c of the
+    // tile at out_row + c * stride
+    const size_t stride = GATEUP ? (size_t)a.I : (size_t)a.H;
+    const size_t out_off = (size_t)(row0 + nt * kBN) * stride + (size_t)wrow;
+    const auto finish = [&](uint32_t (*v)[kCw], int c0) {
+      const int valid = n_hi - c0;  // tokens of this chunk that exist (>= 1)
+      size_t o = out_off + (size_t)c0 * stride;
+#pragma unroll
+      for (int j = 0; j < kCw; ++j, o += stride) {
+        if (valid < kCw && j >= valid) break;
+        if (GATEUP)
+          a.h[o] = __float2bfloat16_rn(silu_mul_fast(__uint_as_float(v[0][j]), __uint_as_float(v[C::kMats - 1][j])));
+        else
+          a.y[o] = __uint_as_float(v[0][j]);
+      }
+    };
+    // this warp's tokens: chunks [wk n / W, (wk + 1) n / W) of the n = kBN / 8
+    constexpr int kChunks = kBN / kCw;
+    const int c_lo = kCw * (wk * kChunks / C::kWorkersPerQuad);
+    const int c_end = kCw * ((wk + 1) * kChunks / C::kWorkersPerQuad);
+    const int c_hi = n_hi < c_end ? n_hi : c_end;
+    if (c_lo < c_hi) {
+      issue(va, c_lo);
+      tmem_wait_ld();
+#pragma unroll 1
+      for (int c0 = c_lo; c0 < c_hi; c0 += 2 * kCw) {
+        if (c0 + kCw < c_hi) issue(vb, c0 + kCw);
+        finish(va, c0);
+        tmem_wait_ld();
+        if (c0 + kCw >= c_hi) break;
+        if (c0 + 2 * kCw < c_hi) issue(va, c0 + 2 * kCw);
+        finish(vb, c0 + kCw);
+        tmem_wait_ld();
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    return true;
+  };
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
@@ -213,8 +290,8 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
         umma_commit(&acc_full[buf]);
       }
       // all MMAs issued by this thread complete before TMEM is released
-      umma_commit(drain);
-      mbar_wait(drain, 0, abort_flag, kWaitLimitNs);
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, abort_flag, kWaitLimitNs);
     }
   } else if (warp < C::kEpiWarp0) {
     // ---------------- dequantise ----------------
@@ -222,8 +299,14 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
     const int r = d & (kBM - 1);              // weight row in the tile
     const int my_half = (d >> 7) & 1;         // 32-weight half of the row's 64 K
     const int mat = GATEUP ? (d >> 8) : 0;    // gate / up
-    uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < total && !warp_aborted(abort_flag); tile += gridDim.x) {
+    // drain worker index of this warp in its TMEM lane quarter (after the
+    // epilogue warps'); it helps drain tile n while working on tile n + 1,
+    // once the ring is full and the MMA waits for that drain
+    const int help_wk = C::kEpiWarps / 4 + ((warp - 2) >> 2);
+    const int help_at = P.k_steps - 1 < C::kStages ? P.k_steps - 1 : C::kStages;
+    int prev_tile = -1;
+    uint32_t it = 0, tcount = 0;
+    for (int tile = blockIdx.x; tile < total && !warp_aborted(abort_flag); tile += gridDim.x, ++tcount) {
       int p, m, nt;
       tile_coords(a, P.m_tiles, np, tile, p, m, nt);
       const int e = a.pre_list[p];
@@ -239,6 +322,10 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
       uint32_t sc = 0;
       bool ok = true;
       for (int ks = 0; ks < P.k_steps; ++ks, ++it) {
+        if (C::kHelp && ks == help_at && prev_tile >= 0 && !drain(prev_tile, tcount - 1, help_wk)) {
+          ok = false;
+          break;
+        }
         if ((ks & 1) == 0) {
           sc = q0;
           q0 = q1;
@@ -280,74 +367,16 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
         if (lane == 0) mbar_arrive(&a_ready[s]);
       }
       if (!ok) break;
+      prev_tile = tile;
     }
+    // the CTA's last tile: no next tile to overlap with, drain it beside the epilogue
+    if (C::kHelp && prev_tile >= 0 && !warp_aborted(abort_flag)) drain(prev_tile, tcount - 1, help_wk);
   } else {
     // ---------------- epilogue ----------------
-    const int quad = warp & 3;          // TMEM lanes 32*quad .. +31
-    const int ehalf = (warp - C::kEpiWarp0) >> 2;  // tokens 128 ehalf .. + 127 of the tile
-    const int row = quad * 32 + lane;   // weight row in the tile
+    const int ehalf = (warp - C::kEpiWarp0) >> 2;  // drain worker 0 or 1 of its TMEM lane quarter
     uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < total && !warp_aborted(abort_flag); tile += gridDim.x, ++tcount) {
-      int p, m, nt;
-      tile_coords(a, P.m_tiles, np, tile, p, m, nt);
-      int e = a.pre_list[p];
-      if (!q4_check((unsigned)e < (unsigned)a.E, a.hdr + kStatus)) e = 0;
-      int n_e = a.counts[e];
-      const int row0 = a.offsets[e];
-      // (a failed check leaves the tile's rows unwritten)
-      if (!q4_check(row0 >= 0 && n_e >= 0 && row0 + n_e <= a.T * a.k, a.hdr + kStatus)) n_e = nt * kBN;
-      const int buf = (int)(tcount % C::kAccBufs);
-      const uint32_t use = tcount / C::kAccBufs;
-      if (!mbar_wait_warp(&acc_full[buf], use & 1, abort_flag, kWaitLimitNs)) break;
-      tc_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * (C::kMats * kBN);
-      const int wrow = m * kBM + row;
-      const int n_hi = n_e - nt * kBN < kBN ? n_e - nt * kBN : kBN;  // tokens of this tile
-      // 8 token columns of every matrix per chunk; the next chunk's TMEM loads
-      // are in flight while this chunk is finished (one wait per chunk)
-      constexpr int kCw = 8;
-      uint32_t va[C::kMats][kCw], vb[C::kMats][kCw];
-      const auto issue = [&](uint32_t (*v)[kCw], int c0) {
-#pragma unroll
-        for (int mt = 0; mt < C::kMats; ++mt) tmem_ld8_nowait(tb + mt * kBN + c0, v[mt]);
-      };
-      // this thread's row in the output rows of the tile's tokens: token c of the
-      // tile at out_row + c * stride
-      const size_t stride = GATEUP ? (size_t)a.I : (size_t)a.H;
-      const size_t out_off = (size_t)(row0 + nt * kBN) * stride + (size_t)wrow;
-      const auto finish = [&](uint32_t (*v)[kCw], int c0) {
-        const int valid = n_hi - c0;  // tokens of this chunk that exist (>= 1)
-        size_t o = out_off + (size_t)c0 * stride;
-#pragma unroll
-        for (int j = 0; j < kCw; ++j, o += stride) {
-          if (valid < kCw && j >= valid) break;
-          if (GATEUP)
-            a.h[o] = __float2bfloat16_rn(silu_mul_fast(__uint_as_float(v[0][j]), __uint_as_float(v[C::kMats - 1][j])));
-          else
-            a.y[o] = __uint_as_float(v[0][j]);
-        }
-      };
-      // this warp's tokens: [c_lo, c_hi) of the tile
-      const int c_lo = (kBN / 2) * ehalf;
-      const int c_hi = n_hi < c_lo + kBN / 2 ? n_hi : c_lo + kBN / 2;
-      if (c_lo < c_hi) {
-        issue(va, c_lo);
-        tmem_wait_ld();
-#pragma unroll 1
-        for (int c0 = c_lo; c0 < c_hi; c0 += 2 * kCw) {
-          if (c0 + kCw < c_hi) issue(vb, c0 + kCw);
-          finish(va, c0);
-          tmem_wait_ld();
-          if (c0 + kCw >= c_hi) break;
-          if (c0 + 2 * kCw < c_hi) issue(va, c0 + 2 * kCw);
-          finish(vb, c0 + kCw);
-          tmem_wait_ld();
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[buf]);
-    }
+    for (int tile = blockIdx.x; tile < total && !warp_aborted(abort_flag); tile += gridDim.x, ++tcount)
+      if (!drain(tile, tcount, ehalf)) break;
   }
 
   // ---------------- teardown ----------------
