@@ -58,14 +58,15 @@ bool shape_ok(const moe_q4_layer* L, int T, int top_k) {
 // Workspace layout, every array 256-byte aligned:
 //   header int32[64] | ids int32[T*k] | w f32[T*k] | counts int32[E] |
 //   offsets int32[E+1] | row_token int32[T*k] | inv int32[T*k] |
-//   dec_list int32[E] | pre_list int32[E] | tiles int32[E+1] | h bf16[T*k][I] |
+//   dec_list int32[E] | pre_list int32[E] | mid_list int32[E] | tiles int32[E+1] | h bf16[T*k][I] |
 //   h_lo bf16[T*k][I] | y f32[T*k][H] | xg bf16[T*k][H] (activation rows in
 //   expert order, T > 16 only) | split-tile counters int32[units] | partial sums of the
 //   small-M kernels f32[2*160][4][min(16,T)][128] (two 128-row tiles per unit,
 //   gate/up then down) | with a shared expert: h_s | y_s | its split partial
 //   sums | with the router gate in front: logits f32[T][E] | its partial sums
 struct Layout {
-  size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, tiles, h, h_lo, y, xg, dk_counter,
+  size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, mid_list, tiles, h, h_lo, y, xg,
+      dk_counter,
       dk_partial, h_s, y_s, sx_partial, logits, router_partial, end;
   int dk_units_gu, dk_units_dn, n_max;
 };
@@ -98,6 +99,8 @@ Layout layout(const moe_q4_layer* L, int T, int k, const moe_q4_shared* S = null
   o.dec_list = p;
   p = align_up(p + sizeof(int32_t) * L->E);
   o.pre_list = p;
+  p = align_up(p + sizeof(int32_t) * L->E);
+  o.mid_list = p;
   p = align_up(p + sizeof(int32_t) * L->E);
   o.tiles = p;
   p = align_up(p + sizeof(int32_t) * (L->E + 1));
@@ -188,6 +191,11 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   a.inv = (int32_t*)(ws + o.inv);
   a.dec_list = (int32_t*)(ws + o.dec_list);
   a.pre_list = (int32_t*)(ws + o.pre_list);
+  a.mid_list = (int32_t*)(ws + o.mid_list);
+  // the wide kernel's weight tiles are 256 rows: layers whose I or H is not a
+  // multiple of 256 keep every tensor-core expert on the swap-AB tiles
+  const bool wide_ok = L->I % 256 == 0 && L->H % 256 == 0;
+  a.wide_max = wide_ok ? q4_prefill_wide_max() : kDecodeMaxRows;
   a.tiles = (int32_t*)(ws + o.tiles);
   a.xg = o.xg ? (__nv_bfloat16*)(ws + o.xg) : nullptr;
   a.dk_counter = (int32_t*)(ws + o.dk_counter);
@@ -241,11 +249,13 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   // copy their rows from x themselves)
   if (rc == MOE_Q4_OK && pre) rc = q4_launch_gather(a, s);
   if (rc == MOE_Q4_OK) rc = mark(2);
-  if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, true, s);
+  if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, true, wide_ok, s);
+  if (rc == MOE_Q4_OK && pre && wide_ok) rc = q4_launch_prefill_wide(a, tp, true, s);
   if (rc == MOE_Q4_OK) rc = mark(3);
   if (rc == MOE_Q4_OK) rc = q4_launch_decode(a, tp, true, part_gu, cnt_gu, grid, s);
   if (rc == MOE_Q4_OK) rc = mark(4);
-  if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, false, s);
+  if (rc == MOE_Q4_OK && pre) rc = q4_launch_prefill(a, tp, false, wide_ok, s);
+  if (rc == MOE_Q4_OK && pre && wide_ok) rc = q4_launch_prefill_wide(a, tp, false, s);
   if (rc == MOE_Q4_OK) rc = mark(5);
   if (rc == MOE_Q4_OK) rc = q4_launch_decode(a, tp, false, part_dn, cnt_dn, grid, s);
   if (rc == MOE_Q4_OK && S) {

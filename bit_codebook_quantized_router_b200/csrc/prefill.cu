@@ -48,35 +48,59 @@ constexpr int kBM = 128;          // weight rows per tile (MMA M)
 constexpr int kBK = 64;           // K per pipeline stage (128 bytes of bf16)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-template <bool GATEUP>
+// WIDE: the orientation for experts with few rows (up to 128): the tokens are
+// the MMA's M = 128 rows (the expert's rows, padded) and 256 weight rows its N,
+// so one instruction covers twice the weight rows of the swap-AB tile (a
+// tcgen05.mma costs about the same whatever its N: a 48-token swap-AB tile
+// would use a fifth of it).  The decoded weights are the B operand
+// (K-major, 128-byte swizzle, like the token tile of the swap-AB kernel), the
+// token tile the A operand; the accumulator's TMEM lanes are tokens and its
+// columns weight rows, so each thread stores 8 contiguous outputs of its token.
+template <bool GATEUP, bool WIDE>
 struct TcCfg {
   static constexpr int kMats = GATEUP ? 2 : 1;
-  // dequant warps: one 16-byte code chunk (32 weights) per thread per k-step:
-  // gate/up 2 matrices x 128 rows x 2 chunks, down 128 rows x 2 chunks
+  static constexpr int kWRows = WIDE ? 256 : kBM;     // weight rows per tile
+  static constexpr int kTRows = WIDE ? 128 : kBN;     // token rows per tile
+  // dequant warps: per k-step one 16-byte code chunk (32 weights) of a row per
+  // thread (swap-AB: 128 rows x 2 chunks per matrix) or both chunks of a row
+  // (WIDE: 256 rows per matrix)
   static constexpr int kDequantThreads = kMats * 256;
   static constexpr int kEpiWarp0 = 2 + kDequantThreads / 32;
-  // epilogue: two warps per 32-lane TMEM quarter, each finishing half the tokens
+  // epilogue: two warps per 32-lane TMEM quarter, each finishing half the columns
   static constexpr int kEpiWarps = 8;
   static constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);
-  static constexpr int kStages = GATEUP ? 3 : 4;
-  static constexpr int kATile = kBM * kBK * 2;        // 16 KB bf16 per matrix
-  static constexpr int kBTile = kBN * kBK * 2;        // 16 KB
-  static constexpr int kCTile = kBM * kBK / 2;        // 4 KB codes per matrix
-  static constexpr int kStageBytes = kMats * kATile + kBTile + kMats * kCTile;
+  static constexpr int kATile = kWRows * kBK * 2;     // bf16 weights per matrix
+  static constexpr int kBTile = kTRows * kBK * 2;     // bf16 token tile
+  static constexpr int kCTile = kWRows * kBK / 2;     // codes per matrix
+  // Two rings: the TMA copies (token tile + codes) and the decoded weights.
+  // Swap-AB: as many weight stages as copy stages; WIDE (weight stages of 32
+  // KB per matrix): a short weight ring and a deeper copy ring, so the copies'
+  // latency stays hidden behind the decode.
+  static constexpr int kWStageBytes = kMats * kATile;
+  static constexpr int kTStageBytes = kBTile + kMats * kCTile;
+  static constexpr int kBudget = 227 * 1024 - 2048;
+  static constexpr int kFitBoth = kBudget / (kWStageBytes + kTStageBytes);
+  static constexpr int kStagesW = WIDE ? (GATEUP ? 2 : 3) : (kFitBoth > 4 ? 4 : kFitBoth);
+  static constexpr int kFitT = (kBudget - kStagesW * kWStageBytes) / kTStageBytes;
+  static constexpr int kStagesT = WIDE ? (kFitT > 4 ? 4 : kFitT) : kStagesW;
+  static_assert(kStagesW >= 2 && kStagesT >= kStagesW, "pipeline stages");
+  static constexpr int kAccCols = 256;                // accumulator columns per matrix
   static constexpr int kAccBufs = GATEUP ? 1 : 2;     // TMEM holds 512 columns
   // single-buffered accumulators (gate/up): the dequant warps, idle while the
   // MMA waits for the drain, drain beside the epilogue warps
   static constexpr bool kHelp = kAccBufs == 1;
   static constexpr int kDrainWarps = kEpiWarps + (kHelp ? kDequantThreads / 32 : 0);
   static constexpr int kWorkersPerQuad = kDrainWarps / 4;
-  static constexpr int kTmemCols = kAccBufs * kMats * kBN;
-  static constexpr int kSmem = kStages * kStageBytes + 1024 /*align*/ + 1024 /*barriers*/;
+  static constexpr int kTmemCols = kAccBufs * kMats * kAccCols;
+  static constexpr int kSmem = kStagesW * kWStageBytes + kStagesT * kTStageBytes + 1024 /*align*/ + 1024 /*barriers*/;
+  static_assert(kSmem <= 227 * 1024, "shared memory plan exceeds 227 KB");
 };
 
 struct TcParams {
   FwdArgs a;
-  int m_tiles;  // weight rows / 128
+  int m_tiles;  // weight rows / rows per tile
   int k_steps;  // K / 64
+  int early_trigger;  // swap-AB followed by the WIDE kernel: let it launch once this one's inputs are complete
 };
 
 // Tile id -> (prefill slot p, m-tile, token tile) with tiles ordered
@@ -98,23 +122,24 @@ __device__ __forceinline__ void tile_coords(const FwdArgs& a, int m_tiles, int n
   nt = local - m * n_tiles_p;
 }
 
-template <bool GATEUP>
-__global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
+template <bool GATEUP, bool WIDE>
+__global__ void __launch_bounds__(TcCfg<GATEUP, WIDE>::kThreads, 1)
     tc_gemm_kernel(const __grid_constant__ TcParams P, const __grid_constant__ TableParams tp,
                    const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_wa,
                    const __grid_constant__ CUtensorMap tm_wb) {
-  using C = TcCfg<GATEUP>;
+  using C = TcCfg<GATEUP, WIDE>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;                                        // [S][mats][128][128 B]
-  uint8_t* sB = sA + C::kStages * C::kMats * C::kATile;      // [S][BN][128 B]
-  uint8_t* sC = sB + C::kStages * C::kBTile;                 // [S][mats][128][32 B]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + C::kStages * C::kMats * C::kCTile);
-  uint64_t* full_c = bars;                       // [S] codes landed
-  uint64_t* full_b = full_c + C::kStages;        // [S] token tile landed
-  uint64_t* a_ready = full_b + C::kStages;       // [S] bf16 A tiles written
-  uint64_t* empty = a_ready + C::kStages;        // [S] stage consumed by the MMAs
-  uint64_t* acc_full = empty + C::kStages;       // [2]
+  uint8_t* sA = smem;                                        // [S][mats][weight rows][128 B]
+  uint8_t* sB = sA + C::kStagesW * C::kMats * C::kATile;     // [T][token rows][128 B]
+  uint8_t* sC = sB + C::kStagesT * C::kBTile;                // [T][mats][weight rows][32 B]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sC + C::kStagesT * C::kMats * C::kCTile);
+  uint64_t* full_c = bars;                       // [T] codes landed
+  uint64_t* full_b = full_c + C::kStagesT;       // [T] token tile landed
+  uint64_t* empty = full_b + C::kStagesT;        // [T] copy stage consumed (codes decoded, tokens by the MMAs)
+  uint64_t* a_ready = empty + C::kStagesT;       // [W] decoded weights written
+  uint64_t* a_empty = a_ready + C::kStagesW;     // [W] decoded weights consumed by the MMAs
+  uint64_t* acc_full = a_empty + C::kStagesW;    // [2]
   uint64_t* acc_empty = acc_full + 2;            // [2]
   uint64_t* mma_done = acc_empty + 2;            // [1] final MMA completion
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -124,11 +149,14 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < C::kStagesT; ++s) {
       mbar_init(&full_c[s], 1);
       mbar_init(&full_b[s], 1);
-      mbar_init(&a_ready[s], C::kDequantThreads / 32);  // one arrival per dequant warp
       mbar_init(&empty[s], 1);
+    }
+    for (int w = 0; w < C::kStagesW; ++w) {
+      mbar_init(&a_ready[w], C::kDequantThreads / 32);  // one arrival per dequant warp
+      mbar_init(&a_empty[w], 1);
     }
     for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&acc_full[b], 1);
@@ -150,11 +178,34 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  pdl_wait();
-  const int np = a.hdr[kNumPrefill];
-  const int total = np > 0 ? P.m_tiles * a.tiles[np] : 0;
+  // The WIDE kernel follows the swap-AB kernel of the same projection and
+  // reads nothing that kernel writes: its inputs (routing tables, activation
+  // rows) were complete before the swap-AB kernel's own wait returned, which
+  // precedes that kernel's early trigger, so its CTAs start as the swap-AB
+  // CTAs leave their SMs (filling that grid's last wave); it waits for the
+  // swap-AB grid only before it exits, so the kernels after it still find
+  // both complete.
+  if (!WIDE) pdl_wait();
+  if (!WIDE && P.early_trigger) pdl_trigger();
+  // routing tables: the WIDE kernel reads them through L2 only (no L1 line of
+  // an earlier call can be stale there)
+  const auto rt = [&](const int32_t* q) -> int { return WIDE ? __ldcg(q) : *q; };
+  const int np = WIDE ? rt(a.hdr + kNumMid) : a.hdr[kNumPrefill];
+  const int total = np > 0 ? P.m_tiles * (WIDE ? np : a.tiles[np]) : 0;
   const int rows_total = GATEUP ? a.I : a.H;
   const int K = GATEUP ? a.H : a.I;
+  // tile -> (expert slot p, weight tile m, token tile nt) and the expert;
+  // WIDE: tiles ordered (expert, weight tile), one token tile per expert
+  const auto coords = [&](int tile, int& p, int& m, int& nt) -> int {
+    if (WIDE) {
+      p = tile / P.m_tiles;
+      m = tile - p * P.m_tiles;
+      nt = 0;
+      return rt(a.mid_list + p);
+    }
+    tile_coords(a, P.m_tiles, np, tile, p, m, nt);
+    return a.pre_list[p];
+  };
 
   // Drain of the accumulators of the tcount-th tile of this CTA by one warp:
   // worker `wk` of the C::kWorkersPerQuad warps of its TMEM lane quarter takes
@@ -163,35 +214,61 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
   // the warp signs off on acc_empty.  False when a wait gave up.
   const auto drain = [&](int tile, uint32_t tcount, int wk) -> bool {
     const int quad = warp & 3;          // TMEM lanes 32*quad .. +31
-    const int row = quad * 32 + lane;   // weight row in the tile
+    const int row = quad * 32 + lane;   // weight row (swap-AB) or token (WIDE) in the tile
     int p, m, nt;
-    tile_coords(a, P.m_tiles, np, tile, p, m, nt);
-    int e = a.pre_list[p];
+    int e = coords(tile, p, m, nt);
     if (!q4_check((unsigned)e < (unsigned)a.E, a.hdr + kStatus)) e = 0;
-    int n_e = a.counts[e];
-    const int row0 = a.offsets[e];
+    int n_e = rt(a.counts + e);
+    const int row0 = rt(a.offsets + e);
     // (a failed check leaves the tile's rows unwritten)
     if (!q4_check(row0 >= 0 && n_e >= 0 && row0 + n_e <= a.T * a.k, a.hdr + kStatus)) n_e = nt * kBN;
     const int buf = (int)(tcount % C::kAccBufs);
     const uint32_t use = tcount / C::kAccBufs;
     if (!mbar_wait_warp(&acc_full[buf], use & 1, abort_flag, kWaitLimitNs)) return false;
     tc_fence_after();
-    const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * (C::kMats * kBN);
-    const int wrow = m * kBM + row;
-    const int n_hi = n_e - nt * kBN < kBN ? n_e - nt * kBN : kBN;  // tokens of this tile
+    const uint32_t tb = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * (C::kMats * C::kAccCols);
+    const int wrow = m * C::kWRows + row;
+    const int n_hi = n_e - nt * kBN < kBN ? n_e - nt * kBN : kBN;  // tokens of this tile (swap-AB)
     // 8 token columns of every matrix per chunk; the next chunk's TMEM loads
     // are in flight while this chunk is finished (one wait per chunk)
     constexpr int kCw = 8;
     uint32_t va[C::kMats][kCw], vb[C::kMats][kCw];
     const auto issue = [&](uint32_t (*v)[kCw], int c0) {
 #pragma unroll
-      for (int mt = 0; mt < C::kMats; ++mt) tmem_ld8_nowait(tb + mt * kBN + c0, v[mt]);
+      for (int mt = 0; mt < C::kMats; ++mt) tmem_ld8_nowait(tb + mt * C::kAccCols + c0, v[mt]);
     };
-    // this thread's row in the output rows of the tile's tokens: token c of the
-    // tile at out_row + c * stride
+    // swap-AB: this thread's row in the output rows of the tile's tokens, token
+    // c of the tile at out_off + c * stride; WIDE: this thread's token, its
+    // outputs m * 256 + c contiguous from out_off
     const size_t stride = GATEUP ? (size_t)a.I : (size_t)a.H;
-    const size_t out_off = (size_t)(row0 + nt * kBN) * stride + (size_t)wrow;
+    const size_t out_off = WIDE ? (size_t)(row0 + row) * stride + (size_t)m * C::kWRows
+                                : (size_t)(row0 + nt * kBN) * stride + (size_t)wrow;
+    const bool tok_ok = !WIDE || row < n_e;  // WIDE: lanes past the expert's rows store nothing
+    const auto finish_wide = [&](uint32_t (*v)[kCw], int c0) {
+      if (!tok_ok) return;
+      if (GATEUP) {
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __nv_bfloat162 hv = __floats2bfloat162_rn(
+              silu_mul_fast(__uint_as_float(v[0][2 * j]), __uint_as_float(v[1][2 * j])),
+              silu_mul_fast(__uint_as_float(v[0][2 * j + 1]), __uint_as_float(v[1][2 * j + 1])));
+          w[j] = *reinterpret_cast<const uint32_t*>(&hv);
+        }
+        *reinterpret_cast<uint4*>(a.h + out_off + c0) = make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+        float4* yo = reinterpret_cast<float4*>(a.y + out_off + c0);
+        yo[0] = make_float4(__uint_as_float(v[0][0]), __uint_as_float(v[0][1]), __uint_as_float(v[0][2]),
+                            __uint_as_float(v[0][3]));
+        yo[1] = make_float4(__uint_as_float(v[0][4]), __uint_as_float(v[0][5]), __uint_as_float(v[0][6]),
+                            __uint_as_float(v[0][7]));
+      }
+    };
     const auto finish = [&](uint32_t (*v)[kCw], int c0) {
+      if (WIDE) {
+        finish_wide(v, c0);
+        return;
+      }
       const int valid = n_hi - c0;  // tokens of this chunk that exist (>= 1)
       size_t o = out_off + (size_t)c0 * stride;
 #pragma unroll
@@ -203,11 +280,12 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
           a.y[o] = __uint_as_float(v[0][j]);
       }
     };
-    // this warp's tokens: chunks [wk n / W, (wk + 1) n / W) of the n = kBN / 8
-    constexpr int kChunks = kBN / kCw;
+    // this warp's columns (tokens; WIDE: weight rows): chunks [wk n / W,
+    // (wk + 1) n / W) of the n = 256 / 8
+    constexpr int kChunks = C::kAccCols / kCw;
     const int c_lo = kCw * (wk * kChunks / C::kWorkersPerQuad);
     const int c_end = kCw * ((wk + 1) * kChunks / C::kWorkersPerQuad);
-    const int c_hi = n_hi < c_end ? n_hi : c_end;
+    const int c_hi = WIDE ? c_end : (n_hi < c_end ? n_hi : c_end);
     if (c_lo < c_hi) {
       issue(va, c_lo);
       tmem_wait_ld();
@@ -234,18 +312,24 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
       uint32_t it = 0;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
         int p, m, nt;
-        tile_coords(a, P.m_tiles, np, tile, p, m, nt);
-        int e = a.pre_list[p];
+        int e = coords(tile, p, m, nt);
         if (!q4_check((unsigned)e < (unsigned)a.E, a.hdr + kStatus)) e = 0;
-        const int wrow = e * rows_total + m * kBM;
-        const int brow = a.offsets[e] + nt * kBN;
+        const int wrow = e * rows_total + m * C::kWRows;
+        const int brow = rt(a.offsets + e) + nt * C::kTRows;
         for (int ks = 0; ks < P.k_steps; ++ks, ++it) {
-          const int s = it % C::kStages;
-          const uint32_t ph = (it / C::kStages) & 1;
+          const int s = it % C::kStagesT;
+          const uint32_t ph = (it / C::kStagesT) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) break;
           mbar_arrive_expect_tx(&full_c[s], C::kMats * C::kCTile);
-          tma_load_2d(sC + (s * C::kMats) * C::kCTile, &tm_wa, &full_c[s], ks * (kBK / 2), wrow);
-          if (GATEUP) tma_load_2d(sC + (s * C::kMats + 1) * C::kCTile, &tm_wb, &full_c[s], ks * (kBK / 2), wrow);
+          // codes: boxes of 128 rows (two per matrix for a 256-row WIDE tile)
+#pragma unroll
+          for (int h = 0; h < C::kWRows / kBM; ++h) {
+            tma_load_2d(sC + (s * C::kMats) * C::kCTile + h * (kBM * kBK / 2), &tm_wa, &full_c[s], ks * (kBK / 2),
+                        wrow + h * kBM);
+            if (GATEUP)
+              tma_load_2d(sC + (s * C::kMats + 1) * C::kCTile + h * (kBM * kBK / 2), &tm_wb, &full_c[s],
+                          ks * (kBK / 2), wrow + h * kBM);
+          }
           mbar_arrive_expect_tx(&full_b[s], C::kBTile);
           tma_load_2d(sB + s * C::kBTile, &tm_b, &full_b[s], ks * kBK, brow);
         }
@@ -257,21 +341,25 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
       uint32_t it = 0, tcount = 0;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++tcount) {
         int p, m, nt;
-        tile_coords(a, P.m_tiles, np, tile, p, m, nt);
-        const int left = a.counts[a.pre_list[p]] - nt * kBN;  // tokens in this tile and after
+        const int e = coords(tile, p, m, nt);
+        // swap-AB: M = 128 weight rows, N = the tile's tokens rounded up to 16;
+        // WIDE: M = 128 token rows (padded), N = 256 weight rows
+        const int left = rt(a.counts + e) - nt * kBN;  // tokens in this tile and after
         const int n_cols = left >= kBN ? kBN : ((left + 15) & ~15);
-        const uint32_t idesc = umma_idesc_bf16(kBM, n_cols);
+        const uint32_t idesc = WIDE ? umma_idesc_bf16(128, 256) : umma_idesc_bf16(kBM, n_cols);
         const int buf = (int)(tcount % C::kAccBufs);
         const uint32_t use = tcount / C::kAccBufs;  // earlier uses of this buffer
         if (!mbar_wait(&acc_empty[buf], (use & 1) ^ 1, abort_flag, kWaitLimitNs)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem_base + buf * (C::kMats * kBN);
+        const uint32_t d0 = tmem_base + buf * (C::kMats * C::kAccCols);
         bool ok = true;
         for (int ks = 0; ks < P.k_steps; ++ks, ++it) {
-          const int s = it % C::kStages;
-          const uint32_t ph = (it / C::kStages) & 1;
+          const int s = it % C::kStagesT;
+          const uint32_t ph = (it / C::kStagesT) & 1;
+          const int w = it % C::kStagesW;
+          const uint32_t wph = (it / C::kStagesW) & 1;
           if (!mbar_wait(&full_b[s], ph, abort_flag, kWaitLimitNs) ||
-              !mbar_wait(&a_ready[s], ph, abort_flag, kWaitLimitNs)) {
+              !mbar_wait(&a_ready[w], wph, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
           }
@@ -279,11 +367,16 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
           const uint64_t db = umma_desc_sw128(smem_u32(sB + s * C::kBTile));
 #pragma unroll
           for (int mat = 0; mat < C::kMats; ++mat) {
-            const uint64_t da = umma_desc_sw128(smem_u32(sA + (s * C::kMats + mat) * C::kATile));
+            const uint64_t da = umma_desc_sw128(smem_u32(sA + (w * C::kMats + mat) * C::kATile));
 #pragma unroll
-            for (int kk = 0; kk < kBK / 16; ++kk)  // +32 bytes of K per MMA (>> 4 -> +2)
-              umma_bf16(d0 + mat * kBN, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0);
+            for (int kk = 0; kk < kBK / 16; ++kk) {  // +32 bytes of K per MMA (>> 4 -> +2)
+              if (WIDE)  // A: the token tile, B: the weights
+                umma_bf16(d0 + mat * C::kAccCols, db + 2 * kk, da + 2 * kk, idesc, (ks | kk) != 0);
+              else
+                umma_bf16(d0 + mat * C::kAccCols, da + 2 * kk, db + 2 * kk, idesc, (ks | kk) != 0);
+            }
           }
+          umma_commit(&a_empty[w]);
           umma_commit(&empty[s]);
         }
         if (!ok) break;
@@ -296,23 +389,23 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
   } else if (warp < C::kEpiWarp0) {
     // ---------------- dequantise ----------------
     const int d = threadIdx.x - 64;           // 0 .. kDequantThreads - 1
-    const int r = d & (kBM - 1);              // weight row in the tile
-    const int my_half = (d >> 7) & 1;         // 32-weight half of the row's 64 K
+    const int r = d & (C::kWRows - 1);        // weight row in the tile
+    const int my_half = WIDE ? -1 : (d >> 7) & 1;  // 32-weight half of the row's 64 K (WIDE: both)
     const int mat = GATEUP ? (d >> 8) : 0;    // gate / up
     // drain worker index of this warp in its TMEM lane quarter (after the
     // epilogue warps'); it helps drain tile n while working on tile n + 1,
     // once the ring is full and the MMA waits for that drain
     const int help_wk = C::kEpiWarps / 4 + ((warp - 2) >> 2);
-    const int help_at = P.k_steps - 1 < C::kStages ? P.k_steps - 1 : C::kStages;
+    const int help_at = P.k_steps - 1 < C::kStagesW ? P.k_steps - 1 : C::kStagesW;
     int prev_tile = -1;
     uint32_t it = 0, tcount = 0;
     for (int tile = blockIdx.x; tile < total && !warp_aborted(abort_flag); tile += gridDim.x, ++tcount) {
       int p, m, nt;
-      tile_coords(a, P.m_tiles, np, tile, p, m, nt);
-      const int e = a.pre_list[p];
+      int e = coords(tile, p, m, nt);
+      if (!q4_check((unsigned)e < (unsigned)a.E, a.hdr + kStatus)) e = 0;
       const Planes PL = make_planes(tp.t[tp.id[e]]);
       const uint8_t* srow = (GATEUP ? (mat ? a.up_s : a.gate_s) : a.down_s) +
-                            ((size_t)e * rows_total + m * kBM + r) * (size_t)(K / 32);
+                            ((size_t)e * rows_total + m * C::kWRows + r) * (size_t)(K / 32);
       // scale bytes of blocks 2ks .. 2ks+3 (k-steps ks, ks+1) as one 4-byte word
       // (K % 128 == 0 keeps every word inside the row and aligned), loaded three
       // words ahead of use so the loads' latency hides behind the decode
@@ -332,19 +425,24 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
           q1 = q2;
           q2 = (ks >> 1) + 3 < n_sw ? sw32[(ks >> 1) + 3] : 0u;
         }
-        const int s = it % C::kStages;
-        const uint32_t ph = (it / C::kStages) & 1;
-        if (!mbar_wait_warp(&full_c[s], ph, abort_flag, kWaitLimitNs)) {
+        const int s = it % C::kStagesT;
+        const uint32_t ph = (it / C::kStagesT) & 1;
+        const int w = it % C::kStagesW;
+        const uint32_t wph = (it / C::kStagesW) & 1;
+        // the codes have landed and the weight stage is free (its previous
+        // contents consumed by the MMAs)
+        if (!mbar_wait_warp(&full_c[s], ph, abort_flag, kWaitLimitNs) ||
+            !mbar_wait_warp(&a_empty[w], wph ^ 1, abort_flag, kWaitLimitNs)) {
           ok = false;
           break;
         }
         const uint8_t* ctile = sC + (s * C::kMats + mat) * C::kCTile;
-        uint8_t* arow = sA + (s * C::kMats + mat) * C::kATile + r * 128;
+        uint8_t* arow = sA + (w * C::kMats + mat) * C::kATile + r * 128;
         // 32-byte swizzle of the codes tile: chunk c of row r at c ^ ((r >> 2) & 1)
         const int sw = (r >> 2) & 1;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          if (half != my_half) continue;
+          if (!WIDE && half != my_half) continue;
           const uint4 cv = *reinterpret_cast<const uint4*>(ctile + r * 32 + ((half ^ sw) << 4));
           const int blk = 2 * (ks & 1) + half;  // block within the 4 loaded
           const uint32_t sbyte = (sc >> (blk * 8)) & 0xffu;
@@ -364,7 +462,7 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&a_ready[s]);
+        if (lane == 0) mbar_arrive(&a_ready[w]);
       }
       if (!ok) break;
       prev_tile = tile;
@@ -384,7 +482,7 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
   if (threadIdx.x == 0 && *abort_flag) record_error(a.hdr + kStatus, MOE_Q4_ETIMEOUT);
   if (warp == 0 && lane == 0 && *abort_flag) {
     // let any copy still in flight land before the CTA's smem goes away
-    for (int s = 0; s < C::kStages; ++s) {
+    for (int s = 0; s < C::kStagesT; ++s) {
       volatile int quick = 0;
       mbar_wait(&full_c[s], 0, &quick, 50000000ull);
       quick = 0;
@@ -400,9 +498,11 @@ __global__ void __launch_bounds__(TcCfg<GATEUP>::kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
   }
-  // triggered at the end: the next kernel's CTAs (shared memory near the SM's
-  // limit) could not share an SM with this one anyway, and launching them while
-  // this persistent grid still runs measured slower
+  // the WIDE kernel completes only after the swap-AB grid before it
+  if (WIDE) pdl_wait();
+  // triggered at the end (unless early, above): the next kernel's CTAs (shared
+  // memory near the SM's limit) could not share an SM with this one anyway, and
+  // launching them while this persistent grid still runs measured slower
   pdl_trigger();
 }
 
@@ -438,30 +538,33 @@ static bool make_map(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, c
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool GATEUP>
-static int launch_tc(const FwdArgs& a, const TableParams& tp, cudaStream_t s) {
-  using C = TcCfg<GATEUP>;
+template <bool GATEUP, bool WIDE>
+static int launch_tc(const FwdArgs& a, const TableParams& tp, cudaStream_t s, bool wide_next) {
+  using C = TcCfg<GATEUP, WIDE>;
   TcParams P;
   P.a = a;
-  P.m_tiles = (GATEUP ? a.I : a.H) / kBM;
+  P.m_tiles = (GATEUP ? a.I : a.H) / C::kWRows;
   P.k_steps = (GATEUP ? a.H : a.I) / kBK;
+  P.early_trigger = !WIDE && wide_next;
   const int R = a.T * a.k;
   CUtensorMap tb, twa, twb;
   bool ok;
   if (GATEUP) {
-    ok = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.xg, a.H, R, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+    ok = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.xg, a.H, R, kBK, C::kTRows,
+                  CU_TENSOR_MAP_SWIZZLE_128B) &&
          make_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.gate_w, a.H / 2, (uint64_t)a.E * a.I, kBK / 2, kBM,
                   CU_TENSOR_MAP_SWIZZLE_32B) &&
          make_map(&twb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.up_w, a.H / 2, (uint64_t)a.E * a.I, kBK / 2, kBM,
                   CU_TENSOR_MAP_SWIZZLE_32B);
   } else {
-    ok = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.h, a.I, R, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B) &&
+    ok = make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.h, a.I, R, kBK, C::kTRows,
+                  CU_TENSOR_MAP_SWIZZLE_128B) &&
          make_map(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.down_w, a.I / 2, (uint64_t)a.E * a.H, kBK / 2, kBM,
                   CU_TENSOR_MAP_SWIZZLE_32B);
     twb = twa;
   }
   if (!ok) return MOE_Q4_ECUDA;
-  if (cudaFuncSetAttribute(tc_gemm_kernel<GATEUP>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
+  if (cudaFuncSetAttribute(tc_gemm_kernel<GATEUP, WIDE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem) !=
       cudaSuccess)
     return MOE_Q4_ECUDA;
   int dev = 0, sms = 148;
@@ -477,8 +580,8 @@ static int launch_tc(const FwdArgs& a, const TableParams& tp, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<GATEUP>, P, tp, tb, twa, twb) == cudaSuccess ? MOE_Q4_OK
-                                                                                                  : MOE_Q4_ECUDA;
+  return cudaLaunchKernelEx(&cfg, tc_gemm_kernel<GATEUP, WIDE>, P, tp, tb, twa, twb) == cudaSuccess ? MOE_Q4_OK
+                                                                                                      : MOE_Q4_ECUDA;
 }
 
 }  // namespace q4
@@ -487,6 +590,12 @@ using namespace q4;
 
 int q4_prefill_tile_n() { return kBN; }
 
-int q4_launch_prefill(const FwdArgs& a, const TableParams& tp, bool gateup, cudaStream_t s) {
-  return gateup ? launch_tc<true>(a, tp, s) : launch_tc<false>(a, tp, s);
+int q4_prefill_wide_max() { return 128; }
+
+int q4_launch_prefill(const FwdArgs& a, const TableParams& tp, bool gateup, bool wide_next, cudaStream_t s) {
+  return gateup ? launch_tc<true, false>(a, tp, s, wide_next) : launch_tc<false, false>(a, tp, s, wide_next);
+}
+
+int q4_launch_prefill_wide(const FwdArgs& a, const TableParams& tp, bool gateup, cudaStream_t s) {
+  return gateup ? launch_tc<true, true>(a, tp, s, false) : launch_tc<false, true>(a, tp, s, false);
 }

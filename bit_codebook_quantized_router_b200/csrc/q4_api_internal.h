@@ -15,6 +15,8 @@ struct TableParams;
 struct FwdArgs {
   int T, k, E, H, I;
   int dec_max;     // experts with 1..dec_max rows take the streaming path
+  int wide_max;    // experts with dec_max+1..wide_max rows take the wide tensor-core kernel
+                   // (tokens as MMA M, 256 weight rows as N); more rows: swap-AB tiles
   int tile_n;      // token tile of the tensor-core path
   const __nv_bfloat16* x;  // [T][H]
   const float* logits;     // [T][E]
@@ -28,6 +30,7 @@ struct FwdArgs {
   int32_t* inv;            // [T*k]
   int32_t* dec_list;       // [E]
   int32_t* pre_list;       // [E]
+  int32_t* mid_list;       // [E] experts of the wide tensor-core kernel (nullptr: none)
   int32_t* tiles;          // [E+1] token-tile offsets of the tensor-core-path experts
   __nv_bfloat16* h;        // [T*k][I] bf16 rounding of silu(g)*u
   __nv_bfloat16* h_lo;     // [T*k][I] bf16 rounding of the remainder silu(g)*u - h
@@ -63,7 +66,11 @@ int q4_launch_router(const void* x, const void* w, int T, int H, int E, float* l
 bool q4_router_route_fused(int T, int H, int k);
 int q4_launch_router_route(const q4::FwdArgs& a, const void* w, cudaStream_t s);
 int q4_launch_gather(const q4::FwdArgs& a, cudaStream_t s);
-int q4_launch_prefill(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, cudaStream_t s);
+// wide_next: the WIDE kernel is launched right after (see prefill.cu)
+int q4_launch_prefill(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, bool wide_next, cudaStream_t s);
+// the wide tensor-core kernel (experts with dec_max+1 .. q4_prefill_wide_max() rows)
+int q4_prefill_wide_max();
+int q4_launch_prefill_wide(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, cudaStream_t s);
 int q4_prefill_tile_n();
 int q4_launch_decode(const q4::FwdArgs& a, const q4::TableParams& tp, bool gateup, float* partial,
                         int32_t* counter, int grid, cudaStream_t s);

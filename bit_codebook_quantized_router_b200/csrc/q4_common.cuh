@@ -35,6 +35,7 @@ enum HeaderWord : int {
   kNumPrefill = 2, // experts on the tensor-core path
   kNumTiles = 3,   // tensor-core path work tiles
   kRouterTicket = 4,  // CTAs of the fused router + routing kernel done with their logits
+  kNumMid = 5,     // experts on the wide tensor-core kernel
   kHeaderWords = 64,
 };
 

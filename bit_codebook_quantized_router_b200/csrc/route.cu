@@ -80,9 +80,11 @@ __device__ void group_rows(const FwdArgs& a, int* sm) {
   const int c = tid < E ? counts[tid] : 0;
   int total;
   const int off = block_exclusive_scan(c, warp_tot, total);
-  const bool fd = c > 0 && c <= a.dec_max, fp = c > a.dec_max;
-  int nd, np;
+  const int wmax = a.mid_list ? a.wide_max : a.dec_max;
+  const bool fd = c > 0 && c <= a.dec_max, fm = c > a.dec_max && c <= wmax, fp = c > wmax;
+  int nd, nm, np;
   const int pd = block_exclusive_scan(fd ? 1 : 0, warp_tot, nd);
+  const int pm = block_exclusive_scan(fm ? 1 : 0, warp_tot, nm);
   const int pp = block_exclusive_scan(fp ? 1 : 0, warp_tot, np);
   // token tiles of each tensor-core-path expert, as an exclusive scan in
   // pre_list order (tiles[p] .. tiles[p+1]-1 are expert pre_list[p]'s)
@@ -95,6 +97,7 @@ __device__ void group_rows(const FwdArgs& a, int* sm) {
     a.counts[tid] = c;
     if (a.user_counts) a.user_counts[tid] = c;
     if (fd) a.dec_list[pd] = tid;
+    if (fm) a.mid_list[pm] = tid;
     if (fp) a.pre_list[pp] = tid;
     if (fp && a.tiles) a.tiles[pp] = ntoff;
   }
@@ -102,6 +105,7 @@ __device__ void group_rows(const FwdArgs& a, int* sm) {
     offs[E] = total;
     a.offsets[E] = total;
     a.hdr[kNumDecode] = nd;
+    a.hdr[kNumMid] = nm;
     a.hdr[kNumPrefill] = np;
     a.hdr[kNumTiles] = ntot;
     if (a.tiles) a.tiles[np] = ntot;

@@ -73,14 +73,17 @@ __device__ void route_small(const FwdArgs& a, int* sm) {
     }
   }
   __syncthreads();
-  // one exclusive scan over experts of four 16-bit fields:
-  //   rows | small-M experts | tensor-core experts | tensor-core tiles
-  // (T*k <= 4096 rows and E <= 512 experts: no field overflows)
+  // one exclusive scan over experts of five packed fields:
+  //   rows [0,13) | small-M experts [13,23) | wide experts [23,33) |
+  //   swap-AB experts [33,43) | their tiles [43,55)
+  // (T*k <= 4096 rows, E <= 512 experts, tiles <= E + T*k/16: no field overflows)
+  const int wmax = a.mid_list ? a.wide_max : a.dec_max;
   const auto pack = [&](int c) -> unsigned long long {
-    const bool fd = c > 0 && c <= a.dec_max, fp = c > a.dec_max;
+    const bool fd = c > 0 && c <= a.dec_max, fm = c > a.dec_max && c <= wmax, fp = c > wmax;
     const int ntl = fp ? (c + a.tile_n - 1) / a.tile_n : 0;
-    return (unsigned long long)c | ((unsigned long long)(fd ? 1 : 0) << 16) |
-           ((unsigned long long)(fp ? 1 : 0) << 32) | ((unsigned long long)ntl << 48);
+    return (unsigned long long)c | ((unsigned long long)(fd ? 1 : 0) << 13) |
+           ((unsigned long long)(fm ? 1 : 0) << 23) | ((unsigned long long)(fp ? 1 : 0) << 33) |
+           ((unsigned long long)ntl << 43);
   };
   const int per = (E + NTH - 1) / NTH;
   const int e0 = tid * per, e1 = e0 + per < E ? e0 + per : E;
@@ -108,27 +111,29 @@ __device__ void route_small(const FwdArgs& a, int* sm) {
   __syncthreads();
   unsigned long long ex = warp_tot[warp] + inc - v;
   const unsigned long long tot = warp_tot[32];
+  const auto field = [](unsigned long long x, int lo, int bits) -> int {
+    return (int)((x >> lo) & ((1ull << bits) - 1));
+  };
   for (int e = e0; e < e1; ++e) {
     const int c = counts[e];
     const unsigned long long pe = pack(c);
-    const int off = (int)(ex & 0xffffu), pd = (int)((ex >> 16) & 0xffffu);
-    const int pp = (int)((ex >> 32) & 0xffffu), ntoff = (int)(ex >> 48);
-    offs[e] = off;
-    a.offsets[e] = off;
+    offs[e] = field(ex, 0, 13);
+    a.offsets[e] = field(ex, 0, 13);
     a.counts[e] = c;
     if (a.user_counts) a.user_counts[e] = c;
-    if ((pe >> 16) & 1u) a.dec_list[pd] = e;
-    if ((pe >> 32) & 1u) {
-      a.pre_list[pp] = e;
-      if (a.tiles) a.tiles[pp] = ntoff;
+    if (field(pe, 13, 10)) a.dec_list[field(ex, 13, 10)] = e;
+    if (field(pe, 23, 10)) a.mid_list[field(ex, 23, 10)] = e;
+    if (field(pe, 33, 10)) {
+      a.pre_list[field(ex, 33, 10)] = e;
+      if (a.tiles) a.tiles[field(ex, 33, 10)] = field(ex, 43, 12);
     }
     ex += pe;
   }
   if (tid == 0) {
-    const int total = (int)(tot & 0xffffu), nd = (int)((tot >> 16) & 0xffffu);
-    const int np = (int)((tot >> 32) & 0xffffu), ntot = (int)(tot >> 48);
-    a.offsets[E] = total;
-    a.hdr[kNumDecode] = nd;
+    const int np = field(tot, 33, 10), ntot = field(tot, 43, 12);
+    a.offsets[E] = field(tot, 0, 13);
+    a.hdr[kNumDecode] = field(tot, 13, 10);
+    a.hdr[kNumMid] = field(tot, 23, 10);
     a.hdr[kNumPrefill] = np;
     a.hdr[kNumTiles] = ntot;
     if (a.tiles) a.tiles[np] = ntot;

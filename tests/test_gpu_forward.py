@@ -83,6 +83,27 @@ def test_small_layer_edge_counts(T, k, bias):
     gpu_support.check_out(out, ref, f"T={T} k={k}")
 
 
+# The wide tensor-core tiles (experts with 17 to 128 rows: the tokens as MMA M,
+# 256 weight rows as N) on a layer whose I and H are multiples of 256 (H=512,
+# I=256, E=8): an expert with exactly the small-M limit (16 rows) and one more
+# (17), with the wide limit (128) and one more (129, swap-AB), a mix of wide
+# and swap-AB experts, and k = E (every expert wide).  Every token against the
+# oracle.
+@pytest.mark.parametrize("T,k,bias", [(16, 1, 3), (17, 1, 3), (128, 1, 3), (129, 1, 3), (100, 2, None),
+                                      (300, 3, 0), (60, 8, None)])
+def test_wide_tensor_core_tiles(T, k, bias):
+    w = inputs.Workload("wide", 18, T, inputs.Shape(H=512, I=256, E=8, k=k))
+    L, dev = _small_device_layer(w)
+    x = inputs.activations(w)
+    lg = inputs.router_logits(w)
+    if bias is not None:
+        lg[:, bias] += 50.0  # every token picks expert `bias` first
+    out, ids, wts, counts = _run(dev, x.cuda(), lg.cuda(), k)
+    ref, rids, _ = oracle.moe_tokens(L, inputs.bf16_bits(x), lg.numpy(), k, return_routing=True)
+    assert np.array_equal(ids.cpu().numpy(), rids)
+    gpu_support.check_out(out, ref, f"wide tiles T={T} k={k}")
+
+
 # K a multiple of 128 but not of 256 (H = I = 384): the small-M path streams
 # 128-K stages of 64-byte code rows, several per tile; T <= 8 and T > 8 take
 # the two activation tile heights of the down projection.
