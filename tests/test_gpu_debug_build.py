@@ -1,7 +1,8 @@
 """The bounds-checking debug build (libmoe_q4_debug.so, MOE_Q4_DEBUG): the
 same forward through its C ABI gives the release build's bits and a clean
 status (no device index check fails on valid inputs), on the tiny layer, the
-small-M and tensor-core paths of a small layer, and the GLM decode layer."""
+small-M and tensor-core paths of a small layer, the wide tensor-core tiles of
+a layer whose I and H are multiples of 256, and the GLM decode layer."""
 import ctypes
 
 import pytest
@@ -47,6 +48,14 @@ def _both(dev, x, lg, k):
 @pytest.mark.parametrize("T,k", [(4, 2), (1, 2), (16, 3), (300, 2)])
 def test_debug_build_matches_release_on_small_layers(T, k):
     w = inputs.Workload("dbg", 17, T, inputs.TINY)
+    _, dev = _small_device_layer(w)
+    got, ref = _both(dev, inputs.activations(w).cuda(), inputs.router_logits(w).cuda(), k)
+    assert torch.equal(got, ref)
+
+
+@pytest.mark.parametrize("T,k", [(100, 2), (300, 3)])
+def test_debug_build_matches_release_on_wide_tiles(T, k):
+    w = inputs.Workload("dbg_wide", 19, T, inputs.Shape(H=512, I=256, E=8, k=k))
     _, dev = _small_device_layer(w)
     got, ref = _both(dev, inputs.activations(w).cuda(), inputs.router_logits(w).cuda(), k)
     assert torch.equal(got, ref)
