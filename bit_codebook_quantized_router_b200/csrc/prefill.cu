@@ -6,30 +6,35 @@
 // decisions" 4 and 6), for the experts whose row count exceeds the streaming
 // path's limit.
 //
-// Swap-AB grouped GEMM: the MMA's M = 128 weight rows, N = a tile of up to
-// BN = 256 tokens of one expert (the expert's last tile takes N = its
-// remaining rows rounded up to 16), K streamed in steps of 64.  Each decoded
-// 128 x 64 weight tile feeds N = 256 columns of MMA work, so the tensor core,
-// not the decode, sets the pace.  A persistent CTA per SM walks tiles ordered
-// (expert, weight m-tile, token tile) so the token tiles of one weight tile
-// run back to back and re-read it from L2.
+// Two tile orientations of one kernel template:
+// * swap-AB (experts with more than 128 rows): the MMA's M = 128 weight rows,
+//   N = a tile of up to 256 tokens of one expert (the expert's last tile takes
+//   N = its remaining rows rounded up to 16), K streamed in steps of 64.  A
+//   persistent CTA per SM walks tiles ordered (expert, weight m-tile, token
+//   tile) so the token tiles of one weight tile run back to back and re-read
+//   it from L2.
+// * WIDE (experts with 17..128 rows, layers whose I and H are multiples of
+//   256): M = the expert's (padded) 128 token rows, N = 256 weight rows; tiles
+//   (expert, 256-row weight tile).  See TcCfg.
 //
-// Warp roles (448 threads):
-//   warp 0       TMA producer: packed codes of the m-tile (128 rows x 32 B per
-//                k-step, 32-byte swizzle) and the token tile (BN rows x 128 B,
-//                128-byte swizzle) into a 3-4 stage ring;
+// Warp roles:
+//   warp 0       TMA producer: packed codes of the weight tile (128-row boxes
+//                x 32 B per k-step, 32-byte swizzle) and the token tile (128
+//                bytes of K per row, 128-byte swizzle) into the copy ring;
 //   warp 1       allocates TMEM and issues tcgen05.mma (one thread): for each
 //                k-step, 4 MMAs of K=16 per weight matrix into fp32 TMEM
 //                accumulators (gate + up fill all 512 columns: one buffer;
 //                down: double-buffered across tiles);
-//   warps 2..9   dequantise: codes -> bf16 through the PRMT byte-plane lookup
+//   next 8 or 16 dequantise: codes -> bf16 through the PRMT byte-plane lookup
 //                of the expert's table, E8M0 scale by an exact bf16x2
-//                multiply, stored to smem in the canonical 128-byte-swizzle
-//                K-major layout the MMA reads ("aidendle94/GLM-5.2-NF4-Lloyd-
-//                Experts-GPTQ", "Codes are indices into the per-layer grid");
-//   warps 10..13 epilogue: tcgen05.ld of the accumulators (one TMEM lane = one
-//                weight row per thread), SwiGLU in fp32, bf16 stores of h (or
-//                fp32 stores of y).
+//                multiply, stored to the decoded-weight ring in the canonical
+//                128-byte-swizzle K-major layout the MMA reads ("aidendle94/
+//                GLM-5.2-NF4-Lloyd-Experts-GPTQ", "Codes are indices into the
+//                per-layer grid"); with single-buffered accumulators they also
+//                help drain them while the MMA waits for that drain;
+//   last 8       epilogue: tcgen05.ld of the accumulators (one TMEM lane = one
+//                weight row, or one token for WIDE tiles), SwiGLU in fp32,
+//                bf16 stores of h (or fp32 stores of y).
 // Every mbarrier wait is bounded; on a timeout the CTA sets the status word
 // to MOE_Q4_ETIMEOUT, drains its own copies and MMAs (bounded), frees TMEM
 // and exits.
