@@ -63,10 +63,12 @@ class DispatchPlan:
 def plan_dispatch(ids: torch.Tensor, E: int, world: int) -> DispatchPlan:
     """Order the (token, slot) rows of ids [T][k] by (owner rank, expert,
     token, slot) -- a stable sort on owner * E + expert of the row-major flat
-    rows -- and count the rows per destination rank."""
-    flat = ids.reshape(-1).to(torch.int64).cpu()
-    own = owner_of(E, world)
-    first = torch.tensor([a for a, _ in expert_ranges(E, world)], dtype=torch.int64)
+    rows, on the ids' own device -- and count the rows per destination rank
+    (the only values that go to the host: the collective's split sizes)."""
+    dev = ids.device
+    flat = ids.reshape(-1).to(torch.int64)
+    own = owner_of(E, world).to(dev)
+    first = torch.tensor([a for a, _ in expert_ranges(E, world)], dtype=torch.int64, device=dev)
     key = own[flat] * E + flat
     order = torch.sort(key, stable=True).indices
     counts = torch.bincount(own[flat], minlength=world).tolist()
@@ -109,16 +111,16 @@ def ep_moe(x: torch.Tensor, ids: torch.Tensor, w: torch.Tensor, E: int, compute,
     the dtype compute() returns (fp32 on the GPU)."""
     T, k = ids.shape
     H = x.shape[1]
-    plan = plan_dispatch(ids, E, world)
+    plan = plan_dispatch(ids.to(x.device), E, world)
     recv_counts = _exchange_counts(plan.send_counts, group, x.device)
-    rows = x[(plan.order // k).to(x.device)]
+    rows = x[plan.order // k]
     recv_x = _a2a(rows, plan.send_counts, recv_counts, group)
-    recv_ids = _a2a(plan.local_ids.to(x.device), plan.send_counts, recv_counts, group)
+    recv_ids = _a2a(plan.local_ids, plan.send_counts, recv_counts, group)
     y_recv = compute(recv_x, recv_ids) if recv_x.shape[0] else torch.zeros((0, H), dtype=out_dtype,
                                                                              device=x.device)
     y_back = _a2a(y_recv.contiguous(), recv_counts, plan.send_counts, group)
     y = torch.empty((T * k, H), dtype=out_dtype, device=x.device)
-    y[plan.order.to(x.device)] = y_back
+    y[plan.order] = y_back
     return combine(y, w)
 
 

@@ -96,15 +96,22 @@ def test_small_layer_gated(T, k):
     gpu_support.check_out(g["out_f32"], ref, f"gated T={T} k={k}")
 
 
-def test_small_layer_gated_with_shared_expert():
-    w = inputs.Workload("gated_shared", 22, 6, inputs.TINY)
-    _, dev = _small_device_layer(w)
+# with a shared expert: at a decode size (fused router + routing) and above it
+# (the router kernels, the routing kernels, then the shared expert's launches)
+@pytest.mark.parametrize("T", [6, 40])
+def test_small_layer_gated_with_shared_expert(T):
+    w = inputs.Workload("gated_shared", 22, T, inputs.TINY)
+    L, dev = _small_device_layer(w)
     gu, dn = inputs.shared_expert_weights(w, I=128, device="cuda")
     sh = q4.Shared(gu, dn)
     gate = inputs.router_weight(w, device="cuda")
     x = inputs.activations(w).cuda()
     g = _gated_guarded(dev, sh, gate, x, 2)
     _check_against_router_and_forward(dev, sh, gate, x, 2, g)
+    lg_h = _check_logits_and_routing(gate, x, 2, g)
+    x_bits = inputs.bf16_bits(x)
+    ref = oracle.moe_tokens(L, x_bits, lg_h, 2) + oracle.shared_ffn(x_bits, inputs.bf16_bits(gu), inputs.bf16_bits(dn))
+    gpu_support.check_out(g["out_f32"], ref, f"gated + shared expert T={T}")
 
 
 def test_gated_calls_in_a_row_share_one_workspace():
