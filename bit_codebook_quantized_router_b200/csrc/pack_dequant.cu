@@ -96,16 +96,18 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint16_t* __restrict__ 
 // 512 contiguous output bytes; each thread takes kDqWords words a grid stride
 // apart, loads first, so several loads are in flight per thread.
 // Fast path (the block's scale keeps every non-zero level a normal bf16):
-// the bf16-rounded levels get the exponent added, then PRMT byte-plane
-// lookups decode the 8 codes.  Rounding commutes with a power-of-two scale in
+// PRMT byte-plane lookups of the bf16-rounded levels decode the 8 codes, then
+// one bf16x2 multiply per pair by the scale 2^e (an exact bf16; the products
+// are normal, so exact too).  Rounding commutes with a power-of-two scale in
 // the normal range, so this equals "fp32 multiply, then RNE to bf16" bit for
-// bit.  Otherwise (subnormal / overflowing results, scale byte 0xFF) every
-// weight takes the literal fp32 path.
+// bit.  Otherwise (subnormal / overflowing results, scale bytes 0 and 0xFF)
+// every weight takes the literal fp32 path.
 // ---------------------------------------------------------------------------
 struct DequantTable {
   uint32_t b[8];     // bf16 bits of each level (RNE)
   int emin, emax;    // exponent fields over non-zero levels
   int has_sub;       // a non-zero level that is a bf16 subnormal
+  Planes pl;         // byte planes of b[] for the PRMT lookup
 };
 
 constexpr int kDqWords = 4;
@@ -114,18 +116,11 @@ __device__ __forceinline__ void dequant_word(uint32_t cw, uint32_t s, const Dequ
                                              uint32_t res[4]) {
   const int e = (int)s - 127;
   // emin + e >= 2 keeps even the unrounded fp32 level times 2^e normal.
-  if (!d.has_sub && s != 255u && d.emin + e >= 2 && d.emax + e <= 254) {
-    uint32_t bb[8];
+  if (!d.has_sub && s != 0u && s != 255u && d.emin + e >= 2 && d.emax + e <= 254) {
+    decode8(cw, d.pl, res);
+    const uint32_t s2 = (s << 7) | (s << 23);  // 2^e in both bf16 halves
 #pragma unroll
-    for (int i = 0; i < 8; ++i) bb[i] = d.b[i] ? (uint32_t)((int)d.b[i] + e * 128) : 0u;
-    const uint32_t w01 = bb[0] | (bb[1] << 16), w23 = bb[2] | (bb[3] << 16);
-    const uint32_t w45 = bb[4] | (bb[5] << 16), w67 = bb[6] | (bb[7] << 16);
-    Planes p;
-    p.l0 = prmt(w01, w23, 0x6420);
-    p.h0 = prmt(w01, w23, 0x7531);
-    p.l1 = prmt(w45, w67, 0x6420);
-    p.h1 = prmt(w45, w67, 0x7531);
-    decode8(cw, p, res);
+    for (int i = 0; i < 4; ++i) res[i] = bf16x2_mul(res[i], s2);
   } else {
     const float mult = __uint_as_float(s == 0u ? 0x00400000u : (s << 23));
 #pragma unroll
@@ -158,12 +153,18 @@ __global__ void __launch_bounds__(256) dequant_kernel(const uint8_t* __restrict_
       const int ef = (d.b[i] >> 7) & 0xff;
       if (lv != 0.0f) {
         // a positive level whose bf16 is zero or subnormal cannot take the
-        // exponent-add path
+        // fast path
         if (ef == 0) d.has_sub = 1;
         d.emin = min(d.emin, ef);
         d.emax = max(d.emax, ef);
       }
     }
+    const uint32_t w01 = d.b[0] | (d.b[1] << 16), w23 = d.b[2] | (d.b[3] << 16);
+    const uint32_t w45 = d.b[4] | (d.b[5] << 16), w67 = d.b[6] | (d.b[7] << 16);
+    d.pl.l0 = prmt(w01, w23, 0x6420);
+    d.pl.h0 = prmt(w01, w23, 0x7531);
+    d.pl.l1 = prmt(w45, w67, 0x6420);
+    d.pl.h1 = prmt(w45, w67, 0x7531);
     st[threadIdx.x] = d;
   }
   __syncthreads();
