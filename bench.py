@@ -720,26 +720,46 @@ def measure_workload(q4, w, args, steps, warmup, world, dev, local, stream, flus
     kern_ms = np.array([[evs[i][j].elapsed_time(evs[i][j + 1]) for j in range(7)] for i in range(n_prof)])
     assert q4.forward_status(ws) == 0
 
-    # e2e through the host-buffer entry point (pinned host memory)
+    # e2e through the host-buffer entry points (pinned host memory): every
+    # step copies its x and logits host->device and its output device->host
+    # inside the timed region.  Throughput (the e2e value): the steps enqueued
+    # back to back with moe_q4_forward_host_async between one pair of events
+    # behind a device-side sleep, as the main timed loop (no flush: the
+    # rotating batches' weights exceed L2), the device status read once at
+    # the end.  Latency (e2e_sync): moe_q4_forward_host, which waits for its
+    # own work, one call at a time after an L2 flush.
     n_e2e = min(steps, 200)
     xh = [x.cpu().pin_memory() for x in xs]
     lh = [l.cpu().pin_memory() for l in lgs]
-    oh = torch.empty((T, sh.H), dtype=torch.bfloat16).pin_memory()
+    ohs = [torch.empty((T, sh.H), dtype=torch.bfloat16).pin_memory() for _ in range(ROTATE)]
     wsh = q4.alloc_workspace(q4.forward_host_workspace(layer, T, k))
     for i in range(3):
-        q4.forward_host(layer, xh[i % ROTATE], lh[i % ROTATE], k, oh, wsh)
-    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e)]
-    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_e2e)]
+        q4.forward_host(layer, xh[i % ROTATE], lh[i % ROTATE], k, ohs[0], wsh)
+    ta, tb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
     torch.cuda.synchronize()
+    torch.cuda._sleep(int(min(n_e2e, 2000) * 400_000))
+    ta.record(stream)
     for i in range(n_e2e):
+        q4.forward_host_async(layer, xh[i % ROTATE], lh[i % ROTATE], k, ohs[i % ROTATE], wsh)
+    tb.record(stream)
+    assert q4.forward_status(wsh) == 0
+    barrier()
+    e2e_ms = max_over_ranks(ta.elapsed_time(tb), dev)
+    e2e_value = job_tokens_per_s(T, n_e2e, world, e2e_ms)
+    n_sync = min(n_e2e, 100)
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(n_sync)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_sync)]
+    torch.cuda.synchronize()
+    for i in range(n_sync):
         flush_l2(i)
         e_s[i].record(stream)
-        st = q4.forward_host(layer, xh[i % ROTATE], lh[i % ROTATE], k, oh, wsh)
+        st = q4.forward_host(layer, xh[i % ROTATE], lh[i % ROTATE], k, ohs[0], wsh)
         e_e[i].record(stream)
         assert st == 0
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), dev)
-    e2e_value = job_tokens_per_s(T, n_e2e, world, e2e_ms)
+    e2e_sync_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), dev)
+    e2e_sync_value = job_tokens_per_s(T, n_sync, world, e2e_sync_ms)
     del wsh
 
     hbm_peak, tf_peak, peak_src = load_peaks()
@@ -774,7 +794,10 @@ def measure_workload(q4, w, args, steps, warmup, world, dev, local, stream, flus
                       "frac_of_peak": layer_bytes / (total_ms / steps / 1e3) / 1e9 / hbm_peak,
                       "frac_of_datasheet": layer_bytes / (total_ms / steps / 1e3) / 1e9 / DATASHEET_HBM_GBS},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": T * sh.H * 2 + T * sh.E * 4,
-                "d2h_bytes_per_step": T * sh.H * 2},
+                "d2h_bytes_per_step": T * sh.H * 2,
+                "api": "moe_q4_forward_host_async, steps back to back, status read at the end"},
+        "e2e_sync": {"value": e2e_sync_value, "unit": UNIT,
+                     "api": "moe_q4_forward_host (waits for each call), one call at a time after an L2 flush"},
         "enqueue_ms": enqueue_ms,
         "gpu_launches": kernels_per_step * steps,
         "clocks": clk.summary(),

@@ -89,7 +89,9 @@ def lib():
         L.moe_q4_lloyd_workspace.restype = sz
         L.moe_q4_lloyd_hist.argtypes = [vp, ctypes.c_longlong, vp, ci, vp, sz, vp]
         L.moe_q4_lloyd_solve.argtypes = [vp, ci, ctypes.c_double, vp, vp, vp, sz, vp]
+        L.moe_q4_forward_host_async.argtypes = L.moe_q4_forward_host.argtypes
         for f in (L.moe_q4_pack, L.moe_q4_dequant, L.moe_q4_forward, L.moe_q4_forward_host,
+                  L.moe_q4_forward_host_async,
                   L.moe_q4_forward_status, L.moe_q4_read_status, L.moe_q4_route,
                   L.moe_q4_forward_stages, L.moe_q4_router, L.moe_q4_lloyd_hist, L.moe_q4_lloyd_solve):
             f.restype = ci
@@ -317,6 +319,17 @@ def forward_host(layer: Layer, x_host: torch.Tensor, logits_host: torch.Tensor, 
     st = layer.struct()
     return int(lib().moe_q4_forward_host(ctypes.byref(st), _ptr(x_host), _ptr(logits_host), T, k,
                                          _ptr(out_host), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def forward_host_async(layer: Layer, x_host: torch.Tensor, logits_host: torch.Tensor, k: int,
+                       out_host: torch.Tensor, ws: torch.Tensor, stream=None) -> None:
+    """forward_host without the wait (pinned host tensors; read the device
+    status later with forward_status on the same stream)."""
+    T = x_host.shape[0]
+    st = layer.struct()
+    _check(lib().moe_q4_forward_host_async(ctypes.byref(st), _ptr(x_host), _ptr(logits_host), T, k,
+                                           _ptr(out_host), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_q4_forward_host_async")
 
 
 def route(logits: torch.Tensor, k: int, stream=None):

@@ -431,9 +431,9 @@ extern "C" int moe_q4_read_status(const int32_t* status, void* stream) {
   return rc != MOE_Q4_OK ? rc : (int)v;
 }
 
-extern "C" int moe_q4_forward_host(const moe_q4_layer* layer, const void* x_host,
-                                   const float* logits_host, int T, int top_k, void* out_host,
-                                   void* ws, size_t ws_bytes, void* stream) {
+extern "C" int moe_q4_forward_host_async(const moe_q4_layer* layer, const void* x_host,
+                                         const float* logits_host, int T, int top_k, void* out_host, void* ws,
+                                         size_t ws_bytes, void* stream) {
   if (!shape_ok(layer, T, top_k)) return MOE_Q4_EINVAL;
   TableParams tp;
   int rc = q4_fill_tables(&tp, layer->tables, layer->n_tables, layer->table_id, layer->E);
@@ -454,6 +454,14 @@ extern "C" int moe_q4_forward_host(const moe_q4_layer* layer, const void* x_host
                    nullptr, nullptr, nullptr, w, s);
   if (rc != MOE_Q4_OK) return rc;
   if (cudaMemcpyAsync(out_host, w + hs.out, xb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return MOE_Q4_ECUDA;
+  return MOE_Q4_OK;
+}
+
+extern "C" int moe_q4_forward_host(const moe_q4_layer* layer, const void* x_host,
+                                   const float* logits_host, int T, int top_k, void* out_host,
+                                   void* ws, size_t ws_bytes, void* stream) {
+  const int rc = moe_q4_forward_host_async(layer, x_host, logits_host, T, top_k, out_host, ws, ws_bytes, stream);
+  if (rc != MOE_Q4_OK || T == 0) return rc;
   return moe_q4_forward_status(ws, stream);
 }
 

@@ -291,6 +291,17 @@ MOE_Q4_API int moe_q4_forward_host(const moe_q4_layer* layer, const void* x_host
                         int T, int top_k, void* out_host, void* ws, size_t ws_bytes,
                         void* stream);
 
+/* moe_q4_forward_host without the wait: the copies in, the forward and the
+ * copy out are enqueued on `stream` and the call returns (MOE_Q4_OK or an
+ * argument / launch error).  x_host and logits_host are read, and out_host
+ * written, when the stream reaches the copies: with pinned memory the caller
+ * keeps them untouched until then (a later moe_q4_forward_status on the
+ * same stream waits for the work and returns its device status).  Calls
+ * enqueued back to back on one stream and workspace run in order. */
+MOE_Q4_API int moe_q4_forward_host_async(const moe_q4_layer* layer, const void* x_host, const float* logits_host,
+                                         int T, int top_k, void* out_host, void* ws, size_t ws_bytes,
+                                         void* stream);
+
 /* ---------------------------------------------------------------------------
  * moe_q4_route -- the routing and grouping steps of moe_q4_forward alone,
  * into caller buffers (all device, all required):

@@ -212,6 +212,27 @@ def test_forward_host_matches_device_forward():
     assert torch.equal(out_h, out_d.cpu())
 
 
+def test_forward_host_async_back_to_back_matches_device_forward():
+    """Several moe_q4_forward_host_async calls enqueued back to back on one
+    stream and workspace (different batches, different pinned outputs), the
+    status read once at the end: each output equals the device forward's."""
+    w = inputs.Workload("host_async", 20, 6, inputs.TINY)
+    _, dev = _small_device_layer(w)
+    xs = [inputs.activations(w, variant=v) for v in range(3)]
+    lgs = [inputs.router_logits(w, variant=v) for v in range(3)]
+    ws = q4.alloc_workspace(q4.forward_host_workspace(dev, 6, 2))
+    outs = [torch.empty((6, 256), dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    xp = [x.pin_memory() for x in xs]
+    lp = [l.pin_memory() for l in lgs]
+    for i in range(3):
+        q4.forward_host_async(dev, xp[i], lp[i], 2, outs[i], ws)
+    assert q4.forward_status(ws) == 0
+    for i in range(3):
+        ref = q4.forward(dev, xs[i].cuda(), lgs[i].cuda(), 2)
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i], ref.cpu()), i
+
+
 def test_non_finite_logit_reports_device_status():
     w = inputs.WORKLOADS["tiny"]
     _, dev = _small_device_layer(w)
