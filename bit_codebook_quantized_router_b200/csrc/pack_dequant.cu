@@ -110,7 +110,7 @@ struct DequantTable {
   Planes pl;         // byte planes of b[] for the PRMT lookup
 };
 
-constexpr int kDqWords = 4;
+constexpr int kDqWords = 8;
 
 __device__ __forceinline__ void dequant_word(uint32_t cw, uint32_t s, const DequantTable& d, const float* t,
                                              uint32_t res[4]) {
