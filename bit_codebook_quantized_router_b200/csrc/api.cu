@@ -58,14 +58,17 @@ bool shape_ok(const moe_q4_layer* L, int T, int top_k) {
 // Workspace layout, every array 256-byte aligned:
 //   header int32[64] | ids int32[T*k] | w f32[T*k] | counts int32[E] |
 //   offsets int32[E+1] | row_token int32[T*k] | inv int32[T*k] |
-//   dec_list int32[E] | pre_list int32[E] | mid_list int32[E] | tiles int32[E+1] | h bf16[T*k][I] |
+//   dec_list int32[E] | pre_list int32[E] | mid_list int32[E] | tiles int32[E+1] |
+//   chunk_cnt int32[chunks][E] | chunk_base int32[chunks][E] (256-token chunks
+//   of the grouping, T > 256 only) | h bf16[T*k][I] |
 //   h_lo bf16[T*k][I] | y f32[T*k][H] | xg bf16[T*k][H] (activation rows in
 //   expert order, T > 16 only) | split-tile counters int32[units] | partial sums of the
 //   small-M kernels f32[2*160][4][min(16,T)][128] (two 128-row tiles per unit,
 //   gate/up then down) | with a shared expert: h_s | y_s | its split partial
 //   sums | with the router gate in front: logits f32[T][E] | its partial sums
 struct Layout {
-  size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, mid_list, tiles, h, h_lo, y, xg,
+  size_t hdr, ids, w, counts, offsets, row_token, inv, dec_list, pre_list, mid_list, tiles, chunk_cnt,
+      chunk_base, h, h_lo, y, xg,
       dk_counter,
       dk_partial, h_s, y_s, sx_partial, logits, router_partial, end;
   int dk_units_gu, dk_units_dn, n_max;
@@ -104,6 +107,11 @@ Layout layout(const moe_q4_layer* L, int T, int k, const moe_q4_shared* S = null
   p = align_up(p + sizeof(int32_t) * L->E);
   o.tiles = p;
   p = align_up(p + sizeof(int32_t) * (L->E + 1));
+  const size_t chunk_words = (size_t)q4_route_chunks(T) * L->E;
+  o.chunk_cnt = p;
+  p = align_up(p + sizeof(int32_t) * chunk_words);
+  o.chunk_base = p;
+  p = align_up(p + sizeof(int32_t) * chunk_words);
   o.h = p;
   p = align_up(p + sizeof(__nv_bfloat16) * R * L->I);
   o.h_lo = p;
@@ -197,6 +205,8 @@ int run_forward(const moe_q4_layer* L, const TableParams& tp, const void* x, con
   const bool wide_ok = L->I % 256 == 0 && L->H % 256 == 0;
   a.wide_max = wide_ok ? q4_prefill_wide_max() : kDecodeMaxRows;
   a.tiles = (int32_t*)(ws + o.tiles);
+  a.chunk_cnt = (int32_t*)(ws + o.chunk_cnt);
+  a.chunk_base = (int32_t*)(ws + o.chunk_base);
   a.xg = o.xg ? (__nv_bfloat16*)(ws + o.xg) : nullptr;
   a.dk_counter = (int32_t*)(ws + o.dk_counter);
   a.dk_counter_n = (o.dk_units_gu + o.dk_units_dn) * kDkSlabs;
@@ -465,11 +475,17 @@ extern "C" int moe_q4_forward_host(const moe_q4_layer* layer, const void* x_host
   return moe_q4_forward_status(ws, stream);
 }
 
-// Routing-only workspace: header | dec_list[E] | pre_list[E].
+// Routing-only workspace: header | dec_list[E] | pre_list[E] | with T > 256:
+// chunk_cnt[chunks][E] | chunk_base[chunks][E].
+static size_t route_chunk_bytes(int E, int T) {
+  return align_up(sizeof(int32_t) * (size_t)q4_route_chunks(T) * E);
+}
+
 extern "C" size_t moe_q4_route_workspace(int E, int T, int top_k) {
   if (E < 1 || E > kMaxExperts || T < 0 || top_k < 1 || top_k > E || top_k > kMaxTopK) return 0;
   if ((long long)T * top_k > (1LL << 24)) return 0;
-  return align_up(sizeof(int32_t) * kHeaderWords) + 2 * align_up(sizeof(int32_t) * E);
+  return align_up(sizeof(int32_t) * kHeaderWords) + 2 * align_up(sizeof(int32_t) * E) +
+         2 * route_chunk_bytes(E, T);
 }
 
 extern "C" int moe_q4_route(const float* logits, int T, int E, int top_k, int32_t* ids, float* w,
@@ -492,6 +508,9 @@ extern "C" int moe_q4_route(const float* logits, int T, int E, int top_k, int32_
   a.hdr = (int32_t*)p;
   a.dec_list = (int32_t*)(p + align_up(sizeof(int32_t) * kHeaderWords));
   a.pre_list = (int32_t*)(p + align_up(sizeof(int32_t) * kHeaderWords) + align_up(sizeof(int32_t) * E));
+  const size_t chunks_at = align_up(sizeof(int32_t) * kHeaderWords) + 2 * align_up(sizeof(int32_t) * E);
+  a.chunk_cnt = (int32_t*)(p + chunks_at);
+  a.chunk_base = (int32_t*)(p + chunks_at + route_chunk_bytes(E, T));
   a.ids = ids;
   a.w = w;
   a.counts = counts;

@@ -32,6 +32,8 @@ struct FwdArgs {
   int32_t* pre_list;       // [E]
   int32_t* mid_list;       // [E] experts of the wide tensor-core kernel (nullptr: none)
   int32_t* tiles;          // [E+1] token-tile offsets of the tensor-core-path experts
+  int32_t* chunk_cnt;      // [chunks][E] rows per expert of each 256-token chunk (T > 256)
+  int32_t* chunk_base;     // [chunks][E] each chunk's first row inside each expert (T > 256)
   __nv_bfloat16* h;        // [T*k][I] bf16 rounding of silu(g)*u
   __nv_bfloat16* h_lo;     // [T*k][I] bf16 rounding of the remainder silu(g)*u - h
   float* y;                // [T*k][H]
@@ -55,6 +57,9 @@ int q4_fill_tables(q4::TableParams* tp, const float* tables, int n_tables, const
 
 // Kernel launchers (return MOE_Q4_OK or MOE_Q4_ECUDA).
 int q4_launch_route(const q4::FwdArgs& a, cudaStream_t s);
+// Chunks of the large-T grouping (0 for T <= 256): chunk_cnt and chunk_base
+// hold q4_route_chunks(T) * E int32 each.
+int q4_route_chunks(int T);
 int q4_launch_combine(const q4::FwdArgs& a, cudaStream_t s);
 // Router gate (router.cu): logits = x . w^T at any T (part: the partial sums,
 // q4_router_partial_bytes; status: the dense GEMM's status word), and at

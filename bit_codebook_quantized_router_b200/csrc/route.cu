@@ -16,8 +16,7 @@
 namespace q4 {
 
 constexpr int kRouteThreads = 1024;
-constexpr int kRouteWarps = kRouteThreads / 32;
-constexpr int kFusedMaxT = 256;  // above this, top-k runs on many CTAs first
+constexpr int kFusedMaxT = 256;  // above this, the chunked three-kernel grouping
 
 // Block-wide exclusive scan of one value per thread (kRouteThreads threads).
 __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& total) {
@@ -48,103 +47,6 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tot, int& t
   return res;
 }
 
-// Grouping by one CTA of kRouteThreads threads, ids already in a.ids.
-// Shared memory: counts[E] | offs[E+1] | running[E] | mask[32][E] | pre[32][E].
-__device__ void group_rows(const FwdArgs& a, int* sm) {
-  const int E = a.E, T = a.T, k = a.k;
-  int* counts = sm;
-  int* offs = counts + E;
-  int* running = offs + E + 1;
-  int* mask = running + E;
-  int* pre = mask + kRouteWarps * E;
-  __shared__ int warp_tot[33];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int e = tid; e < E; e += kRouteThreads) {
-    counts[e] = 0;
-    running[e] = 0;
-  }
-  // per-tile arrival counters of the small-M kernels start at zero every call
-  for (int i = tid; i < a.dk_counter_n; i += kRouteThreads) a.dk_counter[i] = 0;
-  __syncthreads();
-  // ids come from topk_warp and are always < E; a value out of range would be
-  // a library bug: record it and leave the row out rather than index past smem.
-  for (int r = tid; r < T * k; r += kRouteThreads) {
-    const int e = a.ids[r];
-    if ((unsigned)e < (unsigned)E)
-      atomicAdd(&counts[e], 1);
-    else
-      record_error(a.hdr + kStatus, MOE_Q4_EDEVICE);
-  }
-  __syncthreads();
-  // offsets and per-path expert lists (E <= kRouteThreads)
-  const int c = tid < E ? counts[tid] : 0;
-  int total;
-  const int off = block_exclusive_scan(c, warp_tot, total);
-  const int wmax = a.mid_list ? a.wide_max : a.dec_max;
-  const bool fd = c > 0 && c <= a.dec_max, fm = c > a.dec_max && c <= wmax, fp = c > wmax;
-  int nd, nm, np;
-  const int pd = block_exclusive_scan(fd ? 1 : 0, warp_tot, nd);
-  const int pm = block_exclusive_scan(fm ? 1 : 0, warp_tot, nm);
-  const int pp = block_exclusive_scan(fp ? 1 : 0, warp_tot, np);
-  // token tiles of each tensor-core-path expert, as an exclusive scan in
-  // pre_list order (tiles[p] .. tiles[p+1]-1 are expert pre_list[p]'s)
-  int ntot;
-  const int ntl = fp ? (c + a.tile_n - 1) / a.tile_n : 0;
-  const int ntoff = block_exclusive_scan(ntl, warp_tot, ntot);
-  if (tid < E) {
-    offs[tid] = off;
-    a.offsets[tid] = off;
-    a.counts[tid] = c;
-    if (a.user_counts) a.user_counts[tid] = c;
-    if (fd) a.dec_list[pd] = tid;
-    if (fm) a.mid_list[pm] = tid;
-    if (fp) a.pre_list[pp] = tid;
-    if (fp && a.tiles) a.tiles[pp] = ntoff;
-  }
-  if (tid == 0) {
-    offs[E] = total;
-    a.offsets[E] = total;
-    a.hdr[kNumDecode] = nd;
-    a.hdr[kNumMid] = nm;
-    a.hdr[kNumPrefill] = np;
-    a.hdr[kNumTiles] = ntot;
-    if (a.tiles) a.tiles[np] = ntot;
-  }
-  __syncthreads();
-  // stable placement, kRouteThreads tokens per round
-  for (int base = 0; base < T; base += kRouteThreads) {
-    for (int i = tid; i < kRouteWarps * E; i += kRouteThreads) mask[i] = 0;
-    __syncthreads();
-    const int t = base + tid;
-    if (t < T)
-      for (int j = 0; j < k; ++j) {
-        const int e = a.ids[t * k + j];
-        if ((unsigned)e < (unsigned)E) atomicOr(&mask[warp * E + e], 1 << lane);
-      }
-    __syncthreads();
-    for (int e = tid; e < E; e += kRouteThreads) {
-      int acc = running[e];
-      for (int w2 = 0; w2 < kRouteWarps; ++w2) {
-        pre[w2 * E + e] = acc;
-        acc += __popc(mask[w2 * E + e]);
-      }
-      running[e] = acc;
-    }
-    __syncthreads();
-    if (t < T) {
-      const uint32_t below = (1u << lane) - 1u;
-      for (int j = 0; j < k; ++j) {
-        const int e = a.ids[t * k + j];
-        if ((unsigned)e >= (unsigned)E) continue;
-        const int pos = offs[e] + pre[warp * E + e] + __popc(mask[warp * E + e] & below);
-        a.row_token[pos] = t;
-        a.inv[t * k + j] = pos;
-      }
-    }
-    __syncthreads();
-  }
-}
-
 // Small T (<= kFusedMaxT): one CTA routes every token and groups
 // (route_small, ids kept in shared memory).
 __global__ void __launch_bounds__(kRouteThreads) route_fused_kernel(const __grid_constant__ FwdArgs a) {
@@ -157,8 +59,21 @@ __global__ void __launch_bounds__(kRouteThreads) route_fused_kernel(const __grid
   route_small<kRouteThreads, false>(a, sm);
 }
 
-// Large T: top-k on many CTAs (one warp per token; the host clears the
-// status word before this launch) ...
+// Large T: chunks of kChunkT tokens.
+// (1) route_topk_kernel, one warp per token (8 tokens per CTA, the host clears
+//     the status word and chunk_cnt before it): top-k of each token, and each
+//     chosen expert's row count in the token's chunk (global atomics);
+// (2) route_scan_kernel, one CTA: each expert's rows over all chunks, the
+//     exclusive-scan offsets, the per-path expert lists and tile offsets, and
+//     every chunk's first row inside each expert (the rows of earlier chunks
+//     come first: token order is row order within an expert);
+// (3) route_place_kernel, one CTA per chunk: a row's place is its chunk's
+//     base for the expert plus the number of earlier tokens of the chunk that
+//     chose the expert (per-expert token bitmasks, as route_small).
+// Every result is an integer: the same as one CTA grouping all rows.
+constexpr int kChunkT = 256;
+constexpr int kChunkThreads = 256;
+
 __global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__ FwdArgs a) {
   pdl_trigger();  // scheduling only: the next kernel's wait covers this one
   pdl_wait();
@@ -169,15 +84,97 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const __grid_constant__
     float w;
     topk_warp(a.logits + (size_t)t * a.E, a.E, a.k, lane, a.hdr + kStatus, id, w);
     store_route(a, t, lane, id, w);
+    if (lane < a.k) {
+      // ids come from topk_warp and are always < E; a value out of range
+      // would be a library bug: record it and leave the row out
+      if ((unsigned)id < (unsigned)a.E)
+        atomicAdd(a.chunk_cnt + (size_t)(t / kChunkT) * a.E + id, 1);
+      else
+        record_error(a.hdr + kStatus, MOE_Q4_EDEVICE);
+    }
   }
 }
 
-// ... then one CTA groups.
-__global__ void __launch_bounds__(kRouteThreads) route_group_kernel(const __grid_constant__ FwdArgs a) {
-  extern __shared__ int sm[];
+__global__ void __launch_bounds__(kRouteThreads) route_scan_kernel(const __grid_constant__ FwdArgs a,
+                                                                    int n_chunks) {
+  __shared__ int warp_tot[33];
   pdl_trigger();  // scheduling only: the next kernel's wait covers this one
   pdl_wait();
-  group_rows(a, sm);
+  const int E = a.E, tid = threadIdx.x;
+  // per-tile arrival counters of the small-M kernels start at zero every call
+  for (int i = tid; i < a.dk_counter_n; i += kRouteThreads) a.dk_counter[i] = 0;
+  int c = 0;
+  if (tid < E) {
+#pragma unroll 4
+    for (int ch = 0; ch < n_chunks; ++ch) c += a.chunk_cnt[(size_t)ch * E + tid];
+  }
+  // offsets and per-path expert lists (E <= kRouteThreads)
+  int total;
+  const int off = block_exclusive_scan(c, warp_tot, total);
+  const int wmax = a.mid_list ? a.wide_max : a.dec_max;
+  const bool fd = c > 0 && c <= a.dec_max, fm = c > a.dec_max && c <= wmax, fp = c > wmax;
+  int nd, nm, np;
+  const int pd = block_exclusive_scan(fd ? 1 : 0, warp_tot, nd);
+  const int pm = block_exclusive_scan(fm ? 1 : 0, warp_tot, nm);
+  const int pp = block_exclusive_scan(fp ? 1 : 0, warp_tot, np);
+  // token tiles of each swap-AB expert, as an exclusive scan in pre_list order
+  int ntot;
+  const int ntl = fp ? (c + a.tile_n - 1) / a.tile_n : 0;
+  const int ntoff = block_exclusive_scan(ntl, warp_tot, ntot);
+  if (tid < E) {
+    a.offsets[tid] = off;
+    a.counts[tid] = c;
+    if (a.user_counts) a.user_counts[tid] = c;
+    if (fd) a.dec_list[pd] = tid;
+    if (fm) a.mid_list[pm] = tid;
+    if (fp) a.pre_list[pp] = tid;
+    if (fp && a.tiles) a.tiles[pp] = ntoff;
+    // each chunk's first row inside this expert
+    int run = off;
+    for (int ch = 0; ch < n_chunks; ++ch) {
+      const size_t i = (size_t)ch * E + tid;
+      const int n = a.chunk_cnt[i];
+      a.chunk_base[i] = run;
+      run += n;
+    }
+  }
+  if (tid == 0) {
+    a.offsets[E] = total;
+    a.hdr[kNumDecode] = nd;
+    a.hdr[kNumMid] = nm;
+    a.hdr[kNumPrefill] = np;
+    a.hdr[kNumTiles] = ntot;
+    if (a.tiles) a.tiles[np] = ntot;
+  }
+}
+
+__global__ void __launch_bounds__(kChunkThreads) route_place_kernel(const __grid_constant__ FwdArgs a) {
+  extern __shared__ uint32_t tokmask[];  // [E][kChunkT / 32]
+  constexpr int W = kChunkT / 32;
+  pdl_trigger();  // scheduling only: the next kernel's wait covers this one
+  pdl_wait();
+  const int E = a.E, k = a.k;
+  const int t0 = blockIdx.x * kChunkT, t1 = t0 + kChunkT < a.T ? t0 + kChunkT : a.T;
+  const int n_rows = (t1 - t0) * k;
+  for (int i = threadIdx.x; i < E * W; i += kChunkThreads) tokmask[i] = 0u;
+  __syncthreads();
+  for (int r = threadIdx.x; r < n_rows; r += kChunkThreads) {
+    const int lt = r / k, e = a.ids[(size_t)t0 * k + r];
+    if ((unsigned)e < (unsigned)E) atomicOr(&tokmask[e * W + (lt >> 5)], 1u << (lt & 31));
+  }
+  __syncthreads();
+  const int32_t* base = a.chunk_base + (size_t)blockIdx.x * E;
+  for (int r = threadIdx.x; r < n_rows; r += kChunkThreads) {
+    const int lt = r / k, e = a.ids[(size_t)t0 * k + r];
+    if ((unsigned)e >= (unsigned)E) continue;
+    const uint32_t* m = tokmask + e * W;
+    int rank = __popc(m[lt >> 5] & ((1u << (lt & 31)) - 1u));
+    for (int q = 0; q < (lt >> 5); ++q) rank += __popc(m[q]);
+    const int pos = base[e] + rank;
+    if (!q4_check((unsigned)pos < (unsigned)(a.T * k), a.hdr + kStatus)) continue;
+    a.row_token[pos] = t0 + lt;
+    a.inv[(size_t)t0 * k + r] = pos;
+  }
 }
 
 // Gather the activation rows in expert-grouped order for the tensor-core
@@ -201,10 +198,9 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant_
 
 using namespace q4;
 
-static size_t group_smem_bytes(int E) { return sizeof(int) * ((size_t)3 * E + 1 + (size_t)2 * kRouteWarps * E); }
+int q4_route_chunks(int T) { return T > kFusedMaxT ? (T + kChunkT - 1) / kChunkT : 0; }
 
 int q4_launch_route(const FwdArgs& a, cudaStream_t s) {
-  const size_t smem = a.T <= kFusedMaxT ? route_small_smem_bytes(a.E, a.T, a.k) : group_smem_bytes(a.E);
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
@@ -213,29 +209,33 @@ int q4_launch_route(const FwdArgs& a, cudaStream_t s) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (a.T <= kFusedMaxT) {
+    const size_t smem = route_small_smem_bytes(a.E, a.T, a.k);
     if (cudaFuncSetAttribute(route_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return MOE_Q4_ECUDA;
     cfg.gridDim = dim3(1);
     cfg.blockDim = dim3(kRouteThreads);
     cfg.dynamicSmemBytes = smem;
-    if (cudaLaunchKernelEx(&cfg, route_fused_kernel, a) != cudaSuccess) return MOE_Q4_ECUDA;
-  } else {
-    if (cudaFuncSetAttribute(route_group_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-      return MOE_Q4_ECUDA;
-    if (!a.keep_status && cudaMemsetAsync(a.hdr + kStatus, 0, sizeof(int32_t), s) != cudaSuccess)
-      return MOE_Q4_ECUDA;
-    cfg.gridDim = dim3((a.T + 7) / 8);
-    cfg.blockDim = dim3(256);
-    cfg.dynamicSmemBytes = 0;
-    if (cudaLaunchKernelEx(&cfg, route_topk_kernel, a) != cudaSuccess) return MOE_Q4_ECUDA;
-    cfg.gridDim = dim3(1);
-    cfg.blockDim = dim3(kRouteThreads);
-    cfg.dynamicSmemBytes = smem;
-    if (cudaLaunchKernelEx(&cfg, route_group_kernel, a) != cudaSuccess) return MOE_Q4_ECUDA;
+    return cudaLaunchKernelEx(&cfg, route_fused_kernel, a) == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
   }
-  return MOE_Q4_OK;
+  if (!a.chunk_cnt || !a.chunk_base) return MOE_Q4_ECUDA;
+  if (!a.keep_status && cudaMemsetAsync(a.hdr + kStatus, 0, sizeof(int32_t), s) != cudaSuccess)
+    return MOE_Q4_ECUDA;
+  const int n_chunks = q4_route_chunks(a.T);
+  if (cudaMemsetAsync(a.chunk_cnt, 0, sizeof(int32_t) * (size_t)n_chunks * a.E, s) != cudaSuccess)
+    return MOE_Q4_ECUDA;
+  cfg.gridDim = dim3((a.T + 7) / 8);
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  if (cudaLaunchKernelEx(&cfg, route_topk_kernel, a) != cudaSuccess) return MOE_Q4_ECUDA;
+  cfg.gridDim = dim3(1);
+  cfg.blockDim = dim3(kRouteThreads);
+  cfg.dynamicSmemBytes = 0;
+  if (cudaLaunchKernelEx(&cfg, route_scan_kernel, a, n_chunks) != cudaSuccess) return MOE_Q4_ECUDA;
+  cfg.gridDim = dim3(n_chunks);
+  cfg.blockDim = dim3(kChunkThreads);
+  cfg.dynamicSmemBytes = sizeof(uint32_t) * (size_t)a.E * (kChunkT / 32);
+  return cudaLaunchKernelEx(&cfg, route_place_kernel, a) == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
 }
 
 int q4_launch_gather(const FwdArgs& a, cudaStream_t s) {

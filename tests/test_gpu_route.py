@@ -34,7 +34,7 @@ def test_route_glm_shapes(T):
 @pytest.mark.parametrize("E,k", [(8, 1), (8, 2), (3, 3), (512, 16), (33, 5), (1, 1)])
 def test_route_other_shapes(E, k):
     rng = np.random.default_rng(E * 7 + k)
-    for T in (1, 37, 300):
+    for T in (1, 37, 300, 1500):
         _check(rng.standard_normal((T, E)).astype(np.float32), k)
 
 
