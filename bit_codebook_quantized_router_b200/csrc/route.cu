@@ -179,18 +179,25 @@ __global__ void __launch_bounds__(kChunkThreads) route_place_kernel(const __grid
 
 // Gather the activation rows in expert-grouped order for the tensor-core
 // GEMMs (both paths read activations by TMA from contiguous rows):
-// xg[row] = x[row_token[row]] for all T*k rows.
+// xg[row] = x[row_token[row]] for all T*k rows, taken token by token: each
+// 16-byte vector of x[t] is read once and stored to the k grouped rows
+// inv[t][0..k-1] (a row-ordered gather would read every x row k times).
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __grid_constant__ FwdArgs a) {
   pdl_trigger();  // scheduling only: the next kernel's wait covers this one
   pdl_wait();
   const int vec_per_row = a.H / 8;  // 16-byte vectors
-  const int64_t n = (int64_t)a.T * a.k * vec_per_row;
+  const int k = a.k, R = a.T * a.k;
+  const int64_t n = (int64_t)a.T * vec_per_row;
+  const uint4* x = reinterpret_cast<const uint4*>(a.x);
+  uint4* xg = reinterpret_cast<uint4*>(a.xg);
   for (int64_t v = blockIdx.x * 256 + threadIdx.x; v < n; v += (int64_t)gridDim.x * 256) {
-    const int r = (int)(v / vec_per_row);
+    const int t = (int)(v / vec_per_row);
     const int q = (int)(v % vec_per_row);
-    if (!q4_check((unsigned)a.row_token[r] < (unsigned)a.T, a.hdr + kStatus)) continue;
-    const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)a.row_token[r] * a.H) + q;
-    reinterpret_cast<uint4*>(a.xg + (size_t)r * a.H)[q] = *src;
+    const uint4 val = x[v];
+    for (int j = 0; j < k; ++j) {
+      const int pos = a.inv[t * k + j];
+      if (q4_check((unsigned)pos < (unsigned)R, a.hdr + kStatus)) xg[(size_t)pos * vec_per_row + q] = val;
+    }
   }
 }
 
@@ -246,7 +253,7 @@ int q4_launch_gather(const FwdArgs& a, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const long long vecs = (long long)a.T * a.k * (a.H / 8);
+  const long long vecs = (long long)a.T * (a.H / 8);
   const long long blocks = (vecs + 255) / 256;
   cfg.gridDim = dim3((unsigned)(blocks < 148 * 8 ? blocks : 148 * 8));
   cfg.blockDim = dim3(256);
