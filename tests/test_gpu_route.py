@@ -38,6 +38,16 @@ def test_route_other_shapes(E, k):
         _check(rng.standard_normal((T, E)).astype(np.float32), k)
 
 
+@pytest.mark.parametrize("T,E,k", [(65536, 256, 8), (40001, 512, 16)])
+def test_route_many_chunks(T, E, k):
+    # hundreds of 256-token chunks (the last one ragged) in the large-batch
+    # grouping, with a skew so that some experts hold rows in every chunk
+    rng = np.random.default_rng(T + E)
+    lg = rng.standard_normal((T, E)).astype(np.float32)
+    lg[:, : E // 16] += 1.5
+    _check(lg, k)
+
+
 def test_route_ties_and_signed_zeros():
     rng = np.random.default_rng(3)
     lg = (np.round(rng.standard_normal((500, 64)) * 2) / 2).astype(np.float32)  # many exact ties
