@@ -94,6 +94,13 @@ def test_route_workspace_validation(L):
     assert L.moe_q4_route_workspace(256, 8, 8) > 0
     assert L.moe_q4_route_workspace(256, 8, 17) == 0
     assert L.moe_q4_route_workspace(600, 8, 8) == 0
+    # past 256 tokens the grouping keeps each 256-token chunk's row counts and
+    # first rows: two int32 [ceil(T/256)][E] arrays, 256-byte aligned
+    base = L.moe_q4_route_workspace(256, 256, 8)
+    assert L.moe_q4_route_workspace(256, 1, 8) == base
+    assert L.moe_q4_route_workspace(256, 257, 8) == base + 2 * (2 * 256 * 4)
+    assert L.moe_q4_route_workspace(256, 8192, 8) == base + 2 * (32 * 256 * 4)
+    assert L.moe_q4_route_workspace(3, 300, 3) == L.moe_q4_route_workspace(3, 8, 3) + 2 * 256
 
 
 def test_router_workspace_and_argument_validation(L):
