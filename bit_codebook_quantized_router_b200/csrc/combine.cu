@@ -13,39 +13,81 @@
 
 namespace q4 {
 
+// BATCH (few tokens, where the combine is latency-bound): the slots are taken
+// kCombineSlots per round, their row indices and weights loaded first and
+// every y load of the round issued before the first one is used, so a thread
+// waits for one round trip per round instead of two per slot.  Without BATCH
+// (many tokens, bandwidth-bound) one slot at a time in fewer registers, so
+// more CTAs stay resident.  Both add the same products in the same order.
+constexpr int kCombineSlots = 8;
+constexpr int kCombineBatchMaxT = 64;
+
+template <bool BATCH>
 __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ FwdArgs a) {
   pdl_wait();
   pdl_trigger();
   const int n4 = (blockIdx.x * 256 + threadIdx.x) * 4;
   if (n4 >= a.H) return;
+  const int k = a.k, R = a.T * a.k;
+  int32_t* status = a.hdr ? a.hdr + kStatus : nullptr;
   for (int t = blockIdx.y; t < a.T; t += gridDim.y) {
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int j = 0; j < a.k; ++j) {
-    // (no inverse map: the rows are in (token, slot) order)
-    const int r = a.inv ? a.inv[t * a.k + j] : t * a.k + j;
-    const float wj = a.w[t * a.k + j];
-    if (!q4_check((unsigned)r < (unsigned)(a.T * a.k), a.hdr ? a.hdr + kStatus : nullptr)) continue;
-    const float4 v = *reinterpret_cast<const float4*>(a.y + (size_t)r * a.H + n4);
-    acc.x = fmaf(wj, v.x, acc.x);
-    acc.y = fmaf(wj, v.y, acc.y);
-    acc.z = fmaf(wj, v.z, acc.z);
-    acc.w = fmaf(wj, v.w, acc.w);
-  }
-  if (a.y_s) {
-    // the shared expert's output, weight 1, after the routed slots
-    const float4 v = *reinterpret_cast<const float4*>(a.y_s + (size_t)t * a.H + n4);
-    acc.x += v.x;
-    acc.y += v.y;
-    acc.z += v.z;
-    acc.w += v.w;
-  }
-  if (a.out_f32) *reinterpret_cast<float4*>(a.out_f32 + (size_t)t * a.H + n4) = acc;
-  __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-  uint2 pk;
-  pk.x = *reinterpret_cast<uint32_t*>(&lo);
-  pk.y = *reinterpret_cast<uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(a.out + (size_t)t * a.H + n4) = pk;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!BATCH) {
+      for (int j = 0; j < k; ++j) {
+        // (no inverse map: the rows are in (token, slot) order)
+        const int r = a.inv ? a.inv[t * k + j] : t * k + j;
+        const float wj = a.w[t * k + j];
+        if (!q4_check((unsigned)r < (unsigned)R, status)) continue;
+        const float4 v = *reinterpret_cast<const float4*>(a.y + (size_t)r * a.H + n4);
+        acc.x = fmaf(wj, v.x, acc.x);
+        acc.y = fmaf(wj, v.y, acc.y);
+        acc.z = fmaf(wj, v.z, acc.z);
+        acc.w = fmaf(wj, v.w, acc.w);
+      }
+    }
+    for (int j0 = 0; BATCH && j0 < k; j0 += kCombineSlots) {
+      int r[kCombineSlots];
+      float wj[kCombineSlots];
+#pragma unroll
+      for (int u = 0; u < kCombineSlots; ++u) {
+        const int j = j0 + u < k ? j0 + u : k - 1;
+        // (no inverse map: the rows are in (token, slot) order)
+        r[u] = a.inv ? a.inv[t * k + j] : t * k + j;
+        wj[u] = a.w[t * k + j];
+      }
+      bool ok[kCombineSlots];
+#pragma unroll
+      for (int u = 0; u < kCombineSlots; ++u)
+        ok[u] = j0 + u < k && q4_check((unsigned)r[u] < (unsigned)R, status);
+      float4 v[kCombineSlots];
+#pragma unroll
+      for (int u = 0; u < kCombineSlots; ++u)
+        if (ok[u]) v[u] = *reinterpret_cast<const float4*>(a.y + (size_t)r[u] * a.H + n4);
+      // slot order, one fmaf per slot: the same sum as taking the slots one by one
+#pragma unroll
+      for (int u = 0; u < kCombineSlots; ++u)
+        if (ok[u]) {
+          acc.x = fmaf(wj[u], v[u].x, acc.x);
+          acc.y = fmaf(wj[u], v[u].y, acc.y);
+          acc.z = fmaf(wj[u], v[u].z, acc.z);
+          acc.w = fmaf(wj[u], v[u].w, acc.w);
+        }
+    }
+    if (a.y_s) {
+      // the shared expert's output, weight 1, after the routed slots
+      const float4 v = *reinterpret_cast<const float4*>(a.y_s + (size_t)t * a.H + n4);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    if (a.out_f32) *reinterpret_cast<float4*>(a.out_f32 + (size_t)t * a.H + n4) = acc;
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(a.out + (size_t)t * a.H + n4) = pk;
   }
 }
 
@@ -64,7 +106,9 @@ int q4_launch_combine(const FwdArgs& a, cudaStream_t s) {
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, combine_kernel, a) == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
+  const cudaError_t e = a.T <= kCombineBatchMaxT ? cudaLaunchKernelEx(&cfg, combine_kernel<true>, a)
+                                                 : cudaLaunchKernelEx(&cfg, combine_kernel<false>, a);
+  return e == cudaSuccess ? MOE_Q4_OK : MOE_Q4_ECUDA;
 }
 
 // The combine alone: y fp32 [T*k][H] (rows in (token, slot) order, or placed

@@ -16,10 +16,14 @@ from tests.test_gpu_forward import _small_device_layer
 pytestmark = pytest.mark.gpu
 
 
+@pytest.mark.parametrize("T", [37, 300])
+@pytest.mark.parametrize("k", [1, 5, 8, 11, 16])
 @pytest.mark.parametrize("with_inv", [False, True])
-def test_combine_alone(with_inv):
-    g = torch.Generator(device="cuda").manual_seed(3)
-    T, k, H = 37, 5, 384
+def test_combine_alone(with_inv, k, T):
+    # up to 64 tokens the kernel takes the slots eight at a time: k below, at,
+    # between and at twice that round; above 64 tokens one slot at a time
+    g = torch.Generator(device="cuda").manual_seed(3 + k + T)
+    H = 384
     y = torch.randn((T * k, H), generator=g, device="cuda")
     w = torch.rand((T, k), generator=g, device="cuda")
     inv = None
