@@ -1,4 +1,4 @@
-"""Expert parallelism on CPU: the dispatch plan, and two gloo ranks running
+"""Expert parallelism on CPU: the dispatch plan, and two or three gloo ranks running
 the expert-parallel layer (whole experts per rank, "Round 7", "Owner-locked
 decisions" item 11) with the fp64 oracle as every rank's expert computation;
 the result must equal the single-process oracle layer over all tokens."""
@@ -41,17 +41,16 @@ def test_plan_orders_rows_by_owner_then_expert_then_token():
 
 
 TINY = inputs.WORKLOADS["tiny"]
-TOKENS = (5, 3)  # tokens held by rank 0 and rank 1
 
 
-def _global_inputs():
-    T = sum(TOKENS)
+def _global_inputs(tokens):
+    T = sum(tokens)
     x = inputs.bf16_bits(inputs.activations(TINY, T=T, variant=2))
     lg = inputs.router_logits(TINY, T=T, variant=2).numpy()
     return x, lg
 
 
-def _rank(rank, world, port, q):
+def _rank(rank, world, tokens, port, q):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     import torch.distributed as dist
@@ -59,9 +58,9 @@ def _rank(rank, world, port, q):
     try:
         L, _, _ = helpers.build_layer_host(TINY)
         E, k = TINY.shape.E, TINY.shape.k
-        x, lg = _global_inputs()
-        t0 = sum(TOKENS[:rank])
-        xr, lgr = x[t0:t0 + TOKENS[rank]], lg[t0:t0 + TOKENS[rank]]
+        x, lg = _global_inputs(tokens)
+        t0 = sum(tokens[:rank])
+        xr, lgr = x[t0:t0 + tokens[rank]], lg[t0:t0 + tokens[rank]]
         ids, w = oracle.route(lgr, k)
         a, b = ep.expert_ranges(E, world)[rank]
         shard = oracle.Layer(b - a, L.H, L.I, L.tables, L.table_id[a:b])
@@ -88,11 +87,15 @@ def _rank(rank, world, port, q):
         dist.destroy_process_group()
 
 
-def test_two_gloo_ranks_equal_the_single_process_layer():
+# tokens held by each rank: two ranks with 4 experts each; three ranks with
+# 3, 3 and 2 experts, one of them holding no tokens
+@pytest.mark.parametrize("tokens", [(5, 3), (4, 0, 6)])
+def test_gloo_ranks_equal_the_single_process_layer(tokens):
+    world = len(tokens)
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = 29600 + os.getpid() % 300
-    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    port = 29600 + (os.getpid() + 7 * world) % 300
+    procs = [ctx.Process(target=_rank, args=(r, world, tokens, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = dict(q.get(timeout=120) for _ in procs)
@@ -100,7 +103,7 @@ def test_two_gloo_ranks_equal_the_single_process_layer():
         p.join(timeout=60)
         assert p.exitcode == 0
     L, _, _ = helpers.build_layer_host(TINY)
-    x, lg = _global_inputs()
+    x, lg = _global_inputs(tokens)
     ref = oracle.moe_tokens(L, x, lg, TINY.shape.k)
-    got = np.concatenate([res[0], res[1]])
+    got = np.concatenate([res[r] for r in range(world)])
     np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-14 * np.abs(ref).max())
