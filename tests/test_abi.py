@@ -188,3 +188,12 @@ def test_debug_build_exports_every_declared_symbol(L):
         assert hasattr(D, s), s
     D.moe_q4_status_string.restype = ctypes.c_char_p
     assert b"debug" in D.moe_q4_status_string(_lib.EBOUNDS)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    # no CPU fallback: without the built library every entry raises
+    from bit_codebook_quantized_router_b200 import _lib as binding
+    monkeypatch.setattr(binding, "_lib", None)
+    monkeypatch.setattr(binding, "LIB_PATH", str(tmp_path / "libmoe_q4.so"))
+    with pytest.raises(ImportError, match="is missing"):
+        binding.lib()
